@@ -1,0 +1,15 @@
+"""CPU fp64 oracle for block-sparse top-k attention (pool -> score -> top-k -> attention).
+
+TEST INFRASTRUCTURE ONLY.  Only `tests/`, `__graft_entry__.smoke()` and `bench.py`'s
+CPU-baseline / reference leg may import this package.  The product path (the CUDA
+library and its Python binding) never imports, calls or falls back to it.
+
+It shares no code with the CUDA path: it is plain numpy in float64, written step by
+step from the method's definition (see `msa_oracle.py` for the citations), slow on
+purpose, and checked against pins that come from outside itself (tests/test_oracle_*).
+"""
+from .msa_oracle import (  # noqa: F401
+    pool_keys, group_query_sum, prefill_block_scores, select_prefill_row,
+    select_decode_row, attend_row, prefill_rows, decode_rows, PrefillRow, DecodeRow,
+    rel_gap, prefill_keys_of, decode_keys_of,
+)
