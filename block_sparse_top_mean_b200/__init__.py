@@ -1,0 +1,182 @@
+"""B200 (sm_100a) block-sparse top-k attention: pool -> score -> top-k -> sparse attention.
+
+Thin PyTorch-facing binding of the C ABI in include/msa.h.  These functions only
+marshal arguments (shapes, pointers, the current CUDA stream) and allocate outputs
+and workspaces with torch; every step of the computation runs in the library's CUDA
+kernels.  There is no CPU path: tensors must be CUDA tensors and the library must be
+built (`python -m block_sparse_top_mean_b200.build`).
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _lib
+from ._lib import (  # noqa: F401
+    MsaError, MsaParams, OP_DECODE, OP_PREFILL, OP_SPARSE_ATTN, OP_TOPK_SELECT,
+    DEVERR_IDX_RANGE, DEVERR_TIMEOUT, MSA_F32, MSA_BF16,
+)
+
+__all__ = [
+    "params", "workspace", "pool_keys", "block_scores", "topk_select", "sparse_attn_fwd",
+    "prefill_fwd", "decode_fwd", "read_device_error", "clear_device_error", "version",
+    "MsaError", "MsaParams",
+]
+
+_DT = {torch.float32: MSA_F32, torch.bfloat16: MSA_BF16}
+
+
+def version() -> str:
+    return _lib.load().msa_version().decode()
+
+
+def params(*, batch, seq, hq, hkv, d, block, topk, scale, dtype) -> MsaParams:
+    dt = _DT[dtype] if isinstance(dtype, torch.dtype) else int(dtype)
+    return MsaParams(int(batch), int(seq), int(hq), int(hkv), int(d), int(block), int(topk),
+                     float(scale), dt)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("block_sparse_top_mean_b200 takes CUDA tensors only")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def workspace(p: MsaParams, op: int, n_query: int = 0, device="cuda") -> torch.Tensor:
+    """A workspace for `op` (uint8 CUDA tensor, 256-byte aligned by the caching
+    allocator), with the device error word cleared."""
+    n = _lib.load().msa_workspace_bytes(ctypes.byref(p), op, n_query)
+    if n == 0:
+        raise MsaError("msa_workspace_bytes", _lib.MSA_ERR_INVALID_ARG, "invalid shapes")
+    ws = torch.empty(n, dtype=torch.uint8, device=device)
+    ws[:256].zero_()
+    return ws
+
+
+def _prefill_params(q, k, block, topk, scale):
+    b, S, hq, d = q.shape
+    hkv = k.shape[2]
+    return params(batch=b, seq=S, hq=hq, hkv=hkv, d=d, block=block, topk=topk,
+                  scale=scale if scale is not None else d ** -0.5, dtype=q.dtype)
+
+
+def pool_keys(k: torch.Tensor, block: int, split: bool = False):
+    """k [b, S, hkv, d] -> kbar fp32 [b, nb, hkv, d] (and bf16 hi/lo planes if split)."""
+    b, S, hkv, d = k.shape
+    p = params(batch=b, seq=S, hq=hkv, hkv=hkv, d=d, block=block, topk=1, scale=1.0,
+               dtype=k.dtype)
+    nb = -(-S // block)
+    kbar = torch.empty(b, nb, hkv, d, dtype=torch.float32, device=k.device)
+    hi = lo = None
+    if split:
+        hi = torch.empty(b, nb, hkv, d, dtype=torch.bfloat16, device=k.device)
+        lo = torch.empty_like(hi)
+    _lib.check("msa_pool_keys", _lib.load().msa_pool_keys(
+        ctypes.byref(p), _ptr(k), _ptr(kbar), _ptr(hi), _ptr(lo), _stream(k.device)))
+    return (kbar, hi, lo) if split else kbar
+
+
+def block_scores(q: torch.Tensor, kbar: torch.Tensor, block: int, hkv: int) -> torch.Tensor:
+    """Materialised causal block scores [b, hkv, S, nb] (small shapes only)."""
+    b, S, hq, d = q.shape
+    p = params(batch=b, seq=S, hq=hq, hkv=hkv, d=d, block=block, topk=1, scale=1.0,
+               dtype=q.dtype)
+    nb = -(-S // block)
+    out = torch.empty(b, hkv, S, nb, dtype=torch.float32, device=q.device)
+    _lib.check("msa_block_scores", _lib.load().msa_block_scores(
+        ctypes.byref(p), _ptr(q), _ptr(kbar), _ptr(out), _stream(q.device)))
+    return out
+
+
+def topk_select(q, kbar, block: int, topk: int, hkv: int, kbar_hi=None, kbar_lo=None, ws=None):
+    """Causal selection idx [b, hkv, S, topk] (int32, ascending, -1 padded)."""
+    b, S, hq, d = q.shape
+    p = params(batch=b, seq=S, hq=hq, hkv=hkv, d=d, block=block, topk=topk, scale=1.0,
+               dtype=q.dtype)
+    idx = torch.empty(b, hkv, S, topk, dtype=torch.int32, device=q.device)
+    if ws is None:
+        ws = workspace(p, OP_TOPK_SELECT, device=q.device)
+    _lib.check("msa_topk_select", _lib.load().msa_topk_select(
+        ctypes.byref(p), _ptr(q), _ptr(kbar), _ptr(kbar_hi), _ptr(kbar_lo), _ptr(idx),
+        _ptr(ws), ws.numel(), _stream(q.device)))
+    return idx
+
+
+def sparse_attn_fwd(q, k, v, idx, block: int, scale=None, want_lse=True, ws=None):
+    """Causal attention over the blocks in idx.  Returns (o, lse or None)."""
+    topk = idx.shape[-1]
+    p = _prefill_params(q, k, block, topk, scale)
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[0], q.shape[2], q.shape[1], dtype=torch.float32,
+                      device=q.device) if want_lse else None
+    if ws is None:
+        ws = workspace(p, OP_SPARSE_ATTN, device=q.device)
+    _lib.check("msa_sparse_attn_fwd", _lib.load().msa_sparse_attn_fwd(
+        ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(idx), _ptr(o), _ptr(lse), _ptr(ws),
+        ws.numel(), _stream(q.device)))
+    return o, lse
+
+
+def prefill_fwd(q, k, v, block: int, topk: int, scale=None, want_lse=True, ws=None, out=None):
+    """Whole causal prefill.  Returns (o, lse or None, idx).  `out` may pass preallocated
+    (o, lse, idx) tensors."""
+    p = _prefill_params(q, k, block, topk, scale)
+    b, S, hq, d = q.shape
+    hkv = k.shape[2]
+    if out is not None:
+        o, lse, idx = out
+    else:
+        o = torch.empty_like(q)
+        lse = torch.empty(b, hq, S, dtype=torch.float32, device=q.device) if want_lse else None
+        idx = torch.empty(b, hkv, S, topk, dtype=torch.int32, device=q.device)
+    if ws is None:
+        ws = workspace(p, OP_PREFILL, device=q.device)
+    _lib.check("msa_prefill_fwd", _lib.load().msa_prefill_fwd(
+        ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(idx), _ptr(o), _ptr(lse), _ptr(ws),
+        ws.numel(), _stream(q.device)))
+    return o, lse, idx
+
+
+def decode_fwd(q, kbar, k_bank, v_bank, block: int, topk: int, scale=None, kbar_hi=None,
+               want_lse=True, ws=None, out=None):
+    """Decode of q [n_query, hq, d] against a bank (k/v [S, hkv, d], kbar [nb, hkv, d]).
+    Returns (o, lse or None, idx [n_query, hkv, topk])."""
+    nq, hq, d = q.shape
+    S, hkv, _ = k_bank.shape
+    p = params(batch=1, seq=S, hq=hq, hkv=hkv, d=d, block=block, topk=topk,
+               scale=scale if scale is not None else d ** -0.5, dtype=q.dtype)
+    if out is not None:
+        o, lse, idx = out
+    else:
+        o = torch.empty_like(q)
+        lse = torch.empty(nq, hq, dtype=torch.float32, device=q.device) if want_lse else None
+        idx = torch.empty(nq, hkv, topk, dtype=torch.int32, device=q.device)
+    if ws is None:
+        ws = workspace(p, OP_DECODE, nq, device=q.device)
+    _lib.check("msa_decode_fwd", _lib.load().msa_decode_fwd(
+        ctypes.byref(p), nq, _ptr(q), _ptr(kbar), _ptr(kbar_hi), _ptr(k_bank), _ptr(v_bank),
+        _ptr(idx), _ptr(o), _ptr(lse), _ptr(ws), ws.numel(), _stream(q.device)))
+    return o, lse, idx
+
+
+def read_device_error(ws: torch.Tensor) -> int:
+    """Synchronises the current stream and returns the workspace's device error bits."""
+    bits = ctypes.c_int32(0)
+    st = _lib.load().msa_read_device_error(_ptr(ws), ctypes.byref(bits), _stream(ws.device))
+    if st not in (_lib.MSA_OK, _lib.MSA_ERR_DEVICE):
+        _lib.check("msa_read_device_error", st)
+    return bits.value
+
+
+def clear_device_error(ws: torch.Tensor) -> None:
+    _lib.check("msa_clear_device_error", _lib.load().msa_clear_device_error(
+        _ptr(ws), _stream(ws.device)))

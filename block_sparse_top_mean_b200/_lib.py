@@ -1,0 +1,76 @@
+"""ctypes binding of libmsa_b200.so (the C ABI declared in include/msa.h).
+
+Loading fails loudly when the library is missing: there is no fallback of any kind.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from ctypes import POINTER, c_char_p, c_float, c_int32, c_int64, c_size_t, c_void_p
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmsa_b200.so")
+
+MSA_OK, MSA_ERR_INVALID_ARG, MSA_ERR_UNSUPPORTED, MSA_ERR_WORKSPACE, MSA_ERR_CUDA, \
+    MSA_ERR_DEVICE = range(6)
+MSA_F32, MSA_BF16 = 0, 1
+OP_TOPK_SELECT, OP_SPARSE_ATTN, OP_PREFILL, OP_DECODE = range(4)
+DEVERR_IDX_RANGE, DEVERR_TIMEOUT = 0x1, 0x2
+
+# Every symbol include/msa.h declares, with (restype, argtypes).
+SIGNATURES = {
+    "msa_version": (c_char_p, []),
+    "msa_status_string": (c_char_p, [c_int32]),
+    "msa_workspace_bytes": (c_size_t, [c_void_p, c_int32, c_int64]),
+    "msa_pool_keys": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
+    "msa_block_scores": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
+    "msa_topk_select": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                  c_void_p, c_size_t, c_void_p]),
+    "msa_sparse_attn_fwd": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                      c_void_p, c_void_p, c_size_t, c_void_p]),
+    "msa_prefill_fwd": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                  c_void_p, c_void_p, c_size_t, c_void_p]),
+    "msa_decode_fwd": (c_int32, [c_void_p, c_int64, c_void_p, c_void_p, c_void_p, c_void_p,
+                                 c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
+                                 c_void_p]),
+    "msa_read_device_error": (c_int32, [c_void_p, POINTER(c_int32), c_void_p]),
+    "msa_clear_device_error": (c_int32, [c_void_p, c_void_p]),
+}
+
+
+class MsaParams(ctypes.Structure):
+    """Mirror of msa_params (include/msa.h)."""
+    _fields_ = [("batch", c_int64), ("seq", c_int64), ("hq", c_int64), ("hkv", c_int64),
+                ("d", c_int64), ("block", c_int64), ("topk", c_int64), ("scale", c_float),
+                ("dtype", c_int32)]
+
+
+class MsaError(RuntimeError):
+    def __init__(self, fn: str, status: int, text: str):
+        super().__init__(f"{fn} failed: {text} (status {status})")
+        self.status = status
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Loads the library once.  Raises if it has not been built (no fallback)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing: build it with "
+                          "`python -m block_sparse_top_mean_b200.build` (nvcc, sm_100a)")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def check(fn: str, status: int) -> None:
+    if status != MSA_OK:
+        text = load().msa_status_string(status).decode()
+        raise MsaError(fn, status, text)

@@ -1,0 +1,111 @@
+// Shared device helpers and internal launcher declarations of the msa library.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/msa.h"
+
+namespace msa {
+
+constexpr int kWsHeader = 256;   // bytes at the start of every workspace (error word)
+constexpr int kMaxTopk = 32;     // longest selection list a row can hold
+
+__device__ __forceinline__ uint4 ldg16(const void* p) {
+  return __ldg(reinterpret_cast<const uint4*>(p));
+}
+
+// Streaming 16-byte load that does not allocate in L1 (read-once data).
+__device__ __forceinline__ uint4 ldg16_stream(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ float bf16lo_to_f32(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi_to_f32(uint32_t w) {
+  return __uint_as_float(w & 0xffff0000u);
+}
+
+// Unpacks 16 bytes of T into fp32 (exact for both types).
+template <typename T> struct Vec16;
+template <> struct Vec16<float> {
+  static constexpr int N = 4;
+  __device__ __forceinline__ static void unpack(const uint4& u, float* f) {
+    f[0] = __uint_as_float(u.x); f[1] = __uint_as_float(u.y);
+    f[2] = __uint_as_float(u.z); f[3] = __uint_as_float(u.w);
+  }
+};
+template <> struct Vec16<__nv_bfloat16> {
+  static constexpr int N = 8;
+  __device__ __forceinline__ static void unpack(const uint4& u, float* f) {
+    f[0] = bf16lo_to_f32(u.x); f[1] = bf16hi_to_f32(u.x);
+    f[2] = bf16lo_to_f32(u.y); f[3] = bf16hi_to_f32(u.y);
+    f[4] = bf16lo_to_f32(u.z); f[5] = bf16hi_to_f32(u.z);
+    f[6] = bf16lo_to_f32(u.w); f[7] = bf16hi_to_f32(u.w);
+  }
+};
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+template <typename T> __device__ __forceinline__ float to_f32(T x);
+template <> __device__ __forceinline__ float to_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) {
+  return __bfloat162float(x);
+}
+
+__device__ __forceinline__ float warp_max(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+  return x;
+}
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
+__device__ __forceinline__ void set_device_error(int* err, int bits) {
+  if (err != nullptr) atomicOr(err, bits);
+}
+
+// ------------------------------------------------------------------ launchers
+// All return cudaSuccess or the launch error; shapes are validated by the caller.
+
+struct Shape {
+  int64_t batch, seq, hq, hkv, d, block, topk, nb;
+  float scale;
+  int dtype;
+};
+
+cudaError_t launch_pool_keys(const Shape& s, const void* k, float* kbar, void* hi, void* lo,
+                             int64_t n_seq, cudaStream_t st);
+
+cudaError_t launch_block_scores(const Shape& s, const void* q, const float* kbar, float* scores,
+                                cudaStream_t st);
+
+// Causal prefill selection (fused scoring + top-k); writes idx [b, hkv, S, topk].
+cudaError_t launch_topk_prefill(const Shape& s, const void* q, const float* kbar, int32_t* idx,
+                                cudaStream_t st);
+
+// Decode selection: per-split candidate lists then a merge; writes idx [nq, hkv, topk].
+size_t decode_select_ws_bytes(const Shape& s, int64_t n_query);
+cudaError_t launch_topk_decode(const Shape& s, int64_t n_query, const void* q, const float* kbar,
+                               int32_t* idx, void* ws, cudaStream_t st);
+
+// Query-centric attention over selected blocks (SIMT, fp32 math).
+size_t decode_attn_ws_bytes(const Shape& s, int64_t n_query);
+cudaError_t launch_attn_prefill_rows(const Shape& s, const void* q, const void* k, const void* v,
+                                     const int32_t* idx, void* o, float* lse, int* err,
+                                     cudaStream_t st);
+cudaError_t launch_attn_decode(const Shape& s, int64_t n_query, const void* q, const void* k,
+                               const void* v, const int32_t* idx, void* o, float* lse, void* ws,
+                               int* err, cudaStream_t st);
+
+}  // namespace msa

@@ -1,0 +1,218 @@
+// C ABI of the msa library: host-side argument checks, workspace layout, launches.
+// Every check runs before any CUDA call, so a rejected call touches no device state.
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "common.cuh"
+
+using msa::Shape;
+
+namespace {
+
+constexpr int64_t kMaxElems = (int64_t)1 << 40;   // guards every size product below
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
+size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+
+// Shape checks shared by every entry point.  `bank` = decode (seq is bank tokens).
+msa_status check_params(const msa_params* p, bool bank, Shape* s) {
+  if (p == nullptr) return MSA_ERR_INVALID_ARG;
+  if (p->batch < 0 || p->seq < 0 || p->hq < 1 || p->hkv < 1 || p->d < 1 || p->block < 1 ||
+      p->topk < 1)
+    return MSA_ERR_INVALID_ARG;
+  if (p->hq % p->hkv != 0) return MSA_ERR_INVALID_ARG;
+  if (!isfinite(p->scale)) return MSA_ERR_INVALID_ARG;
+  if (p->dtype != MSA_F32 && p->dtype != MSA_BF16) return MSA_ERR_INVALID_ARG;
+  if (p->d != 64 && p->d != 128) return MSA_ERR_UNSUPPORTED;
+  const int64_t G = p->hq / p->hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return MSA_ERR_UNSUPPORTED;
+  if (p->topk > msa::kMaxTopk) return MSA_ERR_UNSUPPORTED;
+  if (p->hkv > 65535) return MSA_ERR_UNSUPPORTED;
+  const int64_t bsz = bank ? 1 : p->batch;
+  if (bsz > 65535) return MSA_ERR_UNSUPPORTED;
+  if (p->seq > kMaxElems / (p->hq * p->d) || (bsz > 0 && p->seq * p->hq * p->d > kMaxElems / bsz))
+    return MSA_ERR_UNSUPPORTED;
+  s->batch = bsz; s->seq = p->seq; s->hq = p->hq; s->hkv = p->hkv; s->d = p->d;
+  s->block = p->block; s->topk = p->topk; s->scale = p->scale; s->dtype = p->dtype;
+  s->nb = (p->seq + p->block - 1) / p->block;
+  if (s->nb > INT32_MAX / 2) return MSA_ERR_UNSUPPORTED;
+  return MSA_OK;
+}
+
+bool empty_prefill(const Shape& s) { return s.batch == 0 || s.seq == 0; }
+
+size_t kbar_bytes(const Shape& s) { return (size_t)s.batch * s.nb * s.hkv * s.d * sizeof(float); }
+
+size_t ws_bytes_for(const Shape& s, int op, int64_t n_query) {
+  switch (op) {
+    case MSA_OP_TOPK_SELECT:
+    case MSA_OP_SPARSE_ATTN:
+      return msa::kWsHeader;
+    case MSA_OP_PREFILL:
+      return msa::kWsHeader + round256(kbar_bytes(s));
+    case MSA_OP_DECODE:
+      return msa::kWsHeader + round256(msa::decode_select_ws_bytes(s, n_query)) +
+             round256(msa::decode_attn_ws_bytes(s, n_query));
+    default:
+      return 0;
+  }
+}
+
+msa_status check_ws(const Shape& s, int op, int64_t n_query, const void* ws, size_t ws_bytes) {
+  const size_t need = ws_bytes_for(s, op, n_query);
+  if (ws == nullptr || ws_bytes < need || !aligned256(ws)) return MSA_ERR_WORKSPACE;
+  return MSA_OK;
+}
+
+msa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MSA_OK : MSA_ERR_CUDA; }
+
+int* err_word(void* ws) { return reinterpret_cast<int*>(ws); }
+char* ws_body(void* ws) { return reinterpret_cast<char*>(ws) + msa::kWsHeader; }
+
+}  // namespace
+
+extern "C" {
+
+const char* msa_version(void) { return "msa-b200 0.1.0 (sm_100a)"; }
+
+const char* msa_status_string(msa_status st) {
+  switch (st) {
+    case MSA_OK: return "ok";
+    case MSA_ERR_INVALID_ARG: return "invalid argument";
+    case MSA_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case MSA_ERR_WORKSPACE: return "workspace missing, too small or misaligned";
+    case MSA_ERR_CUDA: return "CUDA error";
+    case MSA_ERR_DEVICE: return "device-side error flag set";
+    default: return "unknown status";
+  }
+}
+
+size_t msa_workspace_bytes(const msa_params* p, int32_t op, int64_t n_query) {
+  Shape s;
+  if (check_params(p, op == MSA_OP_DECODE, &s) != MSA_OK) return 0;
+  if (op == MSA_OP_DECODE && n_query < 0) return 0;
+  return ws_bytes_for(s, op, n_query);
+}
+
+msa_status msa_pool_keys(const msa_params* p, const void* k, float* kbar, void* kbar_hi,
+                         void* kbar_lo, msa_stream_t stream) {
+  Shape s;
+  msa_status st = check_params(p, false, &s);
+  if (st != MSA_OK) return st;
+  if (empty_prefill(s)) return MSA_OK;
+  if (k == nullptr || kbar == nullptr || !aligned16(k) || !aligned16(kbar))
+    return MSA_ERR_INVALID_ARG;
+  if ((kbar_hi != nullptr && !aligned16(kbar_hi)) || (kbar_lo != nullptr && !aligned16(kbar_lo)))
+    return MSA_ERR_INVALID_ARG;
+  if (s.nb > INT32_MAX) return MSA_ERR_UNSUPPORTED;
+  return cuda_status(msa::launch_pool_keys(s, k, kbar, kbar_hi, kbar_lo, s.batch,
+                                           (cudaStream_t)stream));
+}
+
+msa_status msa_block_scores(const msa_params* p, const void* q, const float* kbar, float* scores,
+                            msa_stream_t stream) {
+  Shape s;
+  msa_status st = check_params(p, false, &s);
+  if (st != MSA_OK) return st;
+  if (empty_prefill(s)) return MSA_OK;
+  if (q == nullptr || kbar == nullptr || scores == nullptr) return MSA_ERR_INVALID_ARG;
+  if ((double)s.batch * s.hkv * s.seq * s.nb > (double)(((int64_t)1 << 31) - 1) * 256)
+    return MSA_ERR_UNSUPPORTED;
+  return cuda_status(msa::launch_block_scores(s, q, kbar, scores, (cudaStream_t)stream));
+}
+
+msa_status msa_topk_select(const msa_params* p, const void* q, const float* kbar,
+                           const void* kbar_hi, const void* kbar_lo, int32_t* idx, void* ws,
+                           size_t ws_bytes, msa_stream_t stream) {
+  (void)kbar_hi; (void)kbar_lo;
+  Shape s;
+  msa_status st = check_params(p, false, &s);
+  if (st != MSA_OK) return st;
+  if (empty_prefill(s)) return MSA_OK;
+  if (q == nullptr || kbar == nullptr || idx == nullptr || !aligned16(q) || !aligned16(kbar))
+    return MSA_ERR_INVALID_ARG;
+  if ((st = check_ws(s, MSA_OP_TOPK_SELECT, 0, ws, ws_bytes)) != MSA_OK) return st;
+  return cuda_status(msa::launch_topk_prefill(s, q, kbar, idx, (cudaStream_t)stream));
+}
+
+msa_status msa_sparse_attn_fwd(const msa_params* p, const void* q, const void* k, const void* v,
+                               const int32_t* idx, void* o, float* lse, void* ws,
+                               size_t ws_bytes, msa_stream_t stream) {
+  Shape s;
+  msa_status st = check_params(p, false, &s);
+  if (st != MSA_OK) return st;
+  if (empty_prefill(s)) return MSA_OK;
+  if (q == nullptr || k == nullptr || v == nullptr || idx == nullptr || o == nullptr)
+    return MSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return MSA_ERR_INVALID_ARG;
+  if ((st = check_ws(s, MSA_OP_SPARSE_ATTN, 0, ws, ws_bytes)) != MSA_OK) return st;
+  return cuda_status(msa::launch_attn_prefill_rows(s, q, k, v, idx, o, lse, err_word(ws),
+                                                   (cudaStream_t)stream));
+}
+
+msa_status msa_prefill_fwd(const msa_params* p, const void* q, const void* k, const void* v,
+                           int32_t* idx, void* o, float* lse, void* ws, size_t ws_bytes,
+                           msa_stream_t stream) {
+  Shape s;
+  msa_status st = check_params(p, false, &s);
+  if (st != MSA_OK) return st;
+  if (empty_prefill(s)) return MSA_OK;
+  if (q == nullptr || k == nullptr || v == nullptr || idx == nullptr || o == nullptr)
+    return MSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return MSA_ERR_INVALID_ARG;
+  if ((st = check_ws(s, MSA_OP_PREFILL, 0, ws, ws_bytes)) != MSA_OK) return st;
+  cudaStream_t cs = (cudaStream_t)stream;
+  float* kbar = reinterpret_cast<float*>(ws_body(ws));
+  cudaError_t e = msa::launch_pool_keys(s, k, kbar, nullptr, nullptr, s.batch, cs);
+  if (e == cudaSuccess) e = msa::launch_topk_prefill(s, q, kbar, idx, cs);
+  if (e == cudaSuccess) e = msa::launch_attn_prefill_rows(s, q, k, v, idx, o, lse, err_word(ws), cs);
+  return cuda_status(e);
+}
+
+msa_status msa_decode_fwd(const msa_params* p, int64_t n_query, const void* q, const float* kbar,
+                          const void* kbar_hi, const void* k_bank, const void* v_bank,
+                          int32_t* idx, void* o, float* lse, void* ws, size_t ws_bytes,
+                          msa_stream_t stream) {
+  (void)kbar_hi;
+  Shape s;
+  msa_status st = check_params(p, true, &s);
+  if (st != MSA_OK) return st;
+  if (n_query < 0) return MSA_ERR_INVALID_ARG;
+  if (n_query == 0 || s.seq == 0) return MSA_OK;
+  if (n_query > 65535 * 64) return MSA_ERR_UNSUPPORTED;
+  if (q == nullptr || kbar == nullptr || k_bank == nullptr || v_bank == nullptr ||
+      idx == nullptr || o == nullptr)
+    return MSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(kbar) || !aligned16(k_bank) || !aligned16(v_bank) ||
+      !aligned16(o))
+    return MSA_ERR_INVALID_ARG;
+  if ((st = check_ws(s, MSA_OP_DECODE, n_query, ws, ws_bytes)) != MSA_OK) return st;
+  cudaStream_t cs = (cudaStream_t)stream;
+  char* sel_ws = ws_body(ws);
+  char* att_ws = sel_ws + round256(msa::decode_select_ws_bytes(s, n_query));
+  cudaError_t e = msa::launch_topk_decode(s, n_query, q, kbar, idx, sel_ws, cs);
+  if (e == cudaSuccess)
+    e = msa::launch_attn_decode(s, n_query, q, k_bank, v_bank, idx, o, lse, att_ws, err_word(ws),
+                                cs);
+  return cuda_status(e);
+}
+
+msa_status msa_read_device_error(const void* ws, int32_t* bits, msa_stream_t stream) {
+  if (ws == nullptr || bits == nullptr) return MSA_ERR_INVALID_ARG;
+  int32_t h = 0;
+  cudaError_t e = cudaMemcpyAsync(&h, ws, sizeof(int32_t), cudaMemcpyDeviceToHost,
+                                  (cudaStream_t)stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return MSA_ERR_CUDA;
+  *bits = h;
+  return h != 0 ? MSA_ERR_DEVICE : MSA_OK;
+}
+
+msa_status msa_clear_device_error(void* ws, msa_stream_t stream) {
+  if (ws == nullptr) return MSA_ERR_INVALID_ARG;
+  return cuda_status(cudaMemsetAsync(ws, 0, sizeof(int32_t), (cudaStream_t)stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,184 @@
+/*
+ * msa.h - C ABI of the B200 (sm_100a) block-sparse top-k attention library.
+ *
+ * The method: pool each KV block into one routing key, score every query against the
+ * pooled keys per GQA group, keep the top-k blocks per (query, group), and run exact
+ * softmax attention over only the selected K/V blocks.  Sources:
+ *   [MiniMax] "MiniMax released MSA: sparse attention speeds up 1M-token context
+ *             processing by 28x" (news.hamidun.com), section "How MSA Works": an index
+ *             branch picks, for each query and each GQA group, the top-k blocks of keys
+ *             and values; a main branch then runs full, exact attention over only those
+ *             blocks.  Section "Why Long Context is Hard to Scale": the main branch is
+ *             kept exact.
+ *   [MoBA]    "MoBA: Mixture of Block Attention for Long-Context LLMs" catalogue card
+ *             (ross.abutalabs.com/products/moba.json), field what_it_is: MoE-style
+ *             top-k gating over KV blocks; full attention is the case where every block
+ *             is selected.
+ *   [MSA-DE]  "100 Millionen Token: Gedaechtnis oder Trugbild?" (aitalk.it), section
+ *             "Das Gehirn mit zwei Geschwindigkeiten": small routing keys stay on the
+ *             GPU and decide relevance; content is attended only once selected; the
+ *             routing keys of a memory bank are computed offline.
+ * Readings where the pages are silent (they print no formula):
+ *   - pooled key = arithmetic mean of the block's keys per KV head (a ragged last block
+ *     averages the tokens it holds);
+ *   - score(t, g, j) = sum over the group's query heads h of q[t,h] . kbar[j,g]
+ *     (unscaled; query head h belongs to group h / (hq/hkv));
+ *   - ranking by (score descending, block index ascending);
+ *   - causal prefill: the query's own block i = t / block is always selected and the
+ *     remaining topk-1 slots go to the best past blocks j < i; inside block i only keys
+ *     p <= t are attended; when fewer than topk-1 past blocks exist all are taken;
+ *   - decode against a bank: every block is eligible, top `topk`, no mask;
+ *   - attention: one softmax per query head over the union of the selected keys,
+ *     logits = scale * q . k.
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers, row-major and contiguous, 16-byte
+ *     aligned.  The caller owns every buffer; the library allocates nothing.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and never synchronise, except msa_read_device_error.
+ *   - Arguments are checked on the host before anything is launched; a failed check
+ *     returns MSA_ERR_INVALID_ARG / MSA_ERR_UNSUPPORTED / MSA_ERR_WORKSPACE and launches
+ *     nothing.  A launch failure returns MSA_ERR_CUDA.
+ *   - Data-dependent faults found on the device (an index out of range, a bounded wait
+ *     that ran out) never trap: the kernel skips the offending work and ORs a bit into
+ *     the error word at the start of the workspace; read it with msa_read_device_error.
+ *   - batch == 0, seq == 0 or n_query == 0 is a valid empty call that launches nothing.
+ *   - Results are bitwise deterministic run to run (no floating-point atomics).
+ *
+ * Layouts (b = batch, S = seq, nb = ceil(S / block), G = hq / hkv):
+ *   q    [b, S, hq, d]       k, v [b, S, hkv, d]      o [b, S, hq, d]   (dtype)
+ *   kbar [b, nb, hkv, d] fp32; kbar_hi / kbar_lo same shape, bf16 (hi = bf16(kbar),
+ *        lo = bf16(kbar - hi))
+ *   idx  [b, hkv, S, topk] int32, ascending, padded with -1 at the end
+ *   lse  [b, hq, S] fp32, natural log of sum_p exp(scale * q . k_p)
+ *   decode: q [n_query, hq, d], bank k/v [S, hkv, d], kbar [nb, hkv, d],
+ *           idx [n_query, hkv, topk], o [n_query, hq, d], lse [n_query, hq]
+ */
+#ifndef MSA_H_
+#define MSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define MSA_API __attribute__((visibility("default")))
+#else
+#define MSA_API
+#endif
+
+struct CUstream_st;
+typedef struct CUstream_st* msa_stream_t; /* same object as cudaStream_t */
+
+typedef enum {
+  MSA_OK = 0,
+  MSA_ERR_INVALID_ARG = 1, /* null pointer, bad shape, misaligned pointer */
+  MSA_ERR_UNSUPPORTED = 2, /* well-formed but outside what the kernels implement */
+  MSA_ERR_WORKSPACE = 3,   /* workspace missing, too small or misaligned */
+  MSA_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed */
+  MSA_ERR_DEVICE = 5       /* returned by msa_read_device_error when a bit is set */
+} msa_status;
+
+typedef enum { MSA_F32 = 0, MSA_BF16 = 1 } msa_dtype;
+
+typedef enum {
+  MSA_OP_TOPK_SELECT = 0,
+  MSA_OP_SPARSE_ATTN = 1,
+  MSA_OP_PREFILL = 2,
+  MSA_OP_DECODE = 3
+} msa_op;
+
+/* Device error bits (msa_read_device_error). */
+#define MSA_DEVERR_IDX_RANGE 0x1   /* an idx entry outside [-1, nb) or violating causality */
+#define MSA_DEVERR_TIMEOUT 0x2     /* a bounded barrier wait ran out */
+
+typedef struct {
+  int64_t batch; /* independent sequences (prefill); ignored by decode */
+  int64_t seq;   /* tokens per sequence (prefill) or bank tokens (decode) */
+  int64_t hq;    /* query heads; hq % hkv == 0 */
+  int64_t hkv;   /* key/value heads (GQA groups) */
+  int64_t d;     /* head dim: 64 or 128 */
+  int64_t block; /* tokens per KV block, >= 1 */
+  int64_t topk;  /* selected blocks per (query, group), 1..32, own block included */
+  float scale;   /* softmax scale, finite */
+  int32_t dtype; /* msa_dtype of q, k, v, o */
+} msa_params;
+
+/* Library version string. */
+MSA_API const char* msa_version(void);
+
+/* Human-readable name of a status code (static storage). */
+MSA_API const char* msa_status_string(msa_status status);
+
+/* Workspace bytes that `op` needs for these shapes (n_query is used by MSA_OP_DECODE
+ * only).  Returns 0 when the shapes are invalid.  Pass a buffer of at least this size,
+ * 256-byte aligned, to the matching call.  The first 256 bytes hold the device error
+ * word; the rest is scratch whose content between calls is unspecified. */
+MSA_API size_t msa_workspace_bytes(const msa_params* p, int32_t op, int64_t n_query);
+
+/* Step 1, block pooling ([MSA-DE] routing keys; [MoBA] KV blocks):
+ *   kbar[b,j,g,:] = (1/n_j) * sum_{t in block j} k[b,t,g,:],  n_j = tokens in block j.
+ * kbar (fp32) is required; kbar_hi / kbar_lo (bf16 split planes) may each be NULL.
+ * Accumulates in fp32 in token order.  Applied to a memory bank this is the offline
+ * encoding of its routing keys. */
+MSA_API msa_status msa_pool_keys(const msa_params* p, const void* k, float* kbar, void* kbar_hi,
+                         void* kbar_lo, msa_stream_t stream);
+
+/* Step 2 materialised, for inspection and small shapes ([MiniMax] index branch):
+ *   scores[b,g,t,j] = sum_{h in group g} q[b,t,h,:] . kbar[b,j,g,:]   for j < t/block,
+ *   -inf for j >= t/block.  fp32, [b, hkv, S, nb].  The fused selection never stores
+ *   scores; this entry is O(S * nb) memory. */
+MSA_API msa_status msa_block_scores(const msa_params* p, const void* q, const float* kbar,
+                            float* scores, msa_stream_t stream);
+
+/* Steps 2+3 fused, causal prefill ([MiniMax] index branch; [MoBA] top-k gating):
+ * idx[b,g,t,:] = {t/block} U top-(topk-1) past blocks by (score desc, index asc),
+ * ascending, -1 padded.  kbar is required; kbar_hi / kbar_lo may be NULL (they are
+ * used when present).  ws: msa_workspace_bytes(p, MSA_OP_TOPK_SELECT, 0). */
+MSA_API msa_status msa_topk_select(const msa_params* p, const void* q, const float* kbar,
+                           const void* kbar_hi, const void* kbar_lo, int32_t* idx, void* ws,
+                           size_t ws_bytes, msa_stream_t stream);
+
+/* Step 4, causal prefill ([MiniMax] main branch, exact):
+ *   o[b,t,h,:] = sum_{p in U} softmax_p(scale * q[b,t,h,:] . k[b,p,g,:]) v[b,p,g,:],
+ *   U = keys of the blocks in idx[b,g,t,:] (entries -1 skipped), keeping p <= t.
+ * lse may be NULL.  Entries outside [-1, nb) or after the own block set
+ * MSA_DEVERR_IDX_RANGE and are skipped.  ws: msa_workspace_bytes(p, MSA_OP_SPARSE_ATTN). */
+MSA_API msa_status msa_sparse_attn_fwd(const msa_params* p, const void* q, const void* k, const void* v,
+                               const int32_t* idx, void* o, float* lse, void* ws,
+                               size_t ws_bytes, msa_stream_t stream);
+
+/* Whole causal prefill: msa_pool_keys -> msa_topk_select -> msa_sparse_attn_fwd, with the
+ * pooled keys kept in the workspace.  idx is written (caller-owned, [b,hkv,S,topk]);
+ * lse may be NULL.  ws: msa_workspace_bytes(p, MSA_OP_PREFILL, 0). */
+MSA_API msa_status msa_prefill_fwd(const msa_params* p, const void* q, const void* k, const void* v,
+                           int32_t* idx, void* o, float* lse, void* ws, size_t ws_bytes,
+                           msa_stream_t stream);
+
+/* Decode against a memory bank ([MSA-DE] routing keys in GPU memory decide which content
+ * is attended; [MiniMax] per query and GQA group top-k):  for each query n and group g,
+ * idx[n,g,:] = top-`topk` of all nb bank blocks by (score desc, index asc), ascending;
+ * then exact attention of the group's heads over those blocks' keys, no mask.
+ * p->seq is the number of bank tokens, p->batch is ignored.  kbar is the bank's pooled
+ * keys from msa_pool_keys (fp32, required); kbar_hi may be NULL.
+ * ws: msa_workspace_bytes(p, MSA_OP_DECODE, n_query). */
+MSA_API msa_status msa_decode_fwd(const msa_params* p, int64_t n_query, const void* q, const float* kbar,
+                          const void* kbar_hi, const void* k_bank, const void* v_bank,
+                          int32_t* idx, void* o, float* lse, void* ws, size_t ws_bytes,
+                          msa_stream_t stream);
+
+/* Copies the workspace's device error word to *bits after synchronising `stream`;
+ * returns MSA_ERR_DEVICE when any bit is set, else MSA_OK. */
+MSA_API msa_status msa_read_device_error(const void* ws, int32_t* bits, msa_stream_t stream);
+
+/* Clears the workspace's device error word (asynchronous on `stream`). */
+MSA_API msa_status msa_clear_device_error(void* ws, msa_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MSA_H_ */

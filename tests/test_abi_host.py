@@ -1,0 +1,117 @@
+"""The C ABI on the host: the library loads, exports every symbol include/msa.h declares,
+and rejects bad arguments before touching the device (these calls need no GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from block_sparse_top_mean_b200 import _lib
+from block_sparse_top_mean_b200._lib import MsaParams
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_symbols():
+    src = open(os.path.join(ROOT, "include", "msa.h")).read()
+    return sorted(set(re.findall(r"MSA_API\s+[\w\s\*]+?\b(msa_\w+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from block_sparse_top_mean_b200 import build
+    build.build()
+    return _lib.load()
+
+
+def test_header_declares_the_boundary():
+    names = _declared_symbols()
+    for n in ["msa_pool_keys", "msa_block_scores", "msa_topk_select", "msa_sparse_attn_fwd",
+              "msa_decode_fwd", "msa_prefill_fwd", "msa_workspace_bytes"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = _declared_symbols()
+    assert set(names) == set(_lib.SIGNATURES), "binding and header disagree"
+    for n in names:
+        assert hasattr(lib, n), n
+    assert lib.msa_version().decode().startswith("msa-b200")
+
+
+def _p(**kw):
+    base = dict(batch=1, seq=1024, hq=32, hkv=8, d=128, block=128, topk=16, scale=0.088,
+                dtype=_lib.MSA_BF16)
+    base.update(kw)
+    return MsaParams(*[base[k] for k in ["batch", "seq", "hq", "hkv", "d", "block", "topk",
+                                         "scale", "dtype"]])
+
+
+FAKE = ctypes.c_void_p(4096)       # non-null, aligned; never dereferenced (checks fail first)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(hq=30), _lib.MSA_ERR_INVALID_ARG),          # hq % hkv != 0
+    (dict(block=0), _lib.MSA_ERR_INVALID_ARG),
+    (dict(topk=0), _lib.MSA_ERR_INVALID_ARG),
+    (dict(seq=-1), _lib.MSA_ERR_INVALID_ARG),
+    (dict(dtype=7), _lib.MSA_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), _lib.MSA_ERR_INVALID_ARG),
+    (dict(d=96), _lib.MSA_ERR_UNSUPPORTED),
+    (dict(topk=33), _lib.MSA_ERR_UNSUPPORTED),
+    (dict(hq=24, hkv=8), _lib.MSA_ERR_UNSUPPORTED),     # G = 3
+])
+def test_bad_params_rejected_before_launch(lib, kw, code):
+    p = _p(**kw)
+    st = lib.msa_sparse_attn_fwd(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE,
+                                 1 << 20, None)
+    assert st == code
+    assert lib.msa_workspace_bytes(ctypes.byref(p), _lib.OP_PREFILL, 0) == 0
+    assert lib.msa_pool_keys(ctypes.byref(p), FAKE, FAKE, None, None, None) == code
+
+
+def test_null_and_misaligned_pointers_rejected(lib):
+    p = _p()
+    assert lib.msa_pool_keys(None, FAKE, FAKE, None, None, None) == _lib.MSA_ERR_INVALID_ARG
+    assert lib.msa_pool_keys(ctypes.byref(p), None, FAKE, None, None, None) == \
+        _lib.MSA_ERR_INVALID_ARG
+    odd = ctypes.c_void_p(4096 + 8)
+    assert lib.msa_pool_keys(ctypes.byref(p), odd, FAKE, None, None, None) == \
+        _lib.MSA_ERR_INVALID_ARG
+    assert lib.msa_sparse_attn_fwd(ctypes.byref(p), FAKE, FAKE, FAKE, None, FAKE, None, FAKE,
+                                   1 << 20, None) == _lib.MSA_ERR_INVALID_ARG
+    assert lib.msa_read_device_error(None, None, None) == _lib.MSA_ERR_INVALID_ARG
+
+
+def test_workspace_checks(lib):
+    p = _p()
+    need = lib.msa_workspace_bytes(ctypes.byref(p), _lib.OP_PREFILL, 0)
+    assert need >= 256 + 8 * 8 * 128 * 4          # header + pooled keys [1, 8, 8, 128] fp32
+    st = lib.msa_prefill_fwd(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE,
+                             need - 1, None)
+    assert st == _lib.MSA_ERR_WORKSPACE
+    st = lib.msa_prefill_fwd(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE, None,
+                             ctypes.c_void_p(4096 + 16), need, None)
+    assert st == _lib.MSA_ERR_WORKSPACE              # not 256-byte aligned
+    st = lib.msa_prefill_fwd(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE, None, None, need, None)
+    assert st == _lib.MSA_ERR_WORKSPACE
+    nd = lib.msa_workspace_bytes(ctypes.byref(_p(seq=10_000_000, block=64, topk=32)),
+                                 _lib.OP_DECODE, 64)
+    assert nd > 256
+    assert lib.msa_workspace_bytes(ctypes.byref(p), 99, 0) == 0
+
+
+def test_empty_inputs_are_noops(lib):
+    for kw in (dict(seq=0), dict(batch=0)):
+        p = _p(**kw)
+        assert lib.msa_prefill_fwd(ctypes.byref(p), None, None, None, None, None, None, None, 0,
+                                   None) == _lib.MSA_OK
+        assert lib.msa_pool_keys(ctypes.byref(p), None, None, None, None, None) == _lib.MSA_OK
+    p = _p()
+    assert lib.msa_decode_fwd(ctypes.byref(p), 0, None, None, None, None, None, None, None,
+                              None, None, 0, None) == _lib.MSA_OK
+
+
+def test_status_strings(lib):
+    for c in range(6):
+        assert lib.msa_status_string(c).decode()

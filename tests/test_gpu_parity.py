@@ -1,0 +1,187 @@
+"""GPU path vs the fp64 oracle, through the C ABI (via the ctypes binding).
+
+Small cases compare every row; they span several kernel tiles and a ragged tail.
+The full-size workloads are checked on a stratified sample of rows, with the same
+launch configuration the benchmark times.
+"""
+import numpy as np
+import pytest
+import torch
+
+import msa_inputs as mi
+import oracle
+from parity_util import (HostView, check_decode, check_prefill, pool_keys_chunked,
+                         sample_tokens)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def msa():
+    import block_sparse_top_mean_b200 as m
+    from block_sparse_top_mean_b200 import build
+    build.build()
+    return m
+
+
+def _inputs(w, seed=0):
+    q, k, v = mi.prefill_inputs(w, device="cuda", seed=seed)
+    return q, k, v
+
+
+SMALL = [
+    mi.WORKLOADS["prefill_tiny_s1k_f32"],
+    mi.Workload("bf16_ragged_b128", "prefill", 1, 3000, 8, 2, 128, 128, 8, "bf16"),
+    mi.Workload("bf16_ragged_b512", "prefill", 1, 5000, 8, 2, 128, 512, 8, "bf16"),
+    mi.Workload("bf16_b256_g4", "prefill", 1, 4096, 16, 4, 128, 256, 6, "bf16"),
+    mi.Workload("f32_d128_g8_b2", "prefill", 2, 700, 16, 2, 128, 64, 5, "f32"),
+    mi.Workload("bf16_d64_g1", "prefill", 1, 2000, 4, 4, 64, 64, 4, "bf16"),
+    mi.Workload("f32_topk1", "prefill", 1, 600, 4, 2, 64, 64, 1, "f32"),
+    mi.Workload("f32_topk_all", "prefill", 1, 1000, 4, 1, 64, 64, 32, "f32"),
+    mi.Workload("f32_one_partial_block", "prefill", 1, 50, 2, 1, 64, 64, 4, "f32"),
+    mi.Workload("bf16_planted", "prefill", 1, 4096, 8, 2, 128, 128, 8, "bf16",
+                planted_frac=0.02, planted_shift=3.0),
+]
+
+
+@pytest.mark.parametrize("w", SMALL, ids=lambda w: w.name)
+def test_prefill_small_all_rows(msa, w):
+    q, k, v = _inputs(w)
+    o, lse, idx = msa.prefill_fwd(q, k, v, w.block, w.topk, w.scale)
+    torch.cuda.synchronize()
+    check_prefill(q, k, v, w.block, w.topk, w.scale, idx, o, lse)
+
+
+@pytest.mark.parametrize("w", SMALL[:4], ids=lambda w: w.name)
+def test_pool_keys_vs_oracle(msa, w):
+    q, k, v = _inputs(w)
+    kbar, hi, lo = msa.pool_keys(k, w.block, split=True)
+    ref = oracle.pool_keys(k.float().cpu().numpy(), w.block)
+    got = kbar.double().cpu().numpy()
+    # fp32 sum of <= block terms of |x| < 6: error <= block * 2^-24 * 6
+    assert np.abs(got - ref).max() <= w.block * 6 * 2.0 ** -24
+    # split planes: hi = bf16(kbar), lo = bf16(kbar - hi)
+    assert torch.equal(hi, kbar.to(torch.bfloat16))
+    assert torch.equal(lo, (kbar - hi.float()).to(torch.bfloat16))
+
+
+@pytest.mark.parametrize("w", SMALL[:3], ids=lambda w: w.name)
+def test_block_scores_vs_oracle(msa, w):
+    q, k, v = _inputs(w)
+    kbar = msa.pool_keys(k, w.block)
+    sc = msa.block_scores(q, kbar, w.block, w.hkv).double().cpu().numpy()
+    kb = oracle.pool_keys(k.float().cpu().numpy(), w.block)
+    Q = q.float().cpu().numpy()
+    for t in range(0, w.seq, 97):
+        i = t // w.block
+        ref = oracle.prefill_block_scores(Q[0, t], kb[0], i)          # [hkv, i]
+        got = sc[0, :, t, :]
+        assert np.all(np.isinf(got[:, i:]))
+        if i:
+            np.testing.assert_allclose(got[:, :i], ref, rtol=1e-4, atol=1e-4)
+
+
+@pytest.mark.parametrize("w", SMALL[1:3], ids=lambda w: w.name)
+def test_topk_select_and_attn_separately(msa, w):
+    """Each step alone: the selection vs the oracle, and the attention fed the
+    oracle's own selection vs the oracle."""
+    q, k, v = _inputs(w)
+    kbar = msa.pool_keys(k, w.block)
+    idx = msa.topk_select(q, kbar, w.block, w.topk, w.hkv)
+    rows = [(0, t) for t in range(0, w.seq, 7)]
+    Q, K, V = HostView(q), HostView(k), HostView(v)
+    ref = oracle.prefill_rows(Q, K, V, w.block, w.topk, w.scale, rows=rows)
+    gi = idx.cpu().numpy()
+    for r in ref:
+        if r.gap > 1e-3:
+            assert list(gi[0, r.g, r.t]) == r.idx
+    oidx = torch.full_like(idx, -1)
+    for r in oracle.prefill_rows(Q, K, V, w.block, w.topk, w.scale):
+        oidx[0, r.g, r.t] = torch.tensor(r.idx)
+    o, lse = msa.sparse_attn_fwd(q, k, v, oidx, w.block, w.scale)
+    check_prefill(q, k, v, w.block, w.topk, w.scale, oidx, o, lse, rows=rows)
+
+
+def test_out_of_range_index_sets_error_word_and_skips(msa):
+    w = SMALL[1]
+    q, k, v = _inputs(w)
+    kbar = msa.pool_keys(k, w.block)
+    idx = msa.topk_select(q, kbar, w.block, w.topk, w.hkv)
+    p = msa.params(batch=1, seq=w.seq, hq=w.hq, hkv=w.hkv, d=w.d, block=w.block, topk=w.topk,
+                   scale=w.scale, dtype=q.dtype)
+    ws = msa.workspace(p, msa.OP_SPARSE_ATTN)
+    o_ref, _ = msa.sparse_attn_fwd(q, k, v, idx, w.block, w.scale, ws=ws)
+    assert msa.read_device_error(ws) == 0
+    bad = idx.clone()
+    t = w.seq - 1
+    bad[0, 0, t, 0] = 10_000          # beyond nb
+    bad[0, 1, 5, 1] = 3               # a future block for token 5 (own block 0)
+    o_bad, _ = msa.sparse_attn_fwd(q, k, v, bad, w.block, w.scale, ws=ws)
+    assert msa.read_device_error(ws) & msa.DEVERR_IDX_RANGE
+    msa.clear_device_error(ws)
+    assert msa.read_device_error(ws) == 0
+    # untouched rows are unchanged
+    assert torch.equal(o_bad[0, :w.seq - 1, :w.hq // w.hkv], o_ref[0, :w.seq - 1, :w.hq // w.hkv])
+
+
+def test_prefill_is_deterministic(msa):
+    w = SMALL[3]
+    q, k, v = _inputs(w)
+    a = msa.prefill_fwd(q, k, v, w.block, w.topk, w.scale)
+    b = msa.prefill_fwd(q, k, v, w.block, w.topk, w.scale)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+
+
+DECODE_SMALL = [
+    mi.Workload("decode_small_bf16", "decode", 1, 50_000, 32, 8, 128, 64, 32, "bf16", n_query=8),
+    mi.Workload("decode_small_f32", "decode", 1, 9_000, 8, 2, 64, 64, 8, "f32", n_query=70),
+    mi.Workload("decode_all_blocks", "decode", 1, 1000, 4, 1, 64, 64, 32, "f32", n_query=3),
+]
+
+
+@pytest.mark.parametrize("w", DECODE_SMALL, ids=lambda w: w.name)
+def test_decode_small(msa, w):
+    q, kb, vb = mi.decode_inputs(w, device="cuda")
+    kbar = msa.pool_keys(kb[None], w.block)[0]
+    o, lse, idx = msa.decode_fwd(q, kbar, kb, vb, w.block, w.topk, w.scale)
+    torch.cuda.synchronize()
+    kbar_np = pool_keys_chunked(kb[None], w.block)[0]
+    check_decode(q, kbar_np, kb, vb, w.block, w.topk, w.scale, idx, o, lse)
+
+
+# ------------------------------------------------------------------ full-size workloads
+
+FULL_PREFILL = ["prefill_tiny_s1k_f32", "prefill_32k_b512_k8", "prefill_128k_b128_k16_planted",
+                "prefill_1m_b256_k16"]
+
+
+@pytest.mark.parametrize("name", FULL_PREFILL)
+def test_prefill_full_size_sampled(msa, name):
+    w = mi.WORKLOADS[name]
+    q, k, v = _inputs(w)
+    o, lse, idx = msa.prefill_fwd(q, k, v, w.block, w.topk, w.scale)
+    torch.cuda.synchronize()
+    rows = [(0, t) for t in sample_tokens(w.seq, w.block, 192)]
+    rep = {}
+    check_prefill(q, k, v, w.block, w.topk, w.scale, idx, o, lse, rows=rows, report=rep)
+    print(name, rep)
+    # properties at every row: own block present, nothing in the future, ascending
+    own = (torch.arange(w.seq, device="cuda") // w.block).view(1, 1, -1)
+    sel = idx.long()
+    assert bool((sel.max(dim=-1).values == own).all())
+    valid = sel >= 0
+    assert bool((sel[..., 1:] > sel[..., :-1])[valid[..., 1:]].all())
+    assert torch.isfinite(o.float()).all()
+
+
+def test_decode_full_size_sampled(msa):
+    w = mi.WORKLOADS["decode_bank10m_b64_k32"]
+    q, kb, vb = mi.decode_inputs(w, device="cuda")
+    kbar = msa.pool_keys(kb[None], w.block)[0]
+    o, lse, idx = msa.decode_fwd(q, kbar, kb, vb, w.block, w.topk, w.scale)
+    torch.cuda.synchronize()
+    kbar_np = pool_keys_chunked(kb[None], w.block, tokens_per_chunk=1 << 21)[0]
+    rep = check_decode(q, kbar_np, kb, vb, w.block, w.topk, w.scale, idx, o, lse,
+                       queries=list(range(0, w.n_query, 4)))
+    print(rep)
