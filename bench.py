@@ -174,6 +174,9 @@ class PrefillRunner:
         self.p = msa.params(batch=w.batch, seq=w.seq, hq=w.hq, hkv=w.hkv, d=w.d, block=w.block,
                             topk=w.topk, scale=w.scale, dtype=self.q.dtype)
         self.kbar = torch.empty(w.batch, w.nb, w.hkv, w.d, dtype=torch.float32, device=dev)
+        # bf16 hi/lo planes of the pooled keys feed the tensor-core selection
+        self.khi = torch.empty(w.batch, w.nb, w.hkv, w.d, dtype=torch.bfloat16, device=dev)
+        self.klo = torch.empty_like(self.khi)
         self.idx = torch.empty(w.batch, w.hkv, w.seq, w.topk, dtype=torch.int32, device=dev)
         self.o = torch.empty_like(self.q)
         self.lse = torch.empty(w.batch, w.hq, w.seq, dtype=torch.float32, device=dev)
@@ -182,7 +185,8 @@ class PrefillRunner:
         self.ws = torch.zeros(n, dtype=torch.uint8, device=dev)
         self.check = _lib.check
         P = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
-        self.ptr = {k: P(getattr(self, k)) for k in ("q", "k", "v", "kbar", "idx", "o", "lse", "ws")}
+        self.ptr = {k: P(getattr(self, k)) for k in ("q", "k", "v", "kbar", "khi", "klo", "idx", "o",
+                                                     "lse", "ws")}
         self.pp = ctypes.byref(self.p)
         self.launches_per_step = 3
 
@@ -191,11 +195,13 @@ class PrefillRunner:
         P, lib = self.ptr, self.lib
         if events:
             events[0].record()
-        self.check("msa_pool_keys", lib.msa_pool_keys(self.pp, P["k"], P["kbar"], None, None, s))
+        self.check("msa_pool_keys", lib.msa_pool_keys(self.pp, P["k"], P["kbar"], P["khi"],
+                                                      P["klo"], s))
         if events:
             events[1].record()
         self.check("msa_topk_select", lib.msa_topk_select(
-            self.pp, P["q"], P["kbar"], None, None, P["idx"], P["ws"], self.ws.numel(), s))
+            self.pp, P["q"], P["kbar"], P["khi"], P["klo"], P["idx"], P["ws"], self.ws.numel(),
+            s))
         if events:
             events[2].record()
         self.check("msa_sparse_attn_fwd", lib.msa_sparse_attn_fwd(

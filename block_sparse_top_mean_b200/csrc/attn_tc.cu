@@ -1,0 +1,556 @@
+// Step 4 on the tensor cores (bf16, d = 128): key-centric block-sparse attention.
+//
+// Every (token, group) selects different blocks, so query-centric tiles would share no
+// keys.  Instead the selection is inverted: for each (sequence, group, block) the list
+// of (token, slot) entries that selected it is built, and one tile = the G query heads
+// of 128/G such tokens (128 rows) against that block's keys.  K/V of a block are loaded
+// once per run of tiles into shared memory with TMA; the tile's query rows are gathered
+// with cp.async into the 128-byte-swizzled K-major layout the MMA reads.
+//
+// Per tile, per 128-key chunk c (a block of 256 keys is 2 chunks; longer blocks are
+// split into 256-key segments, each its own partial slot):
+//   S_c = Q K_c^T      tcgen05.mma, M=128 N=128 K=128, fp32 accumulator in TMEM
+//   softmax            one thread per row reads S_c from TMEM, masks (ragged block,
+//                      causal inside the own block), base-2 exponentials in fp32,
+//                      writes P_c as bf16 back into TMEM over S_c
+//   O_c = P_c V_c      tcgen05.mma with A from TMEM, B = V (MN-major) from shared memory
+// The epilogue merges the chunks and writes a normalised bf16 partial O plus its
+// log-sum-exp for (token, slot); a second kernel merges a row's partials into O.
+// TMEM columns: S_0 [0,128) S_1 [128,256) O_0 [256,384) O_1 [384,512).
+#include <cudaTypedefs.h>
+#include <math_constants.h>
+
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace msa {
+namespace {
+
+using namespace sm100;
+
+constexpr int kD = 128;
+constexpr int kRowsT = 128;          // rows per tile
+constexpr int kChunkKeys = 128;      // keys per MMA chunk
+constexpr int kSegKeys = 256;        // keys per segment
+constexpr int kThreads = 256;        // warps 0-3 softmax, 4 issuer, 5-7 gather
+constexpr int kGatherThreads = 96;
+constexpr uint32_t kTileBytes = 16384;   // 128 rows x 128 B
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+struct Geom {
+  int64_t S, nb, block, nseg;
+  int hq, hkv, G, topk, nsub, kslots, tpt, nch;
+  float scale_log2;
+};
+
+__device__ __forceinline__ bool sub_has_keys(int64_t j, int64_t own, int64_t t, int sub,
+                                             const Geom& g) {
+  const int64_t lo = j * g.block + (int64_t)sub * kSegKeys;
+  if ((int64_t)sub * kSegKeys >= g.block || lo >= g.S) return false;
+  return j < own || lo <= t;
+}
+
+// ------------------------------------------------------------------ index inversion
+__global__ void invert_count_kernel(const int32_t* __restrict__ idx, int* __restrict__ counts,
+                                    int* err, Geom g, int64_t n) {
+  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= n) return;
+  const int64_t row = e / g.topk;                // (b*hkv + gg)*S + t
+  const int64_t t = row % g.S, bg = row / g.S;
+  const int64_t j = idx[e];
+  if (j == -1) return;
+  const int64_t own = t / g.block;
+  if (j < -1 || j >= g.nb || j > own) {
+    set_device_error(err, MSA_DEVERR_IDX_RANGE);
+    return;
+  }
+  for (int sub = 0; sub < g.nsub; ++sub)
+    if (sub_has_keys(j, own, t, sub, g)) atomicAdd(&counts[(bg * g.nb + j) * g.nsub + sub], 1);
+}
+
+// Single-CTA exclusive scans: seg_off (entries), tile_off (tiles of tpt entries).
+__global__ void __launch_bounds__(1024)
+invert_scan_kernel(const int* __restrict__ counts, int* __restrict__ seg_off,
+                   int* __restrict__ cursor, int* __restrict__ tile_off, int* __restrict__ n_tiles,
+                   int64_t nseg, int tpt) {
+  __shared__ long long s_e[1024], s_t[1024];
+  const int tid = threadIdx.x;
+  const int64_t per = (nseg + 1023) / 1024;
+  const int64_t lo = tid * per, hi = lo + per < nseg ? lo + per : nseg;
+  long long se = 0, st = 0;
+  for (int64_t i = lo; i < hi; ++i) { se += counts[i]; st += (counts[i] + tpt - 1) / tpt; }
+  s_e[tid] = se; s_t[tid] = st;
+  __syncthreads();
+  for (int off = 1; off < 1024; off <<= 1) {     // Hillis-Steele inclusive scan
+    long long a = tid >= off ? s_e[tid - off] : 0, b = tid >= off ? s_t[tid - off] : 0;
+    __syncthreads();
+    s_e[tid] += a; s_t[tid] += b;
+    __syncthreads();
+  }
+  long long ce = s_e[tid] - se, ct = s_t[tid] - st;
+  for (int64_t i = lo; i < hi; ++i) {
+    seg_off[i] = (int)ce; cursor[i] = (int)ce; tile_off[i] = (int)ct;
+    ce += counts[i]; ct += (counts[i] + tpt - 1) / tpt;
+  }
+  if (tid == 1023) { seg_off[nseg] = (int)s_e[1023]; tile_off[nseg] = (int)s_t[1023];
+                     *n_tiles = (int)s_t[1023]; }
+}
+
+__global__ void invert_fill_kernel(const int32_t* __restrict__ idx, int* __restrict__ cursor,
+                                   int* __restrict__ entries, Geom g, int64_t n) {
+  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= n) return;
+  const int slot = (int)(e % g.topk);
+  const int64_t row = e / g.topk;
+  const int64_t t = row % g.S, bg = row / g.S;
+  const int64_t j = idx[e];
+  if (j < 0 || j >= g.nb) return;
+  const int64_t own = t / g.block;
+  if (j > own) return;
+  for (int sub = 0; sub < g.nsub; ++sub)
+    if (sub_has_keys(j, own, t, sub, g)) {
+      const int pos = atomicAdd(&cursor[(bg * g.nb + j) * g.nsub + sub], 1);
+      entries[pos] = (int)((t << 6) | (slot * g.nsub + sub));
+    }
+}
+
+__global__ void tile_table_kernel(const int* __restrict__ counts, const int* __restrict__ seg_off,
+                                  const int* __restrict__ tile_off,
+                                  const int* __restrict__ n_tiles, int4* __restrict__ tiles,
+                                  int64_t nseg, int tpt) {
+  const int64_t tile = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (tile >= *n_tiles) return;
+  int64_t lo = 0, hi = nseg;                     // largest s with tile_off[s] <= tile
+  while (hi - lo > 1) {
+    const int64_t mid = (lo + hi) / 2;
+    if (tile_off[mid] <= tile) lo = mid; else hi = mid;
+  }
+  while (lo + 1 < nseg && tile_off[lo + 1] <= tile) ++lo;   // skip empty segments
+  const int k = (int)(tile - tile_off[lo]);
+  const int cnt = min(tpt, counts[lo] - k * tpt);
+  tiles[tile] = make_int4((int)lo, seg_off[lo] + k * tpt, cnt, 0);
+}
+
+// ------------------------------------------------------------------ the tile kernel
+struct __align__(8) Bars {
+  uint64_t q_full[2], q_empty[2], kv_full, s_full[2], p_full[2], o_full, o_empty;
+  uint32_t tmem_base;
+  int abort;
+};
+
+template <int G>
+__global__ void __launch_bounds__(kThreads, 1)
+attn_tiles_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                  const __nv_bfloat16* __restrict__ q, const int4* __restrict__ tiles,
+                  const int* __restrict__ n_tiles_p, const int* __restrict__ entries,
+                  __nv_bfloat16* __restrict__ po, float* __restrict__ plse, int* err, Geom g) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* base = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* Qs = base;                                   // 2 stages x 32 KB
+  unsigned char* Ks = base + 2 * 2 * kTileBytes;              // nch x 2 halves x 16 KB
+  unsigned char* Vs = Ks + g.nch * 2 * kTileBytes;
+  Bars* bars = reinterpret_cast<Bars*>(Vs + g.nch * 2 * kTileBytes);
+
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const int n_tiles = *n_tiles_p;
+  const int per = (n_tiles + gridDim.x - 1) / gridDim.x;
+  const int tile_lo = blockIdx.x * per;
+  const int tile_hi = min(n_tiles, tile_lo + per);
+  const int my_tiles = max(0, tile_hi - tile_lo);
+
+  if (tid == 0) {
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars->q_full[s], kGatherThreads);
+      mbar_init(&bars->q_empty[s], 1);
+      mbar_init(&bars->s_full[s], 1);
+      mbar_init(&bars->p_full[s], 128);
+    }
+    mbar_init(&bars->kv_full, 1);
+    mbar_init(&bars->o_full, 1);
+    mbar_init(&bars->o_empty, 128);
+    bars->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) { tmem_alloc(&bars->tmem_base, 512); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  volatile int* abort_flag = &bars->abort;
+
+  auto fail = [&]() {
+    set_device_error(err, MSA_DEVERR_TIMEOUT);
+    *abort_flag = 1;
+  };
+
+  if (warp == 4) {
+    // ---------------------------------------------------------------- issuer
+    if (lane == 0 && my_tiles > 0) {
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      const uint32_t idS = idesc_bf16(128, kChunkKeys, 0, 0);
+      const uint32_t idO = idesc_bf16(128, kD, 0, 1);
+      int prev_seg = -1;
+      uint32_t kvn = 0;
+      for (int n = 0; n < my_tiles; ++n) {
+        if (*abort_flag) break;
+        const int4 tl = tiles[tile_lo + n];
+        if (n > 0 && !mbar_wait(&bars->o_full, (n - 1) & 1)) { fail(); break; }
+        if (tl.x != prev_seg) {
+          const int64_t seg = tl.x;
+          const int sub = (int)(seg % g.nsub);
+          const int64_t j = (seg / g.nsub) % g.nb;
+          const int64_t gg = (seg / ((int64_t)g.nsub * g.nb)) % g.hkv;
+          const int64_t b = seg / ((int64_t)g.nsub * g.nb * g.hkv);
+          const int y0 = (int)(b * g.S + j * g.block + (int64_t)sub * kSegKeys);
+          mbar_arrive_expect_tx(&bars->kv_full, (uint32_t)(g.nch * 4 * kTileBytes));
+          for (int c = 0; c < g.nch; ++c)
+            for (int hf = 0; hf < 2; ++hf) {
+              const int x = (int)(gg * kD + hf * 64);
+              tma_load_2d(Ks + (c * 2 + hf) * kTileBytes, &tmK, &bars->kv_full, x,
+                          y0 + c * kChunkKeys);
+              tma_load_2d(Vs + (c * 2 + hf) * kTileBytes, &tmV, &bars->kv_full, x,
+                          y0 + c * kChunkKeys);
+            }
+          if (!mbar_wait(&bars->kv_full, kvn & 1)) { fail(); break; }
+          ++kvn;
+          prev_seg = tl.x;
+        }
+        const int st = n & 1;
+        if (!mbar_wait(&bars->q_full[st], (n >> 1) & 1)) { fail(); break; }
+        tc_fence_after();
+        const uint32_t qa = smem_u32(Qs + st * 2 * kTileBytes);
+        for (int c = 0; c < g.nch; ++c) {
+          const uint32_t ka = smem_u32(Ks + c * 2 * kTileBytes);
+          for (int s = 0; s < kD / 16; ++s) {
+            const uint32_t off = (uint32_t)(s >> 2) * kTileBytes + (uint32_t)(s & 3) * 32;
+            umma_ss(tmem + c * kChunkKeys, sdesc_sw128(qa + off, 16, 1024),
+                    sdesc_sw128(ka + off, 16, 1024), idS, s > 0);
+          }
+          umma_commit(&bars->s_full[c]);
+        }
+        umma_commit(&bars->q_empty[st]);
+        if (n > 0 && !mbar_wait(&bars->o_empty, (n - 1) & 1)) { fail(); break; }
+        for (int c = 0; c < g.nch; ++c) {
+          if (!mbar_wait(&bars->p_full[c], n & 1)) { fail(); break; }
+          tc_fence_after();
+          const uint32_t va = smem_u32(Vs + c * 2 * kTileBytes);
+          for (int s = 0; s < kChunkKeys / 16; ++s)
+            umma_ts(tmem + 256 + c * kD, tmem + c * kChunkKeys + s * 8,
+                    sdesc_sw128(va + s * 2048, kTileBytes, 1024), idO, s > 0);
+        }
+        if (*abort_flag) break;
+        umma_commit(&bars->o_full);
+      }
+    }
+  } else if (warp >= 5) {
+    // ---------------------------------------------------------------- Q gather
+    const int gt = tid - 160;
+    for (int n = 0; n < my_tiles; ++n) {
+      if (*abort_flag) break;
+      const int st = n & 1;
+      if (n >= 2 && !mbar_wait(&bars->q_empty[st], ((n >> 1) - 1) & 1)) { fail(); break; }
+      const int4 tl = tiles[tile_lo + n];
+      const int64_t seg = tl.x;
+      const int64_t gg = (seg / ((int64_t)g.nsub * g.nb)) % g.hkv;
+      const int64_t b = seg / ((int64_t)g.nsub * g.nb * g.hkv);
+      unsigned char* qb = Qs + st * 2 * kTileBytes;
+      for (int i = gt; i < kRowsT * 16; i += kGatherThreads) {
+        const int r = i >> 4, c = i & 15;
+        const int tok = r / G, h = r % G;
+        const bool valid = tok < tl.z;
+        const int64_t t = valid ? (int64_t)(entries[tl.y + tok] >> 6) : 0;
+        const __nv_bfloat16* src =
+            q + (((b * g.S + t) * g.hq + gg * G + h) * kD + c * 8);
+        cp_async16(qb + (c >> 3) * kTileBytes + r * 128 + (((c & 7) ^ (r & 7)) << 4),
+                   valid ? src : q, valid);
+      }
+      cp_async_wait_all();
+      fence_proxy_async_smem();
+      mbar_arrive(&bars->q_full[st]);
+    }
+  } else {
+    // ---------------------------------------------------------------- softmax + epilogue
+    const int r = tid;                                   // TMEM lane = tile row
+    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    const int tok = r / G, h = r % G;
+    for (int n = 0; n < my_tiles; ++n) {
+      if (*abort_flag) break;
+      const int4 tl = tiles[tile_lo + n];
+      const int64_t seg = tl.x;
+      const int sub = (int)(seg % g.nsub);
+      const int64_t j = (seg / g.nsub) % g.nb;
+      const int64_t gg = (seg / ((int64_t)g.nsub * g.nb)) % g.hkv;
+      const int64_t b = seg / ((int64_t)g.nsub * g.nb * g.hkv);
+      const bool valid = tok < tl.z;
+      int64_t t = 0;
+      int pslot = 0;
+      if (valid) {
+        const int e = entries[tl.y + tok];
+        t = e >> 6;
+        pslot = e & 63;
+      }
+      const int64_t own = t / g.block;
+      const int64_t kbase = j * g.block + (int64_t)sub * kSegKeys;
+      int64_t khi = (j == own) ? t + 1 : j * g.block + g.block;
+      const int64_t seg_end = j * g.block + min((int64_t)(sub + 1) * kSegKeys, g.block);
+      khi = min(min(khi, seg_end), g.S);
+      float m_c[2] = {-CUDART_INF_F, -CUDART_INF_F}, l_c[2] = {0.f, 0.f};
+      bool ok = true;
+      for (int c = 0; c < g.nch; ++c) {
+        const int64_t rem = khi - (kbase + (int64_t)c * kChunkKeys);
+        const int lim = valid ? (int)max((int64_t)0, min((int64_t)kChunkKeys, rem)) : 0;
+        if (!mbar_wait(&bars->s_full[c], n & 1)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t sv[4][32];
+#pragma unroll
+        for (int qd = 0; qd < 4; ++qd) tmem_ld32(lane_base + c * kChunkKeys + qd * 32, sv[qd]);
+        tmem_ld_wait();
+        float mx = -CUDART_INF_F;
+#pragma unroll
+        for (int qd = 0; qd < 4; ++qd)
+#pragma unroll
+          for (int k = 0; k < 32; ++k)
+            if (qd * 32 + k < lim) mx = fmaxf(mx, __uint_as_float(sv[qd][k]) * g.scale_log2);
+        // P packed two bf16 per 32-bit column, written in place over the consumed scores:
+        // chunk quarter qd lands in sv[qd / 2][(qd % 2) * 16 ...], already read.
+        float sum = 0.f;
+#pragma unroll
+        for (int qd = 0; qd < 4; ++qd)
+#pragma unroll
+          for (int k = 0; k < 32; k += 2) {
+            const int kk = qd * 32 + k;
+            const float p0 = kk < lim ? exp2f(__uint_as_float(sv[qd][k]) * g.scale_log2 - mx) : 0.f;
+            const float p1 =
+                kk + 1 < lim ? exp2f(__uint_as_float(sv[qd][k + 1]) * g.scale_log2 - mx) : 0.f;
+            sum += p0 + p1;
+            sv[qd >> 1][(qd & 1) * 16 + k / 2] = pack_bf16x2(p0, p1);
+          }
+        tmem_st32(lane_base + c * kChunkKeys, sv[0]);
+        tmem_st32(lane_base + c * kChunkKeys + 32, sv[1]);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&bars->p_full[c]);
+        m_c[c] = mx;
+        l_c[c] = sum;
+      }
+      if (!ok || !mbar_wait(&bars->o_full, n & 1)) { fail(); break; }
+      tc_fence_after();
+      const float M = fmaxf(m_c[0], m_c[1]);
+      float w[2];
+#pragma unroll
+      for (int c = 0; c < 2; ++c) w[c] = (c < g.nch && m_c[c] > -CUDART_INF_F) ? exp2f(m_c[c] - M) : 0.f;
+      const float L = w[0] * l_c[0] + w[1] * l_c[1];
+      const float inv = L > 0.f ? 1.f / L : 0.f;
+      __nv_bfloat16* dst = po + ((((b * g.hkv + gg) * g.S + t) * g.kslots + pslot) * G + h) * kD;
+#pragma unroll 1
+      for (int qd = 0; qd < 4; ++qd) {
+        uint32_t o0[32], o1[32];
+        tmem_ld32(lane_base + 256 + qd * 32, o0);
+        if (g.nch > 1) tmem_ld32(lane_base + 384 + qd * 32, o1);
+        tmem_ld_wait();
+        uint32_t ob[16];
+#pragma unroll
+        for (int k = 0; k < 32; k += 2) {
+          float a0 = __uint_as_float(o0[k]) * w[0], a1 = __uint_as_float(o0[k + 1]) * w[0];
+          if (g.nch > 1) {
+            a0 = fmaf(__uint_as_float(o1[k]), w[1], a0);
+            a1 = fmaf(__uint_as_float(o1[k + 1]), w[1], a1);
+          }
+          ob[k / 2] = pack_bf16x2(a0 * inv, a1 * inv);
+        }
+        if (valid) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst + qd * 32);
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            d4[v] = make_uint4(ob[v * 4], ob[v * 4 + 1], ob[v * 4 + 2], ob[v * 4 + 3]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&bars->o_empty);
+      if (valid)
+        plse[(((b * g.hkv + gg) * g.S + t) * g.kslots + pslot) * G + h] =
+            L > 0.f ? (M + log2f(L)) * kLn2 : -CUDART_INF_F;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------ merge partials
+// One row = (sequence, group, token); G*16 threads per row, 8 output elements each.
+template <int G>
+__global__ void merge_partials_kernel(const int32_t* __restrict__ idx,
+                                      const __nv_bfloat16* __restrict__ po,
+                                      const float* __restrict__ plse, __nv_bfloat16* __restrict__ o,
+                                      float* __restrict__ lse, Geom g, int64_t n_rows) {
+  constexpr int TPR = G * 16;
+  constexpr int RPC = 128 / TPR;
+  const int64_t row = (int64_t)blockIdx.x * RPC + threadIdx.x / TPR;
+  if (row >= n_rows) return;
+  const int lt = threadIdx.x % TPR;
+  const int h = lt / 16;
+  const int64_t t = row % g.S, bg = row / g.S;
+  const int64_t gg = bg % g.hkv, b = bg / g.hkv;
+  const int64_t own = t / g.block;
+  const int32_t* irow = idx + row * g.topk;
+  const float* lrow = plse + row * g.kslots * G;
+  const __nv_bfloat16* prow = po + row * g.kslots * G * kD;
+  float mx = -CUDART_INF_F;
+  for (int s = 0; s < g.topk; ++s) {
+    const int64_t j = irow[s];
+    if (j < 0 || j >= g.nb || j > own) continue;
+    for (int sub = 0; sub < g.nsub; ++sub)
+      if (sub_has_keys(j, own, t, sub, g)) mx = fmaxf(mx, lrow[(s * g.nsub + sub) * G + h]);
+  }
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  float den = 0.f;
+  if (mx > -CUDART_INF_F) {
+    for (int s = 0; s < g.topk; ++s) {
+      const int64_t j = irow[s];
+      if (j < 0 || j >= g.nb || j > own) continue;
+      for (int sub = 0; sub < g.nsub; ++sub) {
+        if (!sub_has_keys(j, own, t, sub, g)) continue;
+        const int ps = s * g.nsub + sub;
+        const float lv = lrow[ps * G + h];
+        if (!(lv > -CUDART_INF_F)) continue;
+        const float wgt = exp2f((lv - mx) * kLog2e);
+        den += wgt;
+        float f[8];
+        Vec16<__nv_bfloat16>::unpack(ldg16(prow + (int64_t)ps * G * kD + lt * 8), f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = fmaf(wgt, f[e], acc[e]);
+      }
+    }
+  }
+  const float inv = den > 0.f ? 1.f / den : 0.f;
+  uint4 out;
+  out.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+  out.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
+  out.z = pack_bf16x2(acc[4] * inv, acc[5] * inv);
+  out.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
+  *reinterpret_cast<uint4*>(o + ((b * g.S + t) * g.hq + gg * G) * kD + lt * 8) = out;
+  if (lse != nullptr && (lt % 16) == 0)
+    lse[(b * g.hq + gg * G + h) * g.S + t] = den > 0.f ? mx + logf(den) : -CUDART_INF_F;
+}
+
+// ------------------------------------------------------------------ host side
+struct WsLayout {
+  size_t counts, seg_off, cursor, tile_off, n_tiles, entries, tiles, po, plse, total;
+};
+
+size_t up256(size_t x) { return (x + 255) / 256 * 256; }
+
+Geom make_geom(const Shape& s) {
+  Geom g{};
+  g.S = s.seq; g.nb = s.nb; g.block = s.block;
+  g.hq = (int)s.hq; g.hkv = (int)s.hkv; g.G = (int)(s.hq / s.hkv); g.topk = (int)s.topk;
+  g.nsub = (int)((s.block + kSegKeys - 1) / kSegKeys);
+  g.kslots = g.topk * g.nsub;
+  g.tpt = kRowsT / g.G;
+  g.nch = (int)(((s.block < kSegKeys ? s.block : (int64_t)kSegKeys) + kChunkKeys - 1) / kChunkKeys);
+  g.nseg = s.batch * s.hkv * s.nb * g.nsub;
+  g.scale_log2 = s.scale * kLog2e;
+  return g;
+}
+
+WsLayout layout_for(const Shape& s) {
+  const Geom g = make_geom(s);
+  const int64_t n_sel = s.batch * s.hkv * s.seq * s.topk;
+  const int64_t n_entries = n_sel * g.nsub;
+  const int64_t n_tiles_max = n_entries / g.tpt + g.nseg + 1;
+  const int64_t rows = s.batch * s.hkv * s.seq;
+  WsLayout L{};
+  size_t o = 0;
+  L.counts = o;   o += up256(g.nseg * 4);
+  L.seg_off = o;  o += up256((g.nseg + 1) * 4);
+  L.cursor = o;   o += up256(g.nseg * 4);
+  L.tile_off = o; o += up256((g.nseg + 1) * 4);
+  L.n_tiles = o;  o += 256;
+  L.entries = o;  o += up256(n_entries * 4);
+  L.tiles = o;    o += up256(n_tiles_max * 16);
+  L.po = o;       o += up256((size_t)rows * g.kslots * g.G * kD * 2);
+  L.plse = o;     o += up256((size_t)rows * g.kslots * g.G * 4);
+  L.total = o;
+  return L;
+}
+
+template <int G>
+cudaError_t run_tc(const Shape& s, const Geom& g, const CUtensorMap& mk, const CUtensorMap& mv,
+                   const void* q, const int32_t* idx, void* o, float* lse, char* ws,
+                   const WsLayout& L, int* err, cudaStream_t st) {
+  const size_t smem = 1024 + 2 * 2 * kTileBytes + (size_t)g.nch * 4 * kTileBytes + sizeof(Bars);
+  cudaError_t e = cudaFuncSetAttribute(attn_tiles_kernel<G>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  attn_tiles_kernel<G><<<sm_count(), kThreads, smem, st>>>(
+      mk, mv, (const __nv_bfloat16*)q, (const int4*)(ws + L.tiles), (const int*)(ws + L.n_tiles),
+      (const int*)(ws + L.entries), (__nv_bfloat16*)(ws + L.po), (float*)(ws + L.plse), err, g);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const int64_t rows = s.batch * s.hkv * s.seq;
+  const int rpc = 128 / (G * 16);
+  merge_partials_kernel<G><<<(unsigned)((rows + rpc - 1) / rpc), 128, 0, st>>>(
+      idx, (const __nv_bfloat16*)(ws + L.po), (const float*)(ws + L.plse), (__nv_bfloat16*)o,
+      lse, g, rows);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool tc_attn_supported(const Shape& s) {
+  if (s.dtype != MSA_BF16 || s.d != kD) return false;
+  if (s.block % kChunkKeys != 0) return false;
+  if (s.block > kSegKeys && s.block % kSegKeys != 0) return false;
+  const int64_t G = s.hq / s.hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return false;
+  const int64_t nsub = (s.block + kSegKeys - 1) / kSegKeys;
+  if (s.topk * nsub > 64) return false;                       // pslot fits 6 bits
+  if (s.seq >= ((int64_t)1 << 25)) return false;              // token fits 25 bits
+  if (s.batch * s.hkv * s.seq * s.topk * nsub >= ((int64_t)1 << 31)) return false;
+  if (s.batch * s.seq >= ((int64_t)1 << 31)) return false;    // TMA row coordinate
+  return true;
+}
+
+size_t tc_attn_ws_bytes(const Shape& s) { return layout_for(s).total; }
+
+cudaError_t launch_attn_prefill_tc(const Shape& s, const void* q, const void* k, const void* v,
+                                   const int32_t* idx, void* o, float* lse, void* ws_body,
+                                   int* err, cudaStream_t st) {
+  const Geom g = make_geom(s);
+  const WsLayout L = layout_for(s);
+  char* ws = reinterpret_cast<char*>(ws_body);
+  CUtensorMap mk, mv;
+  if (!make_bf16_2d_map(&mk, k, s.batch * s.seq, s.hkv * kD, 128) ||
+      !make_bf16_2d_map(&mv, v, s.batch * s.seq, s.hkv * kD, 128))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaMemsetAsync(ws + L.counts, 0, g.nseg * 4, st);
+  if (e != cudaSuccess) return e;
+  const int64_t n_sel = s.batch * s.hkv * s.seq * s.topk;
+  const unsigned gb = (unsigned)((n_sel + 255) / 256);
+  invert_count_kernel<<<gb, 256, 0, st>>>(idx, (int*)(ws + L.counts), err, g, n_sel);
+  invert_scan_kernel<<<1, 1024, 0, st>>>((const int*)(ws + L.counts), (int*)(ws + L.seg_off),
+                                         (int*)(ws + L.cursor), (int*)(ws + L.tile_off),
+                                         (int*)(ws + L.n_tiles), g.nseg, g.tpt);
+  invert_fill_kernel<<<gb, 256, 0, st>>>(idx, (int*)(ws + L.cursor), (int*)(ws + L.entries), g,
+                                         n_sel);
+  const int64_t n_tiles_max = n_sel * g.nsub / g.tpt + g.nseg + 1;
+  tile_table_kernel<<<(unsigned)((n_tiles_max + 255) / 256), 256, 0, st>>>(
+      (const int*)(ws + L.counts), (const int*)(ws + L.seg_off), (const int*)(ws + L.tile_off),
+      (const int*)(ws + L.n_tiles), (int4*)(ws + L.tiles), g.nseg, g.tpt);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  switch (g.G) {
+    case 1: return run_tc<1>(s, g, mk, mv, q, idx, o, lse, ws, L, err, st);
+    case 2: return run_tc<2>(s, g, mk, mv, q, idx, o, lse, ws, L, err, st);
+    case 4: return run_tc<4>(s, g, mk, mv, q, idx, o, lse, ws, L, err, st);
+    default: return run_tc<8>(s, g, mk, mv, q, idx, o, lse, ws, L, err, st);
+  }
+}
+
+}  // namespace msa

@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -107,5 +108,23 @@ cudaError_t launch_attn_prefill_rows(const Shape& s, const void* q, const void* 
 cudaError_t launch_attn_decode(const Shape& s, int64_t n_query, const void* q, const void* k,
                                const void* v, const int32_t* idx, void* o, float* lse, void* ws,
                                int* err, cudaStream_t st);
+
+// Host helpers (host_util.cu): a 2-D bf16 TMA map over a row-major [rows, cols] tensor
+// with 64-column x box_rows boxes and 128-byte swizzle; the device's SM count.
+bool make_bf16_2d_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_rows);
+int sm_count();
+
+// Tensor-core prefill selection (bf16, d = 128); see topk_tc.cu.  Needs the pooled keys'
+// bf16 hi/lo planes.
+bool tc_topk_supported(const Shape& s);
+cudaError_t launch_topk_prefill_tc(const Shape& s, const void* q, const void* kbar_hi,
+                                   const void* kbar_lo, int32_t* idx, int* err, cudaStream_t st);
+
+// Key-centric tensor-core attention (bf16, d = 128); see attn_tc.cu.
+bool tc_attn_supported(const Shape& s);
+size_t tc_attn_ws_bytes(const Shape& s);
+cudaError_t launch_attn_prefill_tc(const Shape& s, const void* q, const void* k, const void* v,
+                                   const int32_t* idx, void* o, float* lse, void* ws_body,
+                                   int* err, cudaStream_t st);
 
 }  // namespace msa

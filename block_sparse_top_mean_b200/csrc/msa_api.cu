@@ -15,6 +15,8 @@ constexpr int64_t kMaxElems = (int64_t)1 << 40;   // guards every size product b
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
 size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+int* err_word(void* ws) { return reinterpret_cast<int*>(ws); }
+char* ws_body(void* ws) { return reinterpret_cast<char*>(ws) + msa::kWsHeader; }
 
 // Shape checks shared by every entry point.  `bank` = decode (seq is bank tokens).
 msa_status check_params(const msa_params* p, bool bank, Shape* s) {
@@ -44,14 +46,20 @@ msa_status check_params(const msa_params* p, bool bank, Shape* s) {
 bool empty_prefill(const Shape& s) { return s.batch == 0 || s.seq == 0; }
 
 size_t kbar_bytes(const Shape& s) { return (size_t)s.batch * s.nb * s.hkv * s.d * sizeof(float); }
+// bf16 hi or lo plane of the pooled keys; only the tensor-core selection uses them.
+size_t kbar_split_bytes(const Shape& s) {
+  return msa::tc_topk_supported(s) ? (size_t)s.batch * s.nb * s.hkv * s.d * 2 : 0;
+}
 
 size_t ws_bytes_for(const Shape& s, int op, int64_t n_query) {
   switch (op) {
     case MSA_OP_TOPK_SELECT:
-    case MSA_OP_SPARSE_ATTN:
       return msa::kWsHeader;
+    case MSA_OP_SPARSE_ATTN:
+      return msa::kWsHeader + (msa::tc_attn_supported(s) ? round256(msa::tc_attn_ws_bytes(s)) : 0);
     case MSA_OP_PREFILL:
-      return msa::kWsHeader + round256(kbar_bytes(s));
+      return msa::kWsHeader + round256(kbar_bytes(s)) + 2 * round256(kbar_split_bytes(s)) +
+             (msa::tc_attn_supported(s) ? round256(msa::tc_attn_ws_bytes(s)) : 0);
     case MSA_OP_DECODE:
       return msa::kWsHeader + round256(msa::decode_select_ws_bytes(s, n_query)) +
              round256(msa::decode_attn_ws_bytes(s, n_query));
@@ -68,8 +76,26 @@ msa_status check_ws(const Shape& s, int op, int64_t n_query, const void* ws, siz
 
 msa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MSA_OK : MSA_ERR_CUDA; }
 
-int* err_word(void* ws) { return reinterpret_cast<int*>(ws); }
-char* ws_body(void* ws) { return reinterpret_cast<char*>(ws) + msa::kWsHeader; }
+// bf16 with d = 128 and the split planes present runs the tensor-core selection;
+// otherwise the fp32 SIMT one.
+cudaError_t launch_selection(const Shape& s, const void* q, const float* kbar,
+                             const void* kbar_hi, const void* kbar_lo, int32_t* idx, int* err,
+                             cudaStream_t st) {
+  if (kbar_hi != nullptr && kbar_lo != nullptr && msa::tc_topk_supported(s))
+    return msa::launch_topk_prefill_tc(s, q, kbar_hi, kbar_lo, idx, err, st);
+  return msa::launch_topk_prefill(s, q, kbar, idx, st);
+}
+
+// bf16 with d = 128 and 128-multiple blocks runs on the tensor cores (key-centric tiles);
+// everything else on the query-centric SIMT kernel.
+cudaError_t launch_attention(const Shape& s, const void* q, const void* k, const void* v,
+                             const int32_t* idx, void* o, float* lse, char* scratch, int* err,
+                             cudaStream_t st) {
+  if (msa::tc_attn_supported(s))
+    return msa::launch_attn_prefill_tc(s, q, k, v, idx, o, lse, scratch, err, st);
+  return msa::launch_attn_prefill_rows(s, q, k, v, idx, o, lse, err, st);
+}
+
 
 }  // namespace
 
@@ -126,15 +152,17 @@ msa_status msa_block_scores(const msa_params* p, const void* q, const float* kba
 msa_status msa_topk_select(const msa_params* p, const void* q, const float* kbar,
                            const void* kbar_hi, const void* kbar_lo, int32_t* idx, void* ws,
                            size_t ws_bytes, msa_stream_t stream) {
-  (void)kbar_hi; (void)kbar_lo;
   Shape s;
   msa_status st = check_params(p, false, &s);
   if (st != MSA_OK) return st;
   if (empty_prefill(s)) return MSA_OK;
   if (q == nullptr || kbar == nullptr || idx == nullptr || !aligned16(q) || !aligned16(kbar))
     return MSA_ERR_INVALID_ARG;
+  if ((kbar_hi != nullptr && !aligned16(kbar_hi)) || (kbar_lo != nullptr && !aligned16(kbar_lo)))
+    return MSA_ERR_INVALID_ARG;
   if ((st = check_ws(s, MSA_OP_TOPK_SELECT, 0, ws, ws_bytes)) != MSA_OK) return st;
-  return cuda_status(msa::launch_topk_prefill(s, q, kbar, idx, (cudaStream_t)stream));
+  return cuda_status(launch_selection(s, q, kbar, kbar_hi, kbar_lo, idx, err_word(ws),
+                                      (cudaStream_t)stream));
 }
 
 msa_status msa_sparse_attn_fwd(const msa_params* p, const void* q, const void* k, const void* v,
@@ -148,8 +176,8 @@ msa_status msa_sparse_attn_fwd(const msa_params* p, const void* q, const void* k
     return MSA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return MSA_ERR_INVALID_ARG;
   if ((st = check_ws(s, MSA_OP_SPARSE_ATTN, 0, ws, ws_bytes)) != MSA_OK) return st;
-  return cuda_status(msa::launch_attn_prefill_rows(s, q, k, v, idx, o, lse, err_word(ws),
-                                                   (cudaStream_t)stream));
+  return cuda_status(launch_attention(s, q, k, v, idx, o, lse, ws_body(ws), err_word(ws),
+                                      (cudaStream_t)stream));
 }
 
 msa_status msa_prefill_fwd(const msa_params* p, const void* q, const void* k, const void* v,
@@ -164,10 +192,19 @@ msa_status msa_prefill_fwd(const msa_params* p, const void* q, const void* k, co
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return MSA_ERR_INVALID_ARG;
   if ((st = check_ws(s, MSA_OP_PREFILL, 0, ws, ws_bytes)) != MSA_OK) return st;
   cudaStream_t cs = (cudaStream_t)stream;
-  float* kbar = reinterpret_cast<float*>(ws_body(ws));
-  cudaError_t e = msa::launch_pool_keys(s, k, kbar, nullptr, nullptr, s.batch, cs);
-  if (e == cudaSuccess) e = msa::launch_topk_prefill(s, q, kbar, idx, cs);
-  if (e == cudaSuccess) e = msa::launch_attn_prefill_rows(s, q, k, v, idx, o, lse, err_word(ws), cs);
+  char* body = ws_body(ws);
+  float* kbar = reinterpret_cast<float*>(body);
+  void* hi = nullptr;
+  void* lo = nullptr;
+  size_t off = round256(kbar_bytes(s));
+  if (kbar_split_bytes(s) > 0) {
+    hi = body + off;
+    lo = body + off + round256(kbar_split_bytes(s));
+    off += 2 * round256(kbar_split_bytes(s));
+  }
+  cudaError_t e = msa::launch_pool_keys(s, k, kbar, hi, lo, s.batch, cs);
+  if (e == cudaSuccess) e = launch_selection(s, q, kbar, hi, lo, idx, err_word(ws), cs);
+  if (e == cudaSuccess) e = launch_attention(s, q, k, v, idx, o, lse, body + off, err_word(ws), cs);
   return cuda_status(e);
 }
 

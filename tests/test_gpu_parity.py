@@ -41,6 +41,10 @@ SMALL = [
     mi.Workload("f32_one_partial_block", "prefill", 1, 50, 2, 1, 64, 64, 4, "f32"),
     mi.Workload("bf16_planted", "prefill", 1, 4096, 8, 2, 128, 128, 8, "bf16",
                 planted_frac=0.02, planted_shift=3.0),
+    mi.Workload("bf16_g8_b256", "prefill", 1, 2500, 16, 2, 128, 256, 5, "bf16"),
+    mi.Workload("bf16_g1_b128", "prefill", 1, 1500, 4, 4, 128, 128, 4, "bf16"),
+    mi.Workload("bf16_batch2_g2", "prefill", 2, 1000, 4, 2, 128, 128, 3, "bf16"),
+    mi.Workload("bf16_b384_ragged", "prefill", 1, 2000, 8, 2, 128, 384, 4, "bf16"),
 ]
 
 
@@ -100,6 +104,30 @@ def test_topk_select_and_attn_separately(msa, w):
         oidx[0, r.g, r.t] = torch.tensor(r.idx)
     o, lse = msa.sparse_attn_fwd(q, k, v, oidx, w.block, w.scale)
     check_prefill(q, k, v, w.block, w.topk, w.scale, oidx, o, lse, rows=rows)
+
+
+@pytest.mark.parametrize("w", [SMALL[1], SMALL[2], SMALL[3], SMALL[9], SMALL[10], SMALL[11],
+                               SMALL[12]], ids=lambda w: w.name)
+def test_topk_select_split_planes_vs_oracle(msa, w):
+    """The selection fed the bf16 hi/lo planes (tensor-core path for bf16, d = 128)."""
+    q, k, v = _inputs(w)
+    kbar, hi, lo = msa.pool_keys(k, w.block, split=True)
+    idx = msa.topk_select(q, kbar, w.block, w.topk, w.hkv, kbar_hi=hi, kbar_lo=lo)
+    torch.cuda.synchronize()
+    Q, K, V = HostView(q), HostView(k), HostView(v)
+    kb = oracle.pool_keys(k.float().cpu().numpy(), w.block)
+    rows = [(b, t) for b in range(w.batch) for t in range(0, w.seq, 3)]
+    gi = idx.cpu().numpy()
+    n_strict = 0
+    for r in oracle.prefill_rows(Q, K, V, w.block, w.topk, w.scale, rows=rows, kbar=kb):
+        sel = [int(x) for x in gi[r.b, r.g, r.t]]
+        if r.gap > 1e-3:
+            n_strict += 1
+            assert sel == r.idx, (r.t, r.g, sel, r.idx)
+        else:
+            s = [j for j in sel if j >= 0]
+            assert r.t // w.block in s and max(s) == r.t // w.block
+    assert n_strict > 0
 
 
 def test_out_of_range_index_sets_error_word_and_skips(msa):
