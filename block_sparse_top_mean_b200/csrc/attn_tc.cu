@@ -137,7 +137,14 @@ struct __align__(8) Bars {
   uint64_t q_full[2], q_empty[2], kv_full, s_full[2], p_full[2], o_full, o_empty;
   uint32_t tmem_base;
   int abort;
+  int tok[2][kRowsT];          // per Q stage: token of each tile slot (gather warps only)
 };
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 template <int G>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -249,23 +256,30 @@ attn_tiles_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
     // ---------------------------------------------------------------- Q gather
     const int gt = tid - 160;
     for (int n = 0; n < my_tiles; ++n) {
-      if (*abort_flag) break;
       const int st = n & 1;
-      if (n >= 2 && !mbar_wait(&bars->q_empty[st], ((n >> 1) - 1) & 1)) { fail(); break; }
+      bool bad = *abort_flag != 0;
+      if (!bad && n >= 2 && !mbar_wait(&bars->q_empty[st], ((n >> 1) - 1) & 1)) {
+        fail();
+        bad = true;
+      }
       const int4 tl = tiles[tile_lo + n];
       const int64_t seg = tl.x;
       const int64_t gg = (seg / ((int64_t)g.nsub * g.nb)) % g.hkv;
       const int64_t b = seg / ((int64_t)g.nsub * g.nb * g.hkv);
       unsigned char* qb = Qs + st * 2 * kTileBytes;
+      int* tk = bars->tok[st];
+      for (int i = gt; i < kRowsT / G; i += kGatherThreads)
+        tk[i] = i < tl.z ? (entries[tl.y + i] >> 6) : -1;
+      // all gather threads leave together: the token list is complete, or all abort
+      if (bar_sync_or<1, kGatherThreads>(bad)) break;
+      const __nv_bfloat16* qbase = q + (b * g.S * g.hq + gg * G) * kD;
+#pragma unroll 4
       for (int i = gt; i < kRowsT * 16; i += kGatherThreads) {
         const int r = i >> 4, c = i & 15;
-        const int tok = r / G, h = r % G;
-        const bool valid = tok < tl.z;
-        const int64_t t = valid ? (int64_t)(entries[tl.y + tok] >> 6) : 0;
-        const __nv_bfloat16* src =
-            q + (((b * g.S + t) * g.hq + gg * G + h) * kD + c * 8);
-        cp_async16(qb + (c >> 3) * kTileBytes + r * 128 + (((c & 7) ^ (r & 7)) << 4),
-                   valid ? src : q, valid);
+        const int t = tk[r / G];
+        const bool valid = t >= 0;
+        const __nv_bfloat16* src = qbase + ((int64_t)(valid ? t : 0) * g.hq + r % G) * kD + c * 8;
+        cp_async16(qb + (c >> 3) * kTileBytes + r * 128 + (((c & 7) ^ (r & 7)) << 4), src, valid);
       }
       cp_async_wait_all();
       fence_proxy_async_smem();
@@ -276,22 +290,24 @@ attn_tiles_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
     const int r = tid;                                   // TMEM lane = tile row
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
     const int tok = r / G, h = r % G;
+    int4 tl_next = my_tiles > 0 ? tiles[tile_lo] : make_int4(0, 0, 0, 0);
+    int e_next = (my_tiles > 0 && tok < tl_next.z) ? entries[tl_next.y + tok] : -1;
     for (int n = 0; n < my_tiles; ++n) {
-      if (*abort_flag) break;
-      const int4 tl = tiles[tile_lo + n];
+      if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+      const int4 tl = tl_next;
+      const int ent = e_next;
+      if (n + 1 < my_tiles) {               // prefetch the next tile's row metadata
+        tl_next = tiles[tile_lo + n + 1];
+        e_next = tok < tl_next.z ? entries[tl_next.y + tok] : -1;
+      }
       const int64_t seg = tl.x;
       const int sub = (int)(seg % g.nsub);
       const int64_t j = (seg / g.nsub) % g.nb;
       const int64_t gg = (seg / ((int64_t)g.nsub * g.nb)) % g.hkv;
       const int64_t b = seg / ((int64_t)g.nsub * g.nb * g.hkv);
-      const bool valid = tok < tl.z;
-      int64_t t = 0;
-      int pslot = 0;
-      if (valid) {
-        const int e = entries[tl.y + tok];
-        t = e >> 6;
-        pslot = e & 63;
-      }
+      const bool valid = ent >= 0;
+      const int64_t t = valid ? (ent >> 6) : 0;
+      const int pslot = valid ? (ent & 63) : 0;
       const int64_t own = t / g.block;
       const int64_t kbase = j * g.block + (int64_t)sub * kSegKeys;
       int64_t khi = (j == own) ? t + 1 : j * g.block + g.block;
@@ -302,46 +318,71 @@ attn_tiles_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
       for (int c = 0; c < g.nch; ++c) {
         const int64_t rem = khi - (kbase + (int64_t)c * kChunkKeys);
         const int lim = valid ? (int)max((int64_t)0, min((int64_t)kChunkKeys, rem)) : 0;
-        if (!mbar_wait(&bars->s_full[c], n & 1)) { ok = false; break; }
+        if (!mbar_wait_warp(&bars->s_full[c], n & 1)) { ok = false; break; }
         tc_fence_after();
         uint32_t sv[4][32];
 #pragma unroll
         for (int qd = 0; qd < 4; ++qd) tmem_ld32(lane_base + c * kChunkKeys + qd * 32, sv[qd]);
         tmem_ld_wait();
+        // row max of the raw scores (scale > 0 commutes with max), then
+        // p = 2^(s * scale*log2e - max * scale*log2e) with one FFMA + ex2 per score
+        const bool full = __all_sync(0xffffffffu, lim == kChunkKeys);
         float mx = -CUDART_INF_F;
+        if (full) {
 #pragma unroll
-        for (int qd = 0; qd < 4; ++qd)
+          for (int qd = 0; qd < 4; ++qd)
 #pragma unroll
-          for (int k = 0; k < 32; ++k)
-            if (qd * 32 + k < lim) mx = fmaxf(mx, __uint_as_float(sv[qd][k]) * g.scale_log2);
+            for (int k = 0; k < 32; ++k) mx = fmaxf(mx, __uint_as_float(sv[qd][k]));
+        } else {
+#pragma unroll
+          for (int qd = 0; qd < 4; ++qd)
+#pragma unroll
+            for (int k = 0; k < 32; ++k)
+              if (qd * 32 + k < lim) mx = fmaxf(mx, __uint_as_float(sv[qd][k]));
+        }
+        const float c2 = g.scale_log2;
+        const float mb = lim > 0 ? mx * c2 : 0.f;
         // P packed two bf16 per 32-bit column, written in place over the consumed scores:
         // chunk quarter qd lands in sv[qd / 2][(qd % 2) * 16 ...], already read.
         float sum = 0.f;
+        if (full) {
 #pragma unroll
-        for (int qd = 0; qd < 4; ++qd)
+          for (int qd = 0; qd < 4; ++qd)
 #pragma unroll
-          for (int k = 0; k < 32; k += 2) {
-            const int kk = qd * 32 + k;
-            const float p0 = kk < lim ? exp2f(__uint_as_float(sv[qd][k]) * g.scale_log2 - mx) : 0.f;
-            const float p1 =
-                kk + 1 < lim ? exp2f(__uint_as_float(sv[qd][k + 1]) * g.scale_log2 - mx) : 0.f;
-            sum += p0 + p1;
-            sv[qd >> 1][(qd & 1) * 16 + k / 2] = pack_bf16x2(p0, p1);
-          }
+            for (int k = 0; k < 32; k += 2) {
+              const float p0 = fast_exp2(fmaf(__uint_as_float(sv[qd][k]), c2, -mb));
+              const float p1 = fast_exp2(fmaf(__uint_as_float(sv[qd][k + 1]), c2, -mb));
+              sum += p0 + p1;
+              sv[qd >> 1][(qd & 1) * 16 + k / 2] = pack_bf16x2(p0, p1);
+            }
+        } else {
+#pragma unroll
+          for (int qd = 0; qd < 4; ++qd)
+#pragma unroll
+            for (int k = 0; k < 32; k += 2) {
+              const int kk = qd * 32 + k;
+              const float p0 =
+                  kk < lim ? fast_exp2(fmaf(__uint_as_float(sv[qd][k]), c2, -mb)) : 0.f;
+              const float p1 =
+                  kk + 1 < lim ? fast_exp2(fmaf(__uint_as_float(sv[qd][k + 1]), c2, -mb)) : 0.f;
+              sum += p0 + p1;
+              sv[qd >> 1][(qd & 1) * 16 + k / 2] = pack_bf16x2(p0, p1);
+            }
+        }
         tmem_st32(lane_base + c * kChunkKeys, sv[0]);
         tmem_st32(lane_base + c * kChunkKeys + 32, sv[1]);
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&bars->p_full[c]);
-        m_c[c] = mx;
+        m_c[c] = lim > 0 ? mb : -CUDART_INF_F;
         l_c[c] = sum;
       }
-      if (!ok || !mbar_wait(&bars->o_full, n & 1)) { fail(); break; }
+      if (!ok || !mbar_wait_warp(&bars->o_full, n & 1)) { fail(); break; }
       tc_fence_after();
       const float M = fmaxf(m_c[0], m_c[1]);
       float w[2];
 #pragma unroll
-      for (int c = 0; c < 2; ++c) w[c] = (c < g.nch && m_c[c] > -CUDART_INF_F) ? exp2f(m_c[c] - M) : 0.f;
+      for (int c = 0; c < 2; ++c) w[c] = (c < g.nch && m_c[c] > -CUDART_INF_F) ? fast_exp2(m_c[c] - M) : 0.f;
       const float L = w[0] * l_c[0] + w[1] * l_c[1];
       const float inv = L > 0.f ? 1.f / L : 0.f;
       __nv_bfloat16* dst = po + ((((b * g.hkv + gg) * g.S + t) * g.kslots + pslot) * G + h) * kD;
@@ -403,33 +444,44 @@ __global__ void merge_partials_kernel(const int32_t* __restrict__ idx,
   const int32_t* irow = idx + row * g.topk;
   const float* lrow = plse + row * g.kslots * G;
   const __nv_bfloat16* prow = po + row * g.kslots * G * kD;
-  float mx = -CUDART_INF_F;
+  float mx = -CUDART_INF_F, den = 0.f;
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  int ps_list[4];
+  int np = 0;
+  auto flush = [&]() {
+    float lv[4];
+    uint4 raw[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (u < np) {
+        lv[u] = lrow[ps_list[u] * G + h];
+        raw[u] = ldg16(prow + (int64_t)ps_list[u] * G * kD + lt * 8);
+      }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (u >= np || !(lv[u] > -CUDART_INF_F)) continue;
+      const float mn = fmaxf(mx, lv[u]);
+      const float sc = exp2f((mx - mn) * kLog2e);
+      const float wgt = exp2f((lv[u] - mn) * kLog2e);
+      float f[8];
+      Vec16<__nv_bfloat16>::unpack(raw[u], f);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] = fmaf(wgt, f[e], acc[e] * sc);
+      den = den * sc + wgt;
+      mx = mn;
+    }
+    np = 0;
+  };
   for (int s = 0; s < g.topk; ++s) {
     const int64_t j = irow[s];
     if (j < 0 || j >= g.nb || j > own) continue;
-    for (int sub = 0; sub < g.nsub; ++sub)
-      if (sub_has_keys(j, own, t, sub, g)) mx = fmaxf(mx, lrow[(s * g.nsub + sub) * G + h]);
-  }
-  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  float den = 0.f;
-  if (mx > -CUDART_INF_F) {
-    for (int s = 0; s < g.topk; ++s) {
-      const int64_t j = irow[s];
-      if (j < 0 || j >= g.nb || j > own) continue;
-      for (int sub = 0; sub < g.nsub; ++sub) {
-        if (!sub_has_keys(j, own, t, sub, g)) continue;
-        const int ps = s * g.nsub + sub;
-        const float lv = lrow[ps * G + h];
-        if (!(lv > -CUDART_INF_F)) continue;
-        const float wgt = exp2f((lv - mx) * kLog2e);
-        den += wgt;
-        float f[8];
-        Vec16<__nv_bfloat16>::unpack(ldg16(prow + (int64_t)ps * G * kD + lt * 8), f);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] = fmaf(wgt, f[e], acc[e]);
-      }
+    for (int sub = 0; sub < g.nsub; ++sub) {
+      if (!sub_has_keys(j, own, t, sub, g)) continue;
+      ps_list[np++] = s * g.nsub + sub;
+      if (np == 4) flush();
     }
   }
+  if (np > 0) flush();
   const float inv = den > 0.f ? 1.f / den : 0.f;
   uint4 out;
   out.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);

@@ -57,6 +57,27 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
   return true;
 }
 
+// The same wait, with one outcome for the whole warp (required before warp-collective
+// tcgen05 loads/stores: all 32 lanes must take the same path).
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity) {
+  const bool ok = mbar_wait(bar, parity);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// Named barrier `id` over `n` threads that also ORs a predicate across them, so every
+// participant leaves with the same decision.
+template <int ID, int N>
+__device__ __forceinline__ bool bar_sync_or(bool x) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.or.pred p, %2, %3, q;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)x), "n"(ID), "n"(N)
+      : "memory");
+  return r != 0;
+}
+
 // ------------------------------------------------------------------ TMA and cp.async
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,
                                             int x, int y) {

@@ -3,13 +3,16 @@
 // One CTA = 128 consecutive tokens of one (sequence, group).  The group-summed queries
 // (fp32 sum of the group's heads) are split into bf16 hi + lo planes (x ~ hi + lo to
 // ~2^-17 relative) and kept in shared memory; the pooled keys' hi/lo planes stream in
-// 128-block chunks through a 2-stage TMA ring.  Each chunk's scores
-//     S = Qhi Khi^T + Qhi Klo^T + Qlo Khi^T      (24 tcgen05.mma, M=128 N=128 K=16)
+// 64-block chunks through a 2-stage TMA ring.  Each chunk's scores
+//     S = Qhi Khi^T + Qhi Klo^T + Qlo Khi^T      (24 tcgen05.mma, M=128 N=64 K=16)
 // accumulate in fp32 in one of two TMEM buffers, so the MMAs of chunk c+1 run while the
-// four epilogue warps fold chunk c into per-row top lists held in registers.  The list
-// is kept sorted (score descending, earlier = lower block index first on ties) with a
-// branch-free insertion network; candidates at or below the current last entry are
-// rejected with one compare.  The score matrix never leaves the SM.
+// four epilogue warps fold chunk c into the rows' top lists.  Each warp owns 32 token
+// rows (its TMEM lanes); it copies their scores to shared memory and then walks them
+// row by row with the whole warp: lane l holds entry l of every row's list, sorted by
+// (score desc, block index asc), so a candidate is one ballot against the row's
+// threshold (entry k-1) and an insertion is a ballot, a popcount and two shuffles.
+// Candidates are inserted in ascending block order, which keeps ties on the lower
+// index.  The score matrix never leaves the SM.
 #include <cudaTypedefs.h>
 #include <math_constants.h>
 
@@ -23,9 +26,11 @@ using namespace sm100;
 
 constexpr int kD = 128;
 constexpr int kRows = 128;
-constexpr int kChunk = 128;                  // pooled keys per MMA chunk (N)
+constexpr int kChunk = 64;                   // pooled keys per MMA chunk (N)
+constexpr int kSPad = kChunk + 1;            // row stride of the score copy (no conflicts)
 constexpr int kThreads = 192;                // warps 0-3 epilogue, 4 issuer, 5 idle
-constexpr uint32_t kHalf = 16384;            // 128 rows x 128 B
+constexpr uint32_t kHalf = 16384;            // 128 rows x 128 B (query planes)
+constexpr uint32_t kKHalf = 8192;            // 64 rows x 128 B (pooled-key planes)
 
 struct __align__(8) TBars {
   uint64_t kb_full[2], kb_empty[2], acc_full[2], acc_empty[2], q_full;
@@ -38,22 +43,7 @@ struct TopkGeom {
   int hq, hkv, G, topk;
 };
 
-template <int KP>
-__device__ __forceinline__ void list_insert(float (&ls)[KP], int (&lj)[KP], float s, int j) {
-  // ls descending; strict compares keep the earlier (lower index) entry first on ties.
-#pragma unroll
-  for (int e = KP - 1; e > 0; --e) {
-    const bool up = s > ls[e - 1];
-    const bool here = s > ls[e];
-    const float ns = up ? ls[e - 1] : (here ? s : ls[e]);
-    const int nj = up ? lj[e - 1] : (here ? j : lj[e]);
-    ls[e] = ns;
-    lj[e] = nj;
-  }
-  if (s > ls[0]) { ls[0] = s; lj[0] = j; }
-}
-
-template <int KP>
+template <int G>
 __global__ void __launch_bounds__(kThreads, 1)
 topk_tc_kernel(const __grid_constant__ CUtensorMap tmHi, const __grid_constant__ CUtensorMap tmLo,
                const __nv_bfloat16* __restrict__ q, int32_t* __restrict__ idx, int* err,
@@ -63,8 +53,9 @@ topk_tc_kernel(const __grid_constant__ CUtensorMap tmHi, const __grid_constant__
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* Qhi = base;                     // 2 halves
   unsigned char* Qlo = base + 2 * kHalf;
-  unsigned char* KB = base + 4 * kHalf;          // stage s: hi halves, lo halves (64 KB)
-  TBars* bars = reinterpret_cast<TBars*>(KB + 2 * 4 * kHalf);
+  unsigned char* KB = base + 4 * kHalf;          // stage s: hi halves, lo halves (32 KB)
+  float* sbuf = reinterpret_cast<float*>(KB + 2 * 4 * kKHalf);     // [kRows][kSPad]
+  TBars* bars = reinterpret_cast<TBars*>(sbuf + kRows * kSPad);
 
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   const int64_t n_tiles_t = (g.S + kRows - 1) / kRows;
@@ -87,7 +78,7 @@ topk_tc_kernel(const __grid_constant__ CUtensorMap tmHi, const __grid_constant__
     bars->abort = 0;
     fence_mbar_init();
   }
-  if (warp == 0) { tmem_alloc(&bars->tmem_base, 256); tmem_relinquish(); }
+  if (warp == 0) { tmem_alloc(&bars->tmem_base, 128); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -103,12 +94,12 @@ topk_tc_kernel(const __grid_constant__ CUtensorMap tmHi, const __grid_constant__
       const int y_base = (int)(b * g.nb);
       auto load = [&](int c) {
         const int st = c & 1;
-        unsigned char* dst = KB + st * 4 * kHalf;
-        mbar_arrive_expect_tx(&bars->kb_full[st], 4 * kHalf);
+        unsigned char* dst = KB + st * 4 * kKHalf;
+        mbar_arrive_expect_tx(&bars->kb_full[st], 4 * kKHalf);
         for (int hf = 0; hf < 2; ++hf) {
           const int x = gg * kD + hf * 64;
-          tma_load_2d(dst + hf * kHalf, &tmHi, &bars->kb_full[st], x, y_base + c * kChunk);
-          tma_load_2d(dst + (2 + hf) * kHalf, &tmLo, &bars->kb_full[st], x, y_base + c * kChunk);
+          tma_load_2d(dst + hf * kKHalf, &tmHi, &bars->kb_full[st], x, y_base + c * kChunk);
+          tma_load_2d(dst + (2 + hf) * kKHalf, &tmLo, &bars->kb_full[st], x, y_base + c * kChunk);
         }
       };
       load(0);
@@ -123,15 +114,16 @@ topk_tc_kernel(const __grid_constant__ CUtensorMap tmHi, const __grid_constant__
         if (c >= 2 && !mbar_wait(&bars->acc_empty[st], ((c >> 1) - 1) & 1)) { fail(); break; }
         tc_fence_after();
         const uint32_t qh = smem_u32(Qhi), ql = smem_u32(Qlo);
-        const uint32_t kh = smem_u32(KB + st * 4 * kHalf), kl = kh + 2 * kHalf;
+        const uint32_t kh = smem_u32(KB + st * 4 * kKHalf), kl = kh + 2 * kKHalf;
         const uint32_t acc = tmem + st * kChunk;
         int n_mma = 0;
         for (int pass = 0; pass < 3; ++pass) {
           const uint32_t a = pass == 2 ? ql : qh;
           const uint32_t bb = pass == 1 ? kl : kh;
           for (int s = 0; s < kD / 16; ++s) {
-            const uint32_t off = (uint32_t)(s >> 2) * kHalf + (uint32_t)(s & 3) * 32;
-            umma_ss(acc, sdesc_sw128(a + off, 16, 1024), sdesc_sw128(bb + off, 16, 1024), idS,
+            const uint32_t ko = (uint32_t)(s & 3) * 32;
+            umma_ss(acc, sdesc_sw128(a + (uint32_t)(s >> 2) * kHalf + ko, 16, 1024),
+                    sdesc_sw128(bb + (uint32_t)(s >> 2) * kKHalf + ko, 16, 1024), idS,
                     n_mma++ > 0);
           }
         }
@@ -146,98 +138,143 @@ topk_tc_kernel(const __grid_constant__ CUtensorMap tmHi, const __grid_constant__
     const bool valid = t < g.S;
     // group-summed query row -> bf16 hi/lo planes in the K-major swizzled layout
     {
-      const __nv_bfloat16* qr = q + ((b * g.S + (valid ? t : 0)) * g.hq + (int64_t)gg * g.G) * kD;
+      const __nv_bfloat16* qr = q + ((b * g.S + (valid ? t : 0)) * g.hq + (int64_t)gg * G) * kD;
 #pragma unroll 1
-      for (int c = 0; c < 16; ++c) {                 // 16 chunks of 8 dims
-        float acc8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        if (valid) {
-          for (int h = 0; h < g.G; ++h) {
+      for (int c0 = 0; c0 < 16; c0 += 4) {         // 4 chunks of 8 dims, loads in flight
+        uint4 raw[4][G];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+          for (int h = 0; h < G; ++h)
+            raw[u][h] = valid ? ldg16(qr + (int64_t)h * kD + (c0 + u) * 8) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int c = c0 + u;
+          float acc8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
             float f[8];
-            Vec16<__nv_bfloat16>::unpack(ldg16(qr + (int64_t)h * kD + c * 8), f);
+            Vec16<__nv_bfloat16>::unpack(raw[u][h], f);
 #pragma unroll
             for (int e = 0; e < 8; ++e) acc8[e] += f[e];
           }
-        }
-        uint32_t hw[4], lw[4];
+          uint32_t hw[4], lw[4];
 #pragma unroll
-        for (int e = 0; e < 8; e += 2) {
-          const uint32_t hp = pack_bf16x2(acc8[e], acc8[e + 1]);
-          const float h0 = bf16lo_to_f32(hp), h1 = bf16hi_to_f32(hp);
-          hw[e / 2] = hp;
-          lw[e / 2] = pack_bf16x2(acc8[e] - h0, acc8[e + 1] - h1);
+          for (int e = 0; e < 8; e += 2) {
+            const uint32_t hp = pack_bf16x2(acc8[e], acc8[e + 1]);
+            hw[e / 2] = hp;
+            lw[e / 2] = pack_bf16x2(acc8[e] - bf16lo_to_f32(hp), acc8[e + 1] - bf16hi_to_f32(hp));
+          }
+          const uint32_t off = (c >> 3) * kHalf + r * 128 + (((c & 7) ^ (r & 7)) << 4);
+          *reinterpret_cast<uint4*>(Qhi + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+          *reinterpret_cast<uint4*>(Qlo + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
         }
-        const uint32_t off = (c >> 3) * kHalf + r * 128 + (((c & 7) ^ (r & 7)) << 4);
-        *reinterpret_cast<uint4*>(Qhi + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-        *reinterpret_cast<uint4*>(Qlo + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
       }
       fence_proxy_async_smem();
       mbar_arrive(&bars->q_full);
     }
-    const int64_t own = valid ? t / g.block : 0;
-    const int n_take = (int)(own < (int64_t)g.topk - 1 ? own : (int64_t)g.topk - 1);
-    float ls[KP];
-    int lj[KP];
+    // Lane l keeps entry l of the sorted lists of the warp's 32 rows; K = topk - 1 <= 31
+    // entries are kept (lanes >= K hold the next-best values, also sorted).
+    const int K = g.topk - 1;
+    float ls[32];
+    int lj[32];
 #pragma unroll
-    for (int e = 0; e < KP; ++e) { ls[e] = -CUDART_INF_F; lj[e] = -1; }
+    for (int rr = 0; rr < 32; ++rr) { ls[rr] = -CUDART_INF_F; lj[rr] = -1; }
+    const int64_t row0 = t0 + warp * 32;          // first token of this warp's rows
+    float* wbuf = sbuf + warp * 32 * kSPad;
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
     for (int c = 0; c < nch; ++c) {
       const int st = c & 1;
-      if (!mbar_wait(&bars->acc_full[st], (c >> 1) & 1)) { fail(); break; }
+      if (!mbar_wait_warp(&bars->acc_full[st], (c >> 1) & 1)) { fail(); break; }
       tc_fence_after();
-      uint32_t sv[4][32];
-#pragma unroll
-      for (int qd = 0; qd < 4; ++qd) tmem_ld32(lane_base + st * kChunk + qd * 32, sv[qd]);
+      uint32_t sv[2][32];
+      tmem_ld32(lane_base + st * kChunk, sv[0]);
+      tmem_ld32(lane_base + st * kChunk + 32, sv[1]);
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(&bars->acc_empty[st]);
-      const int64_t j0 = (int64_t)c * kChunk;
-      const int64_t rem = own - j0;
-      const int lim = rem <= 0 ? 0 : (rem >= kChunk ? kChunk : (int)rem);
 #pragma unroll
-      for (int qd = 0; qd < 4; ++qd)
-#pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          const float s = __uint_as_float(sv[qd][k]);
-          if (qd * 32 + k < lim && s > ls[KP - 1]) list_insert<KP>(ls, lj, s, (int)(j0 + qd * 32 + k));
-        }
-    }
-    if (valid) {
-      // the n_take best past blocks plus the own block, ascending, -1 padded
-      int sel[KP + 1];
-      int n = 0;
-#pragma unroll
-      for (int e = 0; e < KP; ++e)
-        if (e < n_take) sel[n++] = lj[e];
-      sel[n++] = (int)own;
-      for (int a = 1; a < n; ++a) {
-        const int x = sel[a];
-        int c = a - 1;
-        while (c >= 0 && sel[c] > x) { sel[c + 1] = sel[c]; --c; }
-        sel[c + 1] = x;
+      for (int k = 0; k < 32; ++k) {
+        wbuf[lane * kSPad + k] = __uint_as_float(sv[0][k]);
+        wbuf[lane * kSPad + 32 + k] = __uint_as_float(sv[1][k]);
       }
-      int32_t* out = idx + ((b * g.hkv + gg) * g.S + t) * (int64_t)g.topk;
-      for (int e = 0; e < g.topk; ++e) out[e] = e < n ? sel[e] : -1;
+      __syncwarp();
+      const int64_t j0 = (int64_t)c * kChunk;
+#pragma unroll
+      for (int rr = 0; rr < 32; ++rr) {
+        const int64_t tr = row0 + rr;
+        const int64_t own_r = tr < g.S ? tr / g.block : 0;
+        const int64_t rem = own_r - j0;
+        const int lim = K <= 0 ? 0 : (rem <= 0 ? 0 : (rem >= kChunk ? kChunk : (int)rem));
+        if (lim == 0) continue;                          // warp-uniform
+        const float s0 = wbuf[rr * kSPad + lane];
+        const float s1 = wbuf[rr * kSPad + 32 + lane];
+        float thr = __shfl_sync(0xffffffffu, ls[rr], K - 1);
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const float sh = half ? s1 : s0;
+          unsigned m = __ballot_sync(0xffffffffu, sh > thr && half * 32 + lane < lim);
+          while (m) {                                    // ascending block index
+            const int src = __ffs(m) - 1;
+            m &= m - 1;
+            const float cs = __shfl_sync(0xffffffffu, sh, src);
+            if (!(cs > thr)) continue;                   // threshold rose meanwhile
+            const int cj = (int)(j0 + half * 32 + src);
+            const int p = __popc(__ballot_sync(0xffffffffu, ls[rr] >= cs));
+            const float us = __shfl_up_sync(0xffffffffu, ls[rr], 1);
+            const int uj = __shfl_up_sync(0xffffffffu, lj[rr], 1);
+            if (lane > p) { ls[rr] = us; lj[rr] = uj; }
+            else if (lane == p) { ls[rr] = cs; lj[rr] = cj; }
+            thr = __shfl_sync(0xffffffffu, ls[rr], K - 1);
+          }
+        }
+      }
+      __syncwarp();
+    }
+    // Output: the kept past blocks ascending, then the own block, -1 padded.
+#pragma unroll 1
+    for (int rr = 0; rr < 32; ++rr) {
+      const int64_t tr = row0 + rr;
+      if (tr >= g.S) break;                              // warp-uniform
+      const int64_t own_r = tr / g.block;
+      const int n_take = (int)(own_r < K ? own_r : K);
+      int key = (lane < n_take) ? lj[rr] : 0x7fffffff;   // bitonic sort, ascending
+#pragma unroll
+      for (int size = 2; size <= 32; size <<= 1)
+#pragma unroll
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+          const int other = __shfl_xor_sync(0xffffffffu, key, stride);
+          const bool up = ((lane & size) == 0);
+          const bool lower = (lane & stride) == 0;
+          key = (lower == up) ? min(key, other) : max(key, other);
+        }
+      int val = key;
+      if (lane == n_take) val = (int)own_r;
+      else if (lane > n_take) val = -1;
+      if (lane < g.topk)
+        idx[((b * g.hkv + gg) * g.S + tr) * (int64_t)g.topk + lane] = val;
     }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, 128);
   }
 }
 
 
-template <int KP>
+template <int G>
 cudaError_t run_topk_tc(const Shape& s, const CUtensorMap& mh, const CUtensorMap& ml,
                         const void* q, int32_t* idx, int* err, cudaStream_t st) {
-  const size_t smem = 1024 + 12 * (size_t)kHalf + sizeof(TBars);
-  cudaError_t e = cudaFuncSetAttribute(topk_tc_kernel<KP>,
+  const size_t smem = 1024 + 4 * (size_t)kHalf + 8 * (size_t)kKHalf +
+                      (size_t)kRows * kSPad * 4 + sizeof(TBars);
+  cudaError_t e = cudaFuncSetAttribute(topk_tc_kernel<G>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   TopkGeom g{s.seq, s.nb, s.block, (int)s.hq, (int)s.hkv, (int)(s.hq / s.hkv), (int)s.topk};
   dim3 grid((unsigned)((s.seq + kRows - 1) / kRows), (unsigned)s.hkv, (unsigned)s.batch);
-  topk_tc_kernel<KP><<<grid, kThreads, smem, st>>>(mh, ml, (const __nv_bfloat16*)q, idx, err, g);
+  topk_tc_kernel<G><<<grid, kThreads, smem, st>>>(mh, ml, (const __nv_bfloat16*)q, idx, err, g);
   return cudaGetLastError();
 }
 
@@ -247,7 +284,7 @@ bool tc_topk_supported(const Shape& s) {
   if (s.dtype != MSA_BF16 || s.d != kD) return false;
   const int64_t G = s.hq / s.hkv;
   if (G != 1 && G != 2 && G != 4 && G != 8) return false;
-  if (s.topk - 1 > 32) return false;
+  if (s.topk > 32) return false;                  // topk - 1 <= 31 list lanes
   if (s.batch * s.nb >= ((int64_t)1 << 31) - kChunk) return false;
   return true;
 }
@@ -258,8 +295,12 @@ cudaError_t launch_topk_prefill_tc(const Shape& s, const void* q, const void* kb
   if (!make_bf16_2d_map(&mh, kbar_hi, s.batch * s.nb, s.hkv * kD, kChunk) ||
       !make_bf16_2d_map(&ml, kbar_lo, s.batch * s.nb, s.hkv * kD, kChunk))
     return cudaErrorInvalidValue;
-  if (s.topk - 1 <= 16) return run_topk_tc<16>(s, mh, ml, q, idx, err, st);
-  return run_topk_tc<32>(s, mh, ml, q, idx, err, st);
+  switch (s.hq / s.hkv) {
+    case 1: return run_topk_tc<1>(s, mh, ml, q, idx, err, st);
+    case 2: return run_topk_tc<2>(s, mh, ml, q, idx, err, st);
+    case 4: return run_topk_tc<4>(s, mh, ml, q, idx, err, st);
+    default: return run_topk_tc<8>(s, mh, ml, q, idx, err, st);
+  }
 }
 
 }  // namespace msa
