@@ -20,7 +20,8 @@ from ._lib import (  # noqa: F401
 
 __all__ = [
     "params", "workspace", "pool_keys", "block_scores", "topk_select", "sparse_attn_fwd",
-    "prefill_fwd", "decode_fwd", "read_device_error", "clear_device_error", "version",
+    "prefill_fwd", "decode_fwd", "decode_fwd_static", "read_device_error",
+    "clear_device_error", "version",
     "MsaError", "MsaParams",
 ]
 
@@ -165,6 +166,26 @@ def decode_fwd(q, kbar, k_bank, v_bank, block: int, topk: int, scale=None, kbar_
     _lib.check("msa_decode_fwd", _lib.load().msa_decode_fwd(
         ctypes.byref(p), nq, _ptr(q), _ptr(kbar), _ptr(kbar_hi), _ptr(k_bank), _ptr(v_bank),
         _ptr(idx), _ptr(o), _ptr(lse), _ptr(ws), ws.numel(), _stream(q.device)))
+    return o, lse, idx
+
+
+def decode_fwd_static(q, kbar, k_bank, v_bank, block: int, topk: int, scale=None,
+                      kbar_hi=None, want_lse=True, out=None):
+    """decode_fwd without a workspace: the library's fixed device scratch is used (for
+    callers that cannot allocate device memory; see msa_decode_fwd_static in msa.h)."""
+    nq, hq, d = q.shape
+    S, hkv, _ = k_bank.shape
+    p = params(batch=1, seq=S, hq=hq, hkv=hkv, d=d, block=block, topk=topk,
+               scale=scale if scale is not None else d ** -0.5, dtype=q.dtype)
+    if out is not None:
+        o, lse, idx = out
+    else:
+        o = torch.empty_like(q)
+        lse = torch.empty(nq, hq, dtype=torch.float32, device=q.device) if want_lse else None
+        idx = torch.empty(nq, hkv, topk, dtype=torch.int32, device=q.device)
+    _lib.check("msa_decode_fwd_static", _lib.load().msa_decode_fwd_static(
+        ctypes.byref(p), nq, _ptr(q), _ptr(kbar), _ptr(kbar_hi), _ptr(k_bank), _ptr(v_bank),
+        _ptr(idx), _ptr(o), _ptr(lse), _stream(q.device)))
     return o, lse, idx
 
 

@@ -170,6 +170,32 @@ MSA_API msa_status msa_decode_fwd(const msa_params* p, int64_t n_query, const vo
                           int32_t* idx, void* o, float* lse, void* ws, size_t ws_bytes,
                           msa_stream_t stream);
 
+/* Bytes of the fixed device scratch used by msa_decode_fwd_static (32 MiB). */
+#define MSA_DECODE_STATIC_SCRATCH_BYTES ((size_t)32 << 20)
+
+/* Decode without a caller workspace, for callers that cannot allocate device memory
+ * where they run a decode step (for example a serving loop inside CUDA-graph capture,
+ * or a runtime that forbids device allocation on its hot path).  The pages have no
+ * counterpart: this is a deployment variant of msa_decode_fwd, with the same arguments
+ * minus the workspace, the same kernels and the same results.
+ *   - Scratch: a file-scope device array of MSA_DECODE_STATIC_SCRATCH_BYTES that every
+ *     GPU loading this library keeps until the process exits.  The call allocates
+ *     nothing (no cudaMalloc/cudaFree, no allocating library routine).
+ *   - Limit: returns MSA_ERR_WORKSPACE, launching nothing, when
+ *     msa_workspace_bytes(p, MSA_OP_DECODE, n_query) exceeds that size (64 queries x 32
+ *     heads against a 10M-token bank need about 14 MB).
+ *   - Set-up: the first call on a device looks up the array's device address with that
+ *     device current (cudaGetSymbolAddress) and caches it; make that first call before
+ *     any stream capture.
+ *   - Sharing: every call on a device uses the same array, which keeps the last call's
+ *     contents; the call clears what must start at zero.  Calls that overlap on the GPU
+ *     (concurrent streams, or several host threads) race on the array: serialise them.
+ *   - Device error bits are not reported to the caller (they live in the shared array). */
+MSA_API msa_status msa_decode_fwd_static(const msa_params* p, int64_t n_query, const void* q,
+                                         const float* kbar, const void* kbar_hi,
+                                         const void* k_bank, const void* v_bank, int32_t* idx,
+                                         void* o, float* lse, msa_stream_t stream);
+
 /* Copies the workspace's device error word to *bits after synchronising `stream`;
  * returns MSA_ERR_DEVICE when any bit is set, else MSA_OK. */
 MSA_API msa_status msa_read_device_error(const void* ws, int32_t* bits, msa_stream_t stream);

@@ -1,0 +1,60 @@
+"""The allocation-free decode entry point (msa_decode_fwd_static).
+
+Callers that cannot allocate device memory at decode time (graph-captured serving loops,
+runtimes that forbid device allocation on the hot path) use a fixed device scratch
+inside the library instead of a workspace.  This checks, through the C ABI, that two
+calls in a row give the same selection and outputs as msa_decode_fwd with a caller
+workspace.  It sits in its own file that pytest collects last, and it holds whether it
+runs alone in a fresh process or after the other tests.
+"""
+import ctypes
+
+import pytest
+import torch
+
+import msa_inputs as mi
+
+pytestmark = pytest.mark.gpu
+
+
+def test_static_scratch_decode_matches_workspace_decode():
+    import block_sparse_top_mean_b200 as msa
+    from block_sparse_top_mean_b200 import _lib, build
+    build.build()
+    lib = _lib.load()
+    w = mi.Workload("decode_static_check", "decode", 1, 60_000, 32, 8, 128, 64, 32, "bf16",
+                    n_query=16)
+    _, kb, vb = mi.decode_inputs(w, device="cuda")
+    kbar = msa.pool_keys(kb[None], w.block)[0]
+    p = msa.params(batch=1, seq=w.seq, hq=w.hq, hkv=w.hkv, d=w.d, block=w.block, topk=w.topk,
+                   scale=w.scale, dtype=torch.bfloat16)
+    assert lib.msa_workspace_bytes(ctypes.byref(p), _lib.OP_DECODE, w.n_query) <= 32 << 20
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    P = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
+    for call, seed in enumerate((11, 12)):          # two calls in a row, different queries
+        q = mi.normal((w.n_query, w.hq, w.d), seed, mi.STREAM_DECODE_Q, "cuda", torch.bfloat16)
+        o_ref, lse_ref, idx_ref = msa.decode_fwd(q, kbar, kb, vb, w.block, w.topk, w.scale)
+        o = torch.empty_like(q)
+        lse = torch.empty(w.n_query, w.hq, dtype=torch.float32, device="cuda")
+        idx = torch.empty(w.n_query, w.hkv, w.topk, dtype=torch.int32, device="cuda")
+        st = lib.msa_decode_fwd_static(ctypes.byref(p), w.n_query, P(q), P(kbar), None, P(kb),
+                                       P(vb), P(idx), P(o), P(lse), stream)
+        assert st == _lib.MSA_OK, (call, st)
+        torch.cuda.synchronize()
+        assert torch.equal(idx, idx_ref), call
+        assert (o.float() - o_ref.float()).abs().max().item() <= 2e-2, call
+        assert (lse - lse_ref).abs().max().item() <= 2e-3, call
+
+
+def test_static_scratch_rejects_sizes_beyond_the_limit():
+    from block_sparse_top_mean_b200 import _lib
+    import block_sparse_top_mean_b200 as msa
+    lib = _lib.load()
+    p = msa.params(batch=1, seq=10_000_000, hq=32, hkv=8, d=128, block=64, topk=32, scale=0.088,
+                   dtype=torch.bfloat16)
+    n_query = 4096                                   # needs far more than 32 MiB
+    assert lib.msa_workspace_bytes(ctypes.byref(p), _lib.OP_DECODE, n_query) > 32 << 20
+    fake = ctypes.c_void_p(4096)
+    st = lib.msa_decode_fwd_static(ctypes.byref(p), n_query, fake, fake, None, fake, fake, fake,
+                                   fake, None, None)
+    assert st == _lib.MSA_ERR_WORKSPACE
