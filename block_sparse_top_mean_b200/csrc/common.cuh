@@ -94,6 +94,10 @@ cudaError_t launch_block_scores(const Shape& s, const void* q, const float* kbar
 // Causal prefill selection (fused scoring + top-k); writes idx [b, hkv, S, topk].
 cudaError_t launch_topk_prefill(const Shape& s, const void* q, const float* kbar, int32_t* idx,
                                 cudaStream_t st);
+// The same selection restricted to the 64-token tiles whose flag byte is set.
+cudaError_t launch_topk_prefill_flagged(const Shape& s, const void* q, const float* kbar,
+                                        int32_t* idx, const uint8_t* flags, int flag_tile,
+                                        cudaStream_t st);
 
 // Decode selection: per-split candidate lists then a merge; writes idx [nq, hkv, topk].
 size_t decode_select_ws_bytes(const Shape& s, int64_t n_query);
@@ -116,9 +120,13 @@ int sm_count();
 
 // Tensor-core prefill selection (bf16, d = 128); see topk_tc.cu.  Needs the pooled keys'
 // bf16 hi/lo planes.
+// A flag byte per (sequence, group, 64-token tile) marks tiles whose selection must be
+// redone exactly by the SIMT kernel (launch_topk_prefill_flagged).
 bool tc_topk_supported(const Shape& s);
-cudaError_t launch_topk_prefill_tc(const Shape& s, const void* q, const void* kbar_hi,
-                                   const void* kbar_lo, int32_t* idx, int* err, cudaStream_t st);
+size_t topk_tc_flag_bytes(const Shape& s);
+cudaError_t launch_topk_prefill_tc(const Shape& s, const void* q, const float* kbar,
+                                   const void* kbar_hi, const void* kbar_lo, int32_t* idx,
+                                   uint8_t* flags, int* err, cudaStream_t st);
 
 // Key-centric tensor-core attention (bf16, d = 128); see attn_tc.cu.
 bool tc_attn_supported(const Shape& s);

@@ -46,6 +46,10 @@ msa_status check_params(const msa_params* p, bool bank, Shape* s) {
 bool empty_prefill(const Shape& s) { return s.batch == 0 || s.seq == 0; }
 
 size_t kbar_bytes(const Shape& s) { return (size_t)s.batch * s.nb * s.hkv * s.d * sizeof(float); }
+// Fallback flags of the tensor-core selection (one byte per 64-token tile).
+size_t topk_flag_ws(const Shape& s) {
+  return msa::tc_topk_supported(s) ? round256(msa::topk_tc_flag_bytes(s)) : 0;
+}
 // bf16 hi or lo plane of the pooled keys; only the tensor-core selection uses them.
 size_t kbar_split_bytes(const Shape& s) {
   return msa::tc_topk_supported(s) ? (size_t)s.batch * s.nb * s.hkv * s.d * 2 : 0;
@@ -54,11 +58,12 @@ size_t kbar_split_bytes(const Shape& s) {
 size_t ws_bytes_for(const Shape& s, int op, int64_t n_query) {
   switch (op) {
     case MSA_OP_TOPK_SELECT:
-      return msa::kWsHeader;
+      return msa::kWsHeader + topk_flag_ws(s);
     case MSA_OP_SPARSE_ATTN:
       return msa::kWsHeader + (msa::tc_attn_supported(s) ? round256(msa::tc_attn_ws_bytes(s)) : 0);
     case MSA_OP_PREFILL:
       return msa::kWsHeader + round256(kbar_bytes(s)) + 2 * round256(kbar_split_bytes(s)) +
+             topk_flag_ws(s) +
              (msa::tc_attn_supported(s) ? round256(msa::tc_attn_ws_bytes(s)) : 0);
     case MSA_OP_DECODE:
       return msa::kWsHeader + round256(msa::decode_select_ws_bytes(s, n_query)) +
@@ -79,10 +84,10 @@ msa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MSA_OK : MSA_E
 // bf16 with d = 128 and the split planes present runs the tensor-core selection;
 // otherwise the fp32 SIMT one.
 cudaError_t launch_selection(const Shape& s, const void* q, const float* kbar,
-                             const void* kbar_hi, const void* kbar_lo, int32_t* idx, int* err,
-                             cudaStream_t st) {
+                             const void* kbar_hi, const void* kbar_lo, int32_t* idx,
+                             uint8_t* flags, int* err, cudaStream_t st) {
   if (kbar_hi != nullptr && kbar_lo != nullptr && msa::tc_topk_supported(s))
-    return msa::launch_topk_prefill_tc(s, q, kbar_hi, kbar_lo, idx, err, st);
+    return msa::launch_topk_prefill_tc(s, q, kbar, kbar_hi, kbar_lo, idx, flags, err, st);
   return msa::launch_topk_prefill(s, q, kbar, idx, st);
 }
 
@@ -161,7 +166,8 @@ msa_status msa_topk_select(const msa_params* p, const void* q, const float* kbar
   if ((kbar_hi != nullptr && !aligned16(kbar_hi)) || (kbar_lo != nullptr && !aligned16(kbar_lo)))
     return MSA_ERR_INVALID_ARG;
   if ((st = check_ws(s, MSA_OP_TOPK_SELECT, 0, ws, ws_bytes)) != MSA_OK) return st;
-  return cuda_status(launch_selection(s, q, kbar, kbar_hi, kbar_lo, idx, err_word(ws),
+  return cuda_status(launch_selection(s, q, kbar, kbar_hi, kbar_lo, idx,
+                                      reinterpret_cast<uint8_t*>(ws_body(ws)), err_word(ws),
                                       (cudaStream_t)stream));
 }
 
@@ -202,8 +208,10 @@ msa_status msa_prefill_fwd(const msa_params* p, const void* q, const void* k, co
     lo = body + off + round256(kbar_split_bytes(s));
     off += 2 * round256(kbar_split_bytes(s));
   }
+  uint8_t* flags = reinterpret_cast<uint8_t*>(body + off);
+  off += topk_flag_ws(s);
   cudaError_t e = msa::launch_pool_keys(s, k, kbar, hi, lo, s.batch, cs);
-  if (e == cudaSuccess) e = launch_selection(s, q, kbar, hi, lo, idx, err_word(ws), cs);
+  if (e == cudaSuccess) e = launch_selection(s, q, kbar, hi, lo, idx, flags, err_word(ws), cs);
   if (e == cudaSuccess) e = launch_attention(s, q, k, v, idx, o, lse, body + off, err_word(ws), cs);
   return cuda_status(e);
 }

@@ -118,12 +118,14 @@ template <typename T, int D>
 __global__ void __launch_bounds__(kThreads)
 topk_prefill_kernel(const T* __restrict__ q, const float* __restrict__ kbar,
                     int32_t* __restrict__ idx, int64_t S, int64_t nb, int hq, int hkv,
-                    int64_t block, int topk) {
+                    int64_t block, int topk, const uint8_t* __restrict__ only) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   TopkSmem<D>& sm = *reinterpret_cast<TopkSmem<D>*>(smem_raw);
   const int64_t t0 = (int64_t)blockIdx.x * kRows;
   const int g = blockIdx.y;
   const int64_t b = blockIdx.z;
+  // restricted run: only the tiles flagged by the tensor-core selection
+  if (only != nullptr && only[((int64_t)b * hkv + g) * gridDim.x + blockIdx.x] == 0) return;
   const int G = hq / hkv;
   const int r = threadIdx.x;
   // rows of this tile: tokens t0 .. t0+kRows-1 of sequence b, group g
@@ -312,14 +314,14 @@ cudaError_t launch_block_scores(const Shape& s, const void* q, const float* kbar
 
 template <typename T, int D>
 static cudaError_t topk_prefill_t(const Shape& s, const void* q, const float* kbar, int32_t* idx,
-                                  cudaStream_t st) {
+                                  cudaStream_t st, const uint8_t* only = nullptr) {
   const size_t smem = sizeof(TopkSmem<D>);
   cudaError_t e = set_smem(topk_prefill_kernel<T, D>, smem);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)((s.seq + kRows - 1) / kRows), (unsigned)s.hkv, (unsigned)s.batch);
   topk_prefill_kernel<T, D><<<grid, kThreads, smem, st>>>((const T*)q, kbar, idx, s.seq, s.nb,
                                                           (int)s.hq, (int)s.hkv, s.block,
-                                                          (int)s.topk);
+                                                          (int)s.topk, only);
   return cudaGetLastError();
 }
 
@@ -330,6 +332,17 @@ cudaError_t launch_topk_prefill(const Shape& s, const void* q, const float* kbar
                       : topk_prefill_t<__nv_bfloat16, 64>(s, q, kbar, idx, st);
   return s.d == 128 ? topk_prefill_t<float, 128>(s, q, kbar, idx, st)
                     : topk_prefill_t<float, 64>(s, q, kbar, idx, st);
+}
+
+cudaError_t launch_topk_prefill_flagged(const Shape& s, const void* q, const float* kbar,
+                                        int32_t* idx, const uint8_t* flags, int flag_tile,
+                                        cudaStream_t st) {
+  if (flag_tile != kRows) return cudaErrorInvalidValue;   // one flag per SIMT tile
+  if (s.dtype == MSA_BF16)
+    return s.d == 128 ? topk_prefill_t<__nv_bfloat16, 128>(s, q, kbar, idx, st, flags)
+                      : topk_prefill_t<__nv_bfloat16, 64>(s, q, kbar, idx, st, flags);
+  return s.d == 128 ? topk_prefill_t<float, 128>(s, q, kbar, idx, st, flags)
+                    : topk_prefill_t<float, 64>(s, q, kbar, idx, st, flags);
 }
 
 size_t decode_select_ws_bytes(const Shape& s, int64_t n_query) {

@@ -6,13 +6,19 @@
 // 64-block chunks through a 2-stage TMA ring.  Each chunk's scores
 //     S = Qhi Khi^T + Qhi Klo^T + Qlo Khi^T      (24 tcgen05.mma, M=128 N=64 K=16)
 // accumulate in fp32 in one of two TMEM buffers, so the MMAs of chunk c+1 run while the
-// four epilogue warps fold chunk c into the rows' top lists.  Each warp owns 32 token
-// rows (its TMEM lanes); it copies their scores to shared memory and then walks them
-// row by row with the whole warp: lane l holds entry l of every row's list, sorted by
-// (score desc, block index asc), so a candidate is one ballot against the row's
-// threshold (entry k-1) and an insertion is a ballot, a popcount and two shuffles.
-// Candidates are inserted in ascending block order, which keeps ties on the lower
-// index.  The score matrix never leaves the SM.
+// four epilogue warps (one TMEM lane = one token row each) process chunk c.
+//
+// Selection is exact and takes two passes over the chunks (the MMAs are cheap):
+//   pass 1: each row keeps, in registers, the k-1 largest maxima of groups of 4
+//           consecutive scores (a branch-free min/max insertion, no divergence).  The
+//           (k-1)-th of them, T, is a lower bound of the row's (k-1)-th score: k-1
+//           different groups each hold a score >= T.
+//   pass 2: the scores are recomputed and every eligible score >= T is appended to the
+//           row's buffer in shared memory (about k entries for long rows).
+// The row's k-1 best buffered blocks by (score desc, block index asc) are then picked
+// exactly.  A row whose buffer would overflow (only degenerate inputs, e.g. exact ties)
+// flags its 64-token tile, which the fp32 SIMT selection then recomputes.
+// The score matrix never leaves the SM.
 #include <cudaTypedefs.h>
 #include <math_constants.h>
 
@@ -27,7 +33,9 @@ using namespace sm100;
 constexpr int kD = 128;
 constexpr int kRows = 128;
 constexpr int kChunk = 64;                   // pooled keys per MMA chunk (N)
-constexpr int kSPad = kChunk + 1;            // row stride of the score copy (no conflicts)
+constexpr int kGroup = 4;                    // scores per group maximum in pass 1
+constexpr int kCap = 64;                     // candidate buffer per row
+constexpr int kFlagTile = 64;                // tokens per fallback flag
 constexpr int kThreads = 192;                // warps 0-3 epilogue, 4 issuer, 5 idle
 constexpr uint32_t kHalf = 16384;            // 128 rows x 128 B (query planes)
 constexpr uint32_t kKHalf = 8192;            // 64 rows x 128 B (pooled-key planes)
@@ -43,19 +51,20 @@ struct TopkGeom {
   int hq, hkv, G, topk;
 };
 
-template <int G>
+template <int G, int KM>
 __global__ void __launch_bounds__(kThreads, 1)
 topk_tc_kernel(const __grid_constant__ CUtensorMap tmHi, const __grid_constant__ CUtensorMap tmLo,
-               const __nv_bfloat16* __restrict__ q, int32_t* __restrict__ idx, int* err,
-               TopkGeom g) {
+               const __nv_bfloat16* __restrict__ q, int32_t* __restrict__ idx,
+               uint8_t* __restrict__ flags, int* err, TopkGeom g) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* base = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* Qhi = base;                     // 2 halves
   unsigned char* Qlo = base + 2 * kHalf;
   unsigned char* KB = base + 4 * kHalf;          // stage s: hi halves, lo halves (32 KB)
-  float* sbuf = reinterpret_cast<float*>(KB + 2 * 4 * kKHalf);     // [kRows][kSPad]
-  TBars* bars = reinterpret_cast<TBars*>(sbuf + kRows * kSPad);
+  float* cand_s = reinterpret_cast<float*>(KB + 2 * 4 * kKHalf);   // [kCap][kRows]
+  int* cand_j = reinterpret_cast<int*>(cand_s + kCap * kRows);     // [kCap][kRows]
+  TBars* bars = reinterpret_cast<TBars*>(cand_j + kCap * kRows);
 
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   const int64_t n_tiles_t = (g.S + kRows - 1) / kRows;
@@ -65,7 +74,8 @@ topk_tc_kernel(const __grid_constant__ CUtensorMap tmHi, const __grid_constant__
   const int64_t t0 = tile * kRows;
   const int64_t t_last = min(t0 + kRows, g.S) - 1;
   const int64_t jmax = t_last / g.block;                    // eligible blocks: j < jmax
-  const int nch = (int)((jmax + kChunk - 1) / kChunk);
+  const int nch = g.topk > 1 ? (int)((jmax + kChunk - 1) / kChunk) : 0;
+  const int nsteps = 2 * nch;                               // pass 1 then pass 2
 
   if (tid == 0) {
     for (int s = 0; s < 2; ++s) {
@@ -95,18 +105,19 @@ topk_tc_kernel(const __grid_constant__ CUtensorMap tmHi, const __grid_constant__
       auto load = [&](int c) {
         const int st = c & 1;
         unsigned char* dst = KB + st * 4 * kKHalf;
+        const int y = y_base + (c % nch) * kChunk;          // step c streams chunk c mod nch
         mbar_arrive_expect_tx(&bars->kb_full[st], 4 * kKHalf);
         for (int hf = 0; hf < 2; ++hf) {
           const int x = gg * kD + hf * 64;
-          tma_load_2d(dst + hf * kKHalf, &tmHi, &bars->kb_full[st], x, y_base + c * kChunk);
-          tma_load_2d(dst + (2 + hf) * kKHalf, &tmLo, &bars->kb_full[st], x, y_base + c * kChunk);
+          tma_load_2d(dst + hf * kKHalf, &tmHi, &bars->kb_full[st], x, y);
+          tma_load_2d(dst + (2 + hf) * kKHalf, &tmLo, &bars->kb_full[st], x, y);
         }
       };
       load(0);
       if (!mbar_wait(&bars->q_full, 0)) fail();
-      for (int c = 0; c < nch && !*abort_flag; ++c) {
+      for (int c = 0; c < nsteps && !*abort_flag; ++c) {
         const int st = c & 1;
-        if (c + 1 < nch) {
+        if (c + 1 < nsteps) {
           if (c >= 1 && !mbar_wait(&bars->kb_empty[(c + 1) & 1], ((c - 1) >> 1) & 1)) { fail(); break; }
           load(c + 1);
         }
@@ -173,18 +184,25 @@ topk_tc_kernel(const __grid_constant__ CUtensorMap tmHi, const __grid_constant__
       fence_proxy_async_smem();
       mbar_arrive(&bars->q_full);
     }
-    // Lane l keeps entry l of the sorted lists of the warp's 32 rows; K = topk - 1 <= 31
-    // entries are kept (lanes >= K hold the next-best values, also sorted).
-    const int K = g.topk - 1;
-    float ls[32];
-    int lj[32];
-#pragma unroll
-    for (int rr = 0; rr < 32; ++rr) { ls[rr] = -CUDART_INF_F; lj[rr] = -1; }
-    const int64_t row0 = t0 + warp * 32;          // first token of this warp's rows
-    float* wbuf = sbuf + warp * 32 * kSPad;
+    const int K = g.topk - 1;                       // past blocks to select
+    const int64_t own = valid ? t / g.block : 0;
+    const int n_take = (int)(own < K ? own : K);
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
-    for (int c = 0; c < nch; ++c) {
+    // pass-1 list of group maxima, descending; entries >= K are spare
+    float gm[KM];
+#pragma unroll
+    for (int e = 0; e < KM; ++e) gm[e] = -CUDART_INF_F;
+    float T = -CUDART_INF_F;
+    int cnt = 0;
+    bool overflow = false;
+    for (int c = 0; c < nsteps; ++c) {
       const int st = c & 1;
+      const bool pass2 = c >= nch;
+      if (c == nch) {                                 // threshold for pass 2
+#pragma unroll
+        for (int e = 0; e < KM; ++e)
+          if (e == K - 1) T = gm[e];
+      }
       if (!mbar_wait_warp(&bars->acc_full[st], (c >> 1) & 1)) { fail(); break; }
       tc_fence_after();
       uint32_t sv[2][32];
@@ -193,66 +211,72 @@ topk_tc_kernel(const __grid_constant__ CUtensorMap tmHi, const __grid_constant__
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(&bars->acc_empty[st]);
+      const int j0 = (pass2 ? c - nch : c) * kChunk;
+      const int64_t rem = own - j0;
+      const int lim = rem <= 0 ? 0 : (rem >= kChunk ? kChunk : (int)rem);
+      if (!pass2) {
 #pragma unroll
-      for (int k = 0; k < 32; ++k) {
-        wbuf[lane * kSPad + k] = __uint_as_float(sv[0][k]);
-        wbuf[lane * kSPad + 32 + k] = __uint_as_float(sv[1][k]);
-      }
-      __syncwarp();
-      const int64_t j0 = (int64_t)c * kChunk;
+        for (int q4 = 0; q4 < kChunk / kGroup; ++q4) {
+          float v = -CUDART_INF_F;
 #pragma unroll
-      for (int rr = 0; rr < 32; ++rr) {
-        const int64_t tr = row0 + rr;
-        const int64_t own_r = tr < g.S ? tr / g.block : 0;
-        const int64_t rem = own_r - j0;
-        const int lim = K <= 0 ? 0 : (rem <= 0 ? 0 : (rem >= kChunk ? kChunk : (int)rem));
-        if (lim == 0) continue;                          // warp-uniform
-        const float s0 = wbuf[rr * kSPad + lane];
-        const float s1 = wbuf[rr * kSPad + 32 + lane];
-        float thr = __shfl_sync(0xffffffffu, ls[rr], K - 1);
+          for (int u = 0; u < kGroup; ++u) {
+            const int k = q4 * kGroup + u;
+            if (k < lim) v = fmaxf(v, __uint_as_float(sv[k >> 5][k & 31]));
+          }
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          const float sh = half ? s1 : s0;
-          unsigned m = __ballot_sync(0xffffffffu, sh > thr && half * 32 + lane < lim);
-          while (m) {                                    // ascending block index
-            const int src = __ffs(m) - 1;
-            m &= m - 1;
-            const float cs = __shfl_sync(0xffffffffu, sh, src);
-            if (!(cs > thr)) continue;                   // threshold rose meanwhile
-            const int cj = (int)(j0 + half * 32 + src);
-            const int p = __popc(__ballot_sync(0xffffffffu, ls[rr] >= cs));
-            const float us = __shfl_up_sync(0xffffffffu, ls[rr], 1);
-            const int uj = __shfl_up_sync(0xffffffffu, lj[rr], 1);
-            if (lane > p) { ls[rr] = us; lj[rr] = uj; }
-            else if (lane == p) { ls[rr] = cs; lj[rr] = cj; }
-            thr = __shfl_sync(0xffffffffu, ls[rr], K - 1);
+          for (int e = 0; e < KM; ++e) {           // bubble v into the descending list
+            const float hi = fmaxf(gm[e], v);
+            v = fminf(gm[e], v);
+            gm[e] = hi;
+          }
+        }
+      } else {
+#pragma unroll
+        for (int k = 0; k < kChunk; ++k) {
+          const float s = __uint_as_float(sv[k >> 5][k & 31]);
+          if (k < lim && s >= T) {
+            if (cnt < kCap) {
+              cand_s[cnt * kRows + r] = s;
+              cand_j[cnt * kRows + r] = j0 + k;
+              ++cnt;
+            } else {
+              overflow = true;
+            }
           }
         }
       }
-      __syncwarp();
     }
-    // Output: the kept past blocks ascending, then the own block, -1 padded.
-#pragma unroll 1
-    for (int rr = 0; rr < 32; ++rr) {
-      const int64_t tr = row0 + rr;
-      if (tr >= g.S) break;                              // warp-uniform
-      const int64_t own_r = tr / g.block;
-      const int n_take = (int)(own_r < K ? own_r : K);
-      int key = (lane < n_take) ? lj[rr] : 0x7fffffff;   // bitonic sort, ascending
-#pragma unroll
-      for (int size = 2; size <= 32; size <<= 1)
-#pragma unroll
-        for (int stride = size >> 1; stride > 0; stride >>= 1) {
-          const int other = __shfl_xor_sync(0xffffffffu, key, stride);
-          const bool up = ((lane & size) == 0);
-          const bool lower = (lane & stride) == 0;
-          key = (lower == up) ? min(key, other) : max(key, other);
+    if (valid) {
+      if (overflow) {
+        flags[(b * g.hkv + gg) * ((g.S + kFlagTile - 1) / kFlagTile) + t / kFlagTile] = 1;
+      } else {
+        // exact: the n_take best by (score desc, block index asc), then ascending order
+        int sel[33];
+        int n = 0;
+        for (int e = 0; e < n_take; ++e) {
+          int best = -1;
+          float bs = 0.f;
+          int bj = 0x7fffffff;
+          for (int x = 0; x < cnt; ++x) {
+            const int xj = cand_j[x * kRows + r];
+            if (xj < 0) continue;                      // taken
+            const float xs = cand_s[x * kRows + r];
+            if (best < 0 || xs > bs || (xs == bs && xj < bj)) { best = x; bs = xs; bj = xj; }
+          }
+          if (best < 0) break;
+          cand_j[best * kRows + r] = -1;
+          sel[n++] = bj;
         }
-      int val = key;
-      if (lane == n_take) val = (int)own_r;
-      else if (lane > n_take) val = -1;
-      if (lane < g.topk)
-        idx[((b * g.hkv + gg) * g.S + tr) * (int64_t)g.topk + lane] = val;
+        sel[n++] = (int)own;
+        for (int a2 = 1; a2 < n; ++a2) {
+          const int x = sel[a2];
+          int c2 = a2 - 1;
+          while (c2 >= 0 && sel[c2] > x) { sel[c2 + 1] = sel[c2]; --c2; }
+          sel[c2 + 1] = x;
+        }
+        int32_t* out = idx + ((b * g.hkv + gg) * g.S + t) * (int64_t)g.topk;
+        for (int e = 0; e < g.topk; ++e) out[e] = e < n ? sel[e] : -1;
+      }
     }
   }
   tc_fence_before();
@@ -264,18 +288,26 @@ topk_tc_kernel(const __grid_constant__ CUtensorMap tmHi, const __grid_constant__
 }
 
 
-template <int G>
+template <int G, int KM>
 cudaError_t run_topk_tc(const Shape& s, const CUtensorMap& mh, const CUtensorMap& ml,
-                        const void* q, int32_t* idx, int* err, cudaStream_t st) {
+                        const void* q, int32_t* idx, uint8_t* flags, int* err, cudaStream_t st) {
   const size_t smem = 1024 + 4 * (size_t)kHalf + 8 * (size_t)kKHalf +
-                      (size_t)kRows * kSPad * 4 + sizeof(TBars);
-  cudaError_t e = cudaFuncSetAttribute(topk_tc_kernel<G>,
+                      2 * (size_t)kCap * kRows * 4 + sizeof(TBars);
+  cudaError_t e = cudaFuncSetAttribute(topk_tc_kernel<G, KM>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   TopkGeom g{s.seq, s.nb, s.block, (int)s.hq, (int)s.hkv, (int)(s.hq / s.hkv), (int)s.topk};
   dim3 grid((unsigned)((s.seq + kRows - 1) / kRows), (unsigned)s.hkv, (unsigned)s.batch);
-  topk_tc_kernel<G><<<grid, kThreads, smem, st>>>(mh, ml, (const __nv_bfloat16*)q, idx, err, g);
+  topk_tc_kernel<G, KM><<<grid, kThreads, smem, st>>>(mh, ml, (const __nv_bfloat16*)q, idx, flags,
+                                                      err, g);
   return cudaGetLastError();
+}
+
+template <int G>
+cudaError_t run_topk_tc_k(const Shape& s, const CUtensorMap& mh, const CUtensorMap& ml,
+                          const void* q, int32_t* idx, uint8_t* flags, int* err, cudaStream_t st) {
+  if (s.topk - 1 <= 16) return run_topk_tc<G, 16>(s, mh, ml, q, idx, flags, err, st);
+  return run_topk_tc<G, 32>(s, mh, ml, q, idx, flags, err, st);
 }
 
 }  // namespace
@@ -289,18 +321,28 @@ bool tc_topk_supported(const Shape& s) {
   return true;
 }
 
-cudaError_t launch_topk_prefill_tc(const Shape& s, const void* q, const void* kbar_hi,
-                                   const void* kbar_lo, int32_t* idx, int* err, cudaStream_t st) {
+size_t topk_tc_flag_bytes(const Shape& s) {
+  return (size_t)s.batch * s.hkv * ((s.seq + kFlagTile - 1) / kFlagTile);
+}
+
+cudaError_t launch_topk_prefill_tc(const Shape& s, const void* q, const float* kbar,
+                                   const void* kbar_hi, const void* kbar_lo, int32_t* idx,
+                                   uint8_t* flags, int* err, cudaStream_t st) {
   CUtensorMap mh, ml;
   if (!make_bf16_2d_map(&mh, kbar_hi, s.batch * s.nb, s.hkv * kD, kChunk) ||
       !make_bf16_2d_map(&ml, kbar_lo, s.batch * s.nb, s.hkv * kD, kChunk))
     return cudaErrorInvalidValue;
+  cudaError_t e = cudaMemsetAsync(flags, 0, topk_tc_flag_bytes(s), st);
+  if (e != cudaSuccess) return e;
   switch (s.hq / s.hkv) {
-    case 1: return run_topk_tc<1>(s, mh, ml, q, idx, err, st);
-    case 2: return run_topk_tc<2>(s, mh, ml, q, idx, err, st);
-    case 4: return run_topk_tc<4>(s, mh, ml, q, idx, err, st);
-    default: return run_topk_tc<8>(s, mh, ml, q, idx, err, st);
+    case 1: e = run_topk_tc_k<1>(s, mh, ml, q, idx, flags, err, st); break;
+    case 2: e = run_topk_tc_k<2>(s, mh, ml, q, idx, flags, err, st); break;
+    case 4: e = run_topk_tc_k<4>(s, mh, ml, q, idx, flags, err, st); break;
+    default: e = run_topk_tc_k<8>(s, mh, ml, q, idx, flags, err, st); break;
   }
+  if (e != cudaSuccess) return e;
+  // rows whose candidate buffer overflowed: exact fp32 selection of their 64-token tiles
+  return launch_topk_prefill_flagged(s, q, kbar, idx, flags, kFlagTile, st);
 }
 
 }  // namespace msa

@@ -130,6 +130,23 @@ def test_topk_select_split_planes_vs_oracle(msa, w):
     assert n_strict > 0
 
 
+def test_selection_exact_ties_take_lowest_blocks(msa):
+    """All-zero queries make every block score exactly 0: the tensor-core selection's
+    candidate buffers overflow and its fallback must return the lowest block indices."""
+    w = mi.Workload("bf16_all_ties", "prefill", 1, 16384, 8, 2, 128, 128, 8, "bf16")
+    _, k, v = _inputs(w)
+    q = torch.zeros(1, w.seq, w.hq, w.d, dtype=torch.bfloat16, device="cuda")
+    kbar, hi, lo = msa.pool_keys(k, w.block, split=True)
+    idx = msa.topk_select(q, kbar, w.block, w.topk, w.hkv, kbar_hi=hi, kbar_lo=lo)
+    own = torch.arange(w.seq, device="cuda") // w.block
+    n_past = torch.clamp(own, max=w.topk - 1)
+    slot = torch.arange(w.topk, device="cuda")
+    want = torch.where(slot[None] < n_past[:, None], slot[None], torch.full_like(slot[None], -1))
+    want = torch.where(slot[None] == n_past[:, None], own[:, None], want)
+    for g in range(w.hkv):
+        assert torch.equal(idx[0, g].long(), want), g
+
+
 def test_out_of_range_index_sets_error_word_and_skips(msa):
     w = SMALL[1]
     q, k, v = _inputs(w)
