@@ -14,9 +14,10 @@
 //                      causal inside the own block), base-2 exponentials in fp32,
 //                      writes P_c as bf16 back into TMEM over S_c
 //   O_c = P_c V_c      tcgen05.mma with A from TMEM, B = V (MN-major) from shared memory
-// The epilogue merges the chunks and writes a normalised bf16 partial O plus its
-// log-sum-exp for (token, slot); a second kernel merges a row's partials into O.
-// TMEM columns: S_0 [0,128) S_1 [128,256) O_0 [256,384) O_1 [384,512).
+// O accumulates over the chunks in TMEM; the epilogue writes a normalised bf16 partial O
+// plus its log-sum-exp for (token, slot); a second kernel merges a row's partials into O.
+// TMEM columns: S/P of tile parity 0 [0,128), 1 [128,256); O of parity 0 [256,384),
+// 1 [384,512).
 #include <cudaTypedefs.h>
 #include <math_constants.h>
 
@@ -32,8 +33,6 @@ constexpr int kD = 128;
 constexpr int kRowsT = 128;          // rows per tile
 constexpr int kChunkKeys = 128;      // keys per MMA chunk
 constexpr int kSegKeys = 256;        // keys per segment
-constexpr int kThreads = 256;        // warps 0-3 softmax, 4 issuer, 5-7 gather
-constexpr int kGatherThreads = 96;
 constexpr uint32_t kTileBytes = 16384;   // 128 rows x 128 B
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -118,7 +117,7 @@ __global__ void invert_fill_kernel(const int32_t* __restrict__ idx, int* __restr
 __global__ void tile_table_kernel(const int* __restrict__ counts, const int* __restrict__ seg_off,
                                   const int* __restrict__ tile_off,
                                   const int* __restrict__ n_tiles, int4* __restrict__ tiles,
-                                  int64_t nseg, int tpt) {
+                                  int64_t nseg, int tpt, int64_t nseg_per_bg) {
   const int64_t tile = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (tile >= *n_tiles) return;
   int64_t lo = 0, hi = nseg;                     // largest s with tile_off[s] <= tile
@@ -129,16 +128,37 @@ __global__ void tile_table_kernel(const int* __restrict__ counts, const int* __r
   while (lo + 1 < nseg && tile_off[lo + 1] <= tile) ++lo;   // skip empty segments
   const int k = (int)(tile - tile_off[lo]);
   const int cnt = min(tpt, counts[lo] - k * tpt);
-  tiles[tile] = make_int4((int)lo, seg_off[lo] + k * tpt, cnt, 0);
+  // x = segment, y = first entry, z = entries, w = sequence * hkv + group
+  tiles[tile] = make_int4((int)lo, seg_off[lo] + k * tpt, cnt, (int)(lo / nseg_per_bg));
 }
 
 // ------------------------------------------------------------------ the tile kernel
+// Two tiles are in flight: tile n (the n-th of this CTA) uses TMEM set X = n & 1
+// (S_X at columns 128X, O_X at 256 + 128X), Q stage X and softmax warpgroup X.  The issuer
+// walks "rounds" of one or two consecutive tiles of the same block and issues, per key
+// chunk c, QK of both tiles then PV of both, so the tensor core works on one tile while
+// the other tile's warpgroup runs its softmax or epilogue.  MMAs of one thread run in
+// issue order, so a QK may reuse the TMEM of a P that an earlier PV reads; only thread
+// accesses of TMEM (softmax, epilogue) and TMA writes of K/V wait for MMA completion.  One O accumulator per tile:
+// chunk 1 reuses chunk 0's row max as its exponent reference unless the max grew by more
+// than 2^8, in which case that warp rescales O in TMEM after chunk 0's PV completed.
+constexpr int kMaxQStages = 4;
 struct __align__(8) Bars {
-  uint64_t q_full[2], q_empty[2], kv_full, s_full[2], p_full[2], o_full, o_empty;
+  uint64_t q_full[kMaxQStages], q_empty[kMaxQStages];
+  uint64_t s_full[2], p_full[2], pv_done[2], o_empty[2], kv_full;
   uint32_t tmem_base;
   int abort;
-  int tok[2][kRowsT];          // per Q stage: token of each tile slot (gather warps only)
 };
+
+// Q stages: a tile holds its stage until its last chunk's QK, so 256-key blocks (two
+// chunks, 128 KB of K/V) get 3 stages and 128-key blocks 4 (both fit 227 KB).
+__host__ __device__ constexpr int q_stages(int nch) { return nch == 1 ? 4 : 3; }
+
+constexpr int kThreads3 = 384;       // WG0 warps 0-3, WG1 warps 4-7, issuer 8, gather 9-11
+constexpr int kIssuerWarp = 8;
+constexpr int kGatherWarp0 = 9;
+constexpr int kGatherThreads = 96;
+constexpr float kRescaleLog2 = 8.f;  // chunk-1 max may exceed the reference by 2^8
 
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
@@ -146,8 +166,42 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// Decodes a tile record into (sequence, group, block, 256-key segment) with 32-bit math.
+struct TileId {
+  int b, gg, j, sub;
+};
+__device__ __forceinline__ TileId decode_tile(const int4& tl, const Geom& g) {
+  TileId d;
+  const int nbs = (int)g.nb * g.nsub;
+  const int js = tl.x - tl.w * nbs;
+  d.j = js / g.nsub;
+  d.sub = js - d.j * g.nsub;
+  d.b = tl.w / g.hkv;
+  d.gg = tl.w - d.b * g.hkv;
+  return d;
+}
+
+// 2^x on the FMA pipe, for part of the softmax exponentials: x = n + f with n = floor(x),
+// 2^f from a degree-4 polynomial fitted here to minimise the relative error on [0, 1)
+// (max 2.6e-6), and 2^n added to the exponent field.  Inputs below -126 return 2^-126.
+__device__ __forceinline__ float poly_exp2(float x) {
+  x = fmaxf(x, -126.f);
+  const float n = floorf(x);
+  const float f = x - n;
+  float p = fmaf(0.013534167241300929f, f, 0.052011461907036594f);
+  p = fmaf(p, f, 0.24144275612530167f);
+  p = fmaf(p, f, 0.6930038346109176f);
+  p = fmaf(p, f, 1.0000025933668424f);
+  return __int_as_float(__float_as_int(p) + ((int)n << 23));
+}
+
+// Phase parity of the per-chunk barriers for chunk c of this CTA's tile n.
+__device__ __forceinline__ uint32_t chunk_phase(int n, int c, int nch) {
+  return (uint32_t)(((n >> 1) * nch + c) & 1);
+}
+
 template <int G>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads3, 1)
 attn_tiles_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const __nv_bfloat16* __restrict__ q, const int4* __restrict__ tiles,
                   const int* __restrict__ n_tiles_p, const int* __restrict__ entries,
@@ -155,10 +209,13 @@ attn_tiles_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* base = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  unsigned char* Qs = base;                                   // 2 stages x 32 KB
-  unsigned char* Ks = base + 2 * 2 * kTileBytes;              // nch x 2 halves x 16 KB
-  unsigned char* Vs = Ks + g.nch * 2 * kTileBytes;
-  Bars* bars = reinterpret_cast<Bars*>(Vs + g.nch * 2 * kTileBytes);
+  const int nch = g.nch;
+  const int nqs = q_stages(nch);
+  unsigned char* Qs = base;                                   // nqs stages x 32 KB
+  unsigned char* Ks = base + nqs * 2 * kTileBytes;            // nch x 2 halves x 16 KB
+  unsigned char* Vs = Ks + nch * 2 * kTileBytes;
+  int* tok_all = reinterpret_cast<int*>(Vs + nch * 2 * kTileBytes);   // [nqs][kRowsT]
+  Bars* bars = reinterpret_cast<Bars*>(tok_all + nqs * kRowsT);
 
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   const int n_tiles = *n_tiles_p;
@@ -168,15 +225,17 @@ attn_tiles_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
   const int my_tiles = max(0, tile_hi - tile_lo);
 
   if (tid == 0) {
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < nqs; ++s) {
       mbar_init(&bars->q_full[s], kGatherThreads);
       mbar_init(&bars->q_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(&bars->s_full[s], 1);
       mbar_init(&bars->p_full[s], 128);
+      mbar_init(&bars->pv_done[s], 1);
+      mbar_init(&bars->o_empty[s], 128);
     }
     mbar_init(&bars->kv_full, 1);
-    mbar_init(&bars->o_full, 1);
-    mbar_init(&bars->o_empty, 128);
     bars->abort = 0;
     fence_mbar_init();
   }
@@ -192,7 +251,7 @@ attn_tiles_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
     *abort_flag = 1;
   };
 
-  if (warp == 4) {
+  if (warp == kIssuerWarp) {
     // ---------------------------------------------------------------- issuer
     if (lane == 0 && my_tiles > 0) {
       prefetch_tmap(&tmK);
@@ -201,19 +260,71 @@ attn_tiles_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
       const uint32_t idO = idesc_bf16(128, kD, 0, 1);
       int prev_seg = -1;
       uint32_t kvn = 0;
-      for (int n = 0; n < my_tiles; ++n) {
+      bool ok = true;
+      // Descriptor bases, computed once: an MMA k-step only adds a constant offset (in
+      // 16-byte units) to the start-address field.
+      // Q stages and K/V chunks are 32 KB apart: (2 * kTileBytes) >> 4 descriptor units.
+      constexpr uint64_t kStep = (2 * kTileBytes) >> 4;
+      const uint64_t qdesc0 = sdesc_sw128(smem_u32(Qs), 16, 1024);
+      const uint64_t kdesc0 = sdesc_sw128(smem_u32(Ks), 16, 1024);
+      const uint64_t vdesc0 = sdesc_sw128(smem_u32(Vs), kTileBytes, 1024);
+      // QK of tile m, chunk c, into S_X
+      auto issue_qk = [&](int m, int c) -> bool {
+        const int X = m & 1;
+        const int qs = m % nqs;
+        // S_X is overwritten while an earlier PV may still be reading P_X from it: the
+        // MMAs of this thread execute in issue order, so no completion wait is needed.
+        if (c == 0 && !mbar_wait(&bars->q_full[qs], (m / nqs) & 1)) return false;
+        tc_fence_after();
+        const uint64_t qd = qdesc0 + (uint64_t)qs * kStep, kd = kdesc0 + (uint64_t)c * kStep;
+        const uint32_t dt = tmem + X * 128;
+#pragma unroll
+        for (int s = 0; s < kD / 16; ++s) {
+          const uint64_t off = (uint64_t)((s >> 2) * (kTileBytes >> 4) + (s & 3) * 2);
+          umma_ss(dt, qd + off, kd + off, idS, s > 0);
+        }
+        umma_commit(&bars->s_full[X]);
+        if (c == nch - 1) umma_commit(&bars->q_empty[qs]);
+        return true;
+      };
+      // PV of tile m, chunk c, into O_X (P read from TMEM over S_X)
+      auto issue_pv = [&](int m, int c) -> bool {
+        const int X = m & 1;
+        if (!mbar_wait(&bars->p_full[X], chunk_phase(m, c, nch))) return false;
+        if (c == 0 && m >= 2 && !mbar_wait(&bars->o_empty[X], ((m >> 1) - 1) & 1)) return false;
+        tc_fence_after();
+        const uint64_t vd = vdesc0 + (uint64_t)c * kStep;
+        const uint32_t dt = tmem + 256 + X * 128, at = tmem + X * 128;
+#pragma unroll
+        for (int s = 0; s < kChunkKeys / 16; ++s)
+          umma_ts(dt, at + s * 8, vd + (uint64_t)(s * (2048 >> 4)), idO, (c > 0 || s > 0) ? 1u : 0u);
+        umma_commit(&bars->pv_done[X]);
+        return true;
+      };
+      int n = 0;
+      int4 tl_a = tiles[tile_lo];                                   // tile n
+      int4 tl_b = my_tiles > 1 ? tiles[tile_lo + 1] : make_int4(-1, 0, 0, 0);   // tile n+1
+      while (n < my_tiles && ok) {
         if (*abort_flag) break;
-        const int4 tl = tiles[tile_lo + n];
-        if (n > 0 && !mbar_wait(&bars->o_full, (n - 1) & 1)) { fail(); break; }
+        const int4 tl = tl_a;
+        const int pair = (n + 1 < my_tiles && tl_b.x == tl.x) ? 2 : 1;
+        // records of the next round's first two tiles, loaded ahead of time
+        const int nn = n + pair;
+        int4 nx_a = pair == 2 ? (nn < my_tiles ? tiles[tile_lo + nn] : make_int4(-1, 0, 0, 0))
+                              : tl_b;
+        const int4 nx_b = nn + 1 < my_tiles ? tiles[tile_lo + nn + 1] : make_int4(-1, 0, 0, 0);
         if (tl.x != prev_seg) {
-          const int64_t seg = tl.x;
-          const int sub = (int)(seg % g.nsub);
-          const int64_t j = (seg / g.nsub) % g.nb;
-          const int64_t gg = (seg / ((int64_t)g.nsub * g.nb)) % g.hkv;
-          const int64_t b = seg / ((int64_t)g.nsub * g.nb * g.hkv);
-          const int y0 = (int)(b * g.S + j * g.block + (int64_t)sub * kSegKeys);
-          mbar_arrive_expect_tx(&bars->kv_full, (uint32_t)(g.nch * 4 * kTileBytes));
-          for (int c = 0; c < g.nch; ++c)
+          // every MMA of earlier tiles must be done before K/V are overwritten
+          if (n > 0 && !mbar_wait(&bars->pv_done[(n - 1) & 1], chunk_phase(n - 1, nch - 1, nch))) {
+            ok = false;
+            break;
+          }
+          const TileId id = decode_tile(tl, g);
+          const int y0 = (int)((int64_t)id.b * g.S + (int64_t)id.j * g.block +
+                               (int64_t)id.sub * kSegKeys);
+          const int64_t gg = id.gg;
+          mbar_arrive_expect_tx(&bars->kv_full, (uint32_t)(nch * 4 * kTileBytes));
+          for (int c = 0; c < nch; ++c)
             for (int hf = 0; hf < 2; ++hf) {
               const int x = (int)(gg * kD + hf * 64);
               tma_load_2d(Ks + (c * 2 + hf) * kTileBytes, &tmK, &bars->kv_full, x,
@@ -221,57 +332,72 @@ attn_tiles_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
               tma_load_2d(Vs + (c * 2 + hf) * kTileBytes, &tmV, &bars->kv_full, x,
                           y0 + c * kChunkKeys);
             }
-          if (!mbar_wait(&bars->kv_full, kvn & 1)) { fail(); break; }
+          if (!mbar_wait(&bars->kv_full, kvn & 1)) { ok = false; break; }
           ++kvn;
           prev_seg = tl.x;
         }
-        const int st = n & 1;
-        if (!mbar_wait(&bars->q_full[st], (n >> 1) & 1)) { fail(); break; }
-        tc_fence_after();
-        const uint32_t qa = smem_u32(Qs + st * 2 * kTileBytes);
-        for (int c = 0; c < g.nch; ++c) {
-          const uint32_t ka = smem_u32(Ks + c * 2 * kTileBytes);
-          for (int s = 0; s < kD / 16; ++s) {
-            const uint32_t off = (uint32_t)(s >> 2) * kTileBytes + (uint32_t)(s & 3) * 32;
-            umma_ss(tmem + c * kChunkKeys, sdesc_sw128(qa + off, 16, 1024),
-                    sdesc_sw128(ka + off, 16, 1024), idS, s > 0);
-          }
-          umma_commit(&bars->s_full[c]);
+        for (int c = 0; c < nch && ok; ++c) {
+          for (int i = 0; i < pair && ok; ++i) ok = issue_qk(n + i, c);
+          for (int i = 0; i < pair && ok; ++i) ok = issue_pv(n + i, c);
         }
-        umma_commit(&bars->q_empty[st]);
-        if (n > 0 && !mbar_wait(&bars->o_empty, (n - 1) & 1)) { fail(); break; }
-        for (int c = 0; c < g.nch; ++c) {
-          if (!mbar_wait(&bars->p_full[c], n & 1)) { fail(); break; }
-          tc_fence_after();
-          const uint32_t va = smem_u32(Vs + c * 2 * kTileBytes);
-          for (int s = 0; s < kChunkKeys / 16; ++s)
-            umma_ts(tmem + 256 + c * kD, tmem + c * kChunkKeys + s * 8,
-                    sdesc_sw128(va + s * 2048, kTileBytes, 1024), idO, s > 0);
-        }
-        if (*abort_flag) break;
-        umma_commit(&bars->o_full);
+        n = nn;
+        tl_a = nx_a;
+        tl_b = nx_b;
       }
+      if (!ok) fail();
     }
-  } else if (warp >= 5) {
+  } else if (warp >= kGatherWarp0) {
     // ---------------------------------------------------------------- Q gather
-    const int gt = tid - 160;
+    // Tile n's copies are issued before waiting for tile n-1's, so two gathers are in
+    // flight; the next tile's record and token ids are loaded while copies run.
+    const int gt = tid - kGatherWarp0 * 32;
+    constexpr int kPerThread = (kRowsT / G + kGatherThreads - 1) / kGatherThreads;
+    int4 tl_n = my_tiles > 0 ? tiles[tile_lo] : make_int4(0, 0, 0, 0);
+    int ent_n[kPerThread];
+#pragma unroll
+    for (int u = 0; u < kPerThread; ++u) {
+      const int i = gt + u * kGatherThreads;
+      ent_n[u] = (my_tiles > 0 && i < kRowsT / G && i < tl_n.z) ? entries[tl_n.y + i] : -1;
+    }
+    int pending = -1;                                    // tile whose copies are in flight
     for (int n = 0; n < my_tiles; ++n) {
-      const int st = n & 1;
+      const int st = n % nqs;
       bool bad = *abort_flag != 0;
-      if (!bad && n >= 2 && !mbar_wait(&bars->q_empty[st], ((n >> 1) - 1) & 1)) {
-        fail();
-        bad = true;
+      if (!bad && n >= nqs) {
+        const uint32_t par = ((n / nqs) - 1) & 1;
+        // Never block on a stage while holding an unpublished tile: its consumer may be
+        // what frees the stage (with two key chunks, QK of tile n-1 needs tile n-1's Q
+        // before tile n-2's stage is released).
+        if (pending >= 0 && !mbar_try_wait(&bars->q_empty[st], par)) {
+          cp_async_wait_all();
+          fence_proxy_async_smem();
+          mbar_arrive(&bars->q_full[pending % nqs]);
+          pending = -1;
+        }
+        if (!mbar_wait(&bars->q_empty[st], par)) {
+          fail();
+          bad = true;
+        }
       }
-      const int4 tl = tiles[tile_lo + n];
-      const int64_t seg = tl.x;
-      const int64_t gg = (seg / ((int64_t)g.nsub * g.nb)) % g.hkv;
-      const int64_t b = seg / ((int64_t)g.nsub * g.nb * g.hkv);
-      unsigned char* qb = Qs + st * 2 * kTileBytes;
-      int* tk = bars->tok[st];
-      for (int i = gt; i < kRowsT / G; i += kGatherThreads)
-        tk[i] = i < tl.z ? (entries[tl.y + i] >> 6) : -1;
+      const int4 tl = tl_n;
+      int* tk = tok_all + st * kRowsT;
+#pragma unroll
+      for (int u = 0; u < kPerThread; ++u) {
+        const int i = gt + u * kGatherThreads;
+        if (i < kRowsT / G) tk[i] = ent_n[u] >= 0 ? (ent_n[u] >> 6) : -1;
+      }
       // all gather threads leave together: the token list is complete, or all abort
       if (bar_sync_or<1, kGatherThreads>(bad)) break;
+      if (n + 1 < my_tiles) {                            // prefetch the next tile's record
+        tl_n = tiles[tile_lo + n + 1];
+#pragma unroll
+        for (int u = 0; u < kPerThread; ++u) {
+          const int i = gt + u * kGatherThreads;
+          ent_n[u] = (i < kRowsT / G && i < tl_n.z) ? entries[tl_n.y + i] : -1;
+        }
+      }
+      const int64_t b = tl.w / g.hkv, gg = tl.w - b * g.hkv;
+      unsigned char* qb = Qs + st * 2 * kTileBytes;
       const __nv_bfloat16* qbase = q + (b * g.S * g.hq + gg * G) * kD;
 #pragma unroll 4
       for (int i = gt; i < kRowsT * 16; i += kGatherThreads) {
@@ -281,139 +407,159 @@ attn_tiles_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
         const __nv_bfloat16* src = qbase + ((int64_t)(valid ? t : 0) * g.hq + r % G) * kD + c * 8;
         cp_async16(qb + (c >> 3) * kTileBytes + r * 128 + (((c & 7) ^ (r & 7)) << 4), src, valid);
       }
+      cp_async_commit();
+      if (pending >= 0) {                                // the previous tile's copies landed
+        cp_async_wait_group1();
+        fence_proxy_async_smem();
+        mbar_arrive(&bars->q_full[pending % nqs]);
+      }
+      pending = n;
+    }
+    if (pending >= 0) {
       cp_async_wait_all();
       fence_proxy_async_smem();
-      mbar_arrive(&bars->q_full[st]);
+      mbar_arrive(&bars->q_full[pending % nqs]);
     }
   } else {
     // ---------------------------------------------------------------- softmax + epilogue
-    const int r = tid;                                   // TMEM lane = tile row
-    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    const int X = warp >> 2;                             // this warpgroup's tile parity
+    const int r = tid & 127;                             // TMEM lane = tile row
+    const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    const uint32_t sX = lane_base + X * 128, oX = lane_base + 256 + X * 128;
     const int tok = r / G, h = r % G;
-    int4 tl_next = my_tiles > 0 ? tiles[tile_lo] : make_int4(0, 0, 0, 0);
-    int e_next = (my_tiles > 0 && tok < tl_next.z) ? entries[tl_next.y + tok] : -1;
-    for (int n = 0; n < my_tiles; ++n) {
+    const float c2 = g.scale_log2;
+    int4 tl_next = X < my_tiles ? tiles[tile_lo + X] : make_int4(0, 0, 0, 0);
+    int e_next = (X < my_tiles && tok < tl_next.z) ? entries[tl_next.y + tok] : -1;
+    for (int n = X; n < my_tiles; n += 2) {
       if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
       const int4 tl = tl_next;
       const int ent = e_next;
-      if (n + 1 < my_tiles) {               // prefetch the next tile's row metadata
-        tl_next = tiles[tile_lo + n + 1];
+      if (n + 2 < my_tiles) {                            // this warpgroup's next tile
+        tl_next = tiles[tile_lo + n + 2];
         e_next = tok < tl_next.z ? entries[tl_next.y + tok] : -1;
       }
-      const int64_t seg = tl.x;
-      const int sub = (int)(seg % g.nsub);
-      const int64_t j = (seg / g.nsub) % g.nb;
-      const int64_t gg = (seg / ((int64_t)g.nsub * g.nb)) % g.hkv;
-      const int64_t b = seg / ((int64_t)g.nsub * g.nb * g.hkv);
+      const TileId id = decode_tile(tl, g);
+      const int sub = id.sub;
+      const int64_t j = id.j, gg = id.gg, b = id.b;
       const bool valid = ent >= 0;
       const int64_t t = valid ? (ent >> 6) : 0;
       const int pslot = valid ? (ent & 63) : 0;
-      const int64_t own = t / g.block;
+      const int64_t own = (int)t / (int)g.block;
       const int64_t kbase = j * g.block + (int64_t)sub * kSegKeys;
       int64_t khi = (j == own) ? t + 1 : j * g.block + g.block;
       const int64_t seg_end = j * g.block + min((int64_t)(sub + 1) * kSegKeys, g.block);
       khi = min(min(khi, seg_end), g.S);
-      float m_c[2] = {-CUDART_INF_F, -CUDART_INF_F}, l_c[2] = {0.f, 0.f};
+      float mref = -CUDART_INF_F;      // exponent reference (scaled, base 2)
+      float l = 0.f;
       bool ok = true;
-      for (int c = 0; c < g.nch; ++c) {
+      for (int c = 0; c < nch; ++c) {
         const int64_t rem = khi - (kbase + (int64_t)c * kChunkKeys);
         const int lim = valid ? (int)max((int64_t)0, min((int64_t)kChunkKeys, rem)) : 0;
-        if (!mbar_wait_warp(&bars->s_full[c], n & 1)) { ok = false; break; }
+        const uint32_t ph = chunk_phase(n, c, nch);
+        if (!mbar_wait_warp(&bars->s_full[X], ph)) { ok = false; break; }
         tc_fence_after();
-        uint32_t sv[4][32];
-#pragma unroll
-        for (int qd = 0; qd < 4; ++qd) tmem_ld32(lane_base + c * kChunkKeys + qd * 32, sv[qd]);
-        tmem_ld_wait();
-        // row max of the raw scores (scale > 0 commutes with max), then
-        // p = 2^(s * scale*log2e - max * scale*log2e) with one FFMA + ex2 per score
         const bool full = __all_sync(0xffffffffu, lim == kChunkKeys);
+        // pass 1: row max of the raw scores (two TMEM loads per wait)
         float mx = -CUDART_INF_F;
-        if (full) {
 #pragma unroll
-          for (int qd = 0; qd < 4; ++qd)
+        for (int hq2 = 0; hq2 < 2; ++hq2) {
+          uint32_t sv[2][32];
+          tmem_ld32(sX + hq2 * 64, sv[0]);
+          tmem_ld32(sX + hq2 * 64 + 32, sv[1]);
+          tmem_ld_wait();
 #pragma unroll
-            for (int k = 0; k < 32; ++k) mx = fmaxf(mx, __uint_as_float(sv[qd][k]));
-        } else {
+          for (int u = 0; u < 2; ++u) {
+            const int qd = hq2 * 2 + u;
+            if (full) {
 #pragma unroll
-          for (int qd = 0; qd < 4; ++qd)
+              for (int k = 0; k < 32; ++k) mx = fmaxf(mx, __uint_as_float(sv[u][k]));
+            } else {
 #pragma unroll
-            for (int k = 0; k < 32; ++k)
-              if (qd * 32 + k < lim) mx = fmaxf(mx, __uint_as_float(sv[qd][k]));
+              for (int k = 0; k < 32; ++k)
+                if (qd * 32 + k < lim) mx = fmaxf(mx, __uint_as_float(sv[u][k]));
+            }
+          }
         }
-        const float c2 = g.scale_log2;
-        const float mb = lim > 0 ? mx * c2 : 0.f;
-        // P packed two bf16 per 32-bit column, written in place over the consumed scores:
-        // chunk quarter qd lands in sv[qd / 2][(qd % 2) * 16 ...], already read.
+        const float mc = lim > 0 ? mx * c2 : -CUDART_INF_F;
+        // exponent reference: chunk 0 sets it; a later chunk keeps it unless its max is
+        // more than 2^8 larger, which requires rescaling O (after the earlier PV is done)
+        const bool need = mc > mref + kRescaleLog2;
+        if (c > 0 && __any_sync(0xffffffffu, need)) {
+          if (!mbar_wait_warp(&bars->pv_done[X], chunk_phase(n, c - 1, nch))) { ok = false; break; }
+          tc_fence_after();
+          const float f = need ? fast_exp2(mref - mc) : 1.f;
+#pragma unroll
+          for (int qd = 0; qd < 4; ++qd) {
+            uint32_t ov[32];
+            tmem_ld32(oX + qd * 32, ov);
+            tmem_ld_wait();
+#pragma unroll
+            for (int k = 0; k < 32; ++k) ov[k] = __float_as_uint(__uint_as_float(ov[k]) * f);
+            tmem_st32(oX + qd * 32, ov);
+          }
+          tmem_st_wait();
+          l *= f;
+        }
+        if (need) mref = mc;
+        const float mb = mref > -CUDART_INF_F ? mref : 0.f;
+        // pass 2: P = 2^(s*c2 - mref), packed two bf16 per column over S_X
         float sum = 0.f;
-        if (full) {
 #pragma unroll
-          for (int qd = 0; qd < 4; ++qd)
+        for (int hq2 = 0; hq2 < 2; ++hq2) {
+          uint32_t sv[2][32];
+          tmem_ld32(sX + hq2 * 64, sv[0]);
+          tmem_ld32(sX + hq2 * 64 + 32, sv[1]);
+          tmem_ld_wait();
+          uint32_t pk[32];
 #pragma unroll
-            for (int k = 0; k < 32; k += 2) {
-              const float p0 = fast_exp2(fmaf(__uint_as_float(sv[qd][k]), c2, -mb));
-              const float p1 = fast_exp2(fmaf(__uint_as_float(sv[qd][k + 1]), c2, -mb));
-              sum += p0 + p1;
-              sv[qd >> 1][(qd & 1) * 16 + k / 2] = pack_bf16x2(p0, p1);
-            }
-        } else {
-#pragma unroll
-          for (int qd = 0; qd < 4; ++qd)
+          for (int u = 0; u < 2; ++u)
 #pragma unroll
             for (int k = 0; k < 32; k += 2) {
-              const int kk = qd * 32 + k;
-              const float p0 =
-                  kk < lim ? fast_exp2(fmaf(__uint_as_float(sv[qd][k]), c2, -mb)) : 0.f;
-              const float p1 =
-                  kk + 1 < lim ? fast_exp2(fmaf(__uint_as_float(sv[qd][k + 1]), c2, -mb)) : 0.f;
+              const int kk = (hq2 * 2 + u) * 32 + k;
+              // one exponential in four on the FMA pipe, the rest on the MUFU unit
+              float p0 = fast_exp2(fmaf(__uint_as_float(sv[u][k]), c2, -mb));
+              const float x1 = fmaf(__uint_as_float(sv[u][k + 1]), c2, -mb);
+              float p1 = (k & 3) == 2 ? poly_exp2(x1) : fast_exp2(x1);
+              if (!full) {
+                p0 = kk < lim ? p0 : 0.f;
+                p1 = kk + 1 < lim ? p1 : 0.f;
+              }
               sum += p0 + p1;
-              sv[qd >> 1][(qd & 1) * 16 + k / 2] = pack_bf16x2(p0, p1);
+              pk[u * 16 + k / 2] = pack_bf16x2(p0, p1);
             }
+          tmem_st32(sX + hq2 * 32, pk);
         }
-        tmem_st32(lane_base + c * kChunkKeys, sv[0]);
-        tmem_st32(lane_base + c * kChunkKeys + 32, sv[1]);
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(&bars->p_full[c]);
-        m_c[c] = lim > 0 ? mb : -CUDART_INF_F;
-        l_c[c] = sum;
+        mbar_arrive(&bars->p_full[X]);
+        l += sum;
       }
-      if (!ok || !mbar_wait_warp(&bars->o_full, n & 1)) { fail(); break; }
+      if (!ok || !mbar_wait_warp(&bars->pv_done[X], chunk_phase(n, nch - 1, nch))) {
+        fail();
+        break;
+      }
       tc_fence_after();
-      const float M = fmaxf(m_c[0], m_c[1]);
-      float w[2];
-#pragma unroll
-      for (int c = 0; c < 2; ++c) w[c] = (c < g.nch && m_c[c] > -CUDART_INF_F) ? fast_exp2(m_c[c] - M) : 0.f;
-      const float L = w[0] * l_c[0] + w[1] * l_c[1];
-      const float inv = L > 0.f ? 1.f / L : 0.f;
+      const float inv = l > 0.f ? 1.f / l : 0.f;
       __nv_bfloat16* dst = po + ((((b * g.hkv + gg) * g.S + t) * g.kslots + pslot) * G + h) * kD;
 #pragma unroll 1
       for (int qd = 0; qd < 4; ++qd) {
-        uint32_t o0[32], o1[32];
-        tmem_ld32(lane_base + 256 + qd * 32, o0);
-        if (g.nch > 1) tmem_ld32(lane_base + 384 + qd * 32, o1);
+        uint32_t ov[32];
+        tmem_ld32(oX + qd * 32, ov);
         tmem_ld_wait();
         uint32_t ob[16];
 #pragma unroll
-        for (int k = 0; k < 32; k += 2) {
-          float a0 = __uint_as_float(o0[k]) * w[0], a1 = __uint_as_float(o0[k + 1]) * w[0];
-          if (g.nch > 1) {
-            a0 = fmaf(__uint_as_float(o1[k]), w[1], a0);
-            a1 = fmaf(__uint_as_float(o1[k + 1]), w[1], a1);
-          }
-          ob[k / 2] = pack_bf16x2(a0 * inv, a1 * inv);
-        }
+        for (int k = 0; k < 32; k += 2)
+          ob[k / 2] = pack_bf16x2(__uint_as_float(ov[k]) * inv, __uint_as_float(ov[k + 1]) * inv);
         if (valid) {
-          uint4* d4 = reinterpret_cast<uint4*>(dst + qd * 32);
-#pragma unroll
-          for (int v = 0; v < 4; ++v)
-            d4[v] = make_uint4(ob[v * 4], ob[v * 4 + 1], ob[v * 4 + 2], ob[v * 4 + 3]);
+          st_global_v8(dst + qd * 32, ob);
+          st_global_v8(dst + qd * 32 + 16, ob + 8);
         }
       }
       tc_fence_before();
-      mbar_arrive(&bars->o_empty);
+      mbar_arrive(&bars->o_empty[X]);
       if (valid)
         plse[(((b * g.hkv + gg) * g.S + t) * g.kslots + pslot) * G + h] =
-            L > 0.f ? (M + log2f(L)) * kLn2 : -CUDART_INF_F;
+            l > 0.f ? (mref + log2f(l)) * kLn2 : -CUDART_INF_F;
     }
   }
 
@@ -538,11 +684,12 @@ template <int G>
 cudaError_t run_tc(const Shape& s, const Geom& g, const CUtensorMap& mk, const CUtensorMap& mv,
                    const void* q, const int32_t* idx, void* o, float* lse, char* ws,
                    const WsLayout& L, int* err, cudaStream_t st) {
-  const size_t smem = 1024 + 2 * 2 * kTileBytes + (size_t)g.nch * 4 * kTileBytes + sizeof(Bars);
+  const size_t smem = 1024 + (size_t)q_stages(g.nch) * (2 * kTileBytes + kRowsT * 4) +
+                      (size_t)g.nch * 4 * kTileBytes + sizeof(Bars);
   cudaError_t e = cudaFuncSetAttribute(attn_tiles_kernel<G>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  attn_tiles_kernel<G><<<sm_count(), kThreads, smem, st>>>(
+  attn_tiles_kernel<G><<<sm_count(), kThreads3, smem, st>>>(
       mk, mv, (const __nv_bfloat16*)q, (const int4*)(ws + L.tiles), (const int*)(ws + L.n_tiles),
       (const int*)(ws + L.entries), (__nv_bfloat16*)(ws + L.po), (float*)(ws + L.plse), err, g);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -595,7 +742,8 @@ cudaError_t launch_attn_prefill_tc(const Shape& s, const void* q, const void* k,
   const int64_t n_tiles_max = n_sel * g.nsub / g.tpt + g.nseg + 1;
   tile_table_kernel<<<(unsigned)((n_tiles_max + 255) / 256), 256, 0, st>>>(
       (const int*)(ws + L.counts), (const int*)(ws + L.seg_off), (const int*)(ws + L.tile_off),
-      (const int*)(ws + L.n_tiles), (int4*)(ws + L.tiles), g.nseg, g.tpt);
+      (const int*)(ws + L.n_tiles), (int4*)(ws + L.tiles), g.nseg, g.tpt,
+      (int64_t)g.nb * g.nsub);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   switch (g.G) {
     case 1: return run_tc<1>(s, g, mk, mv, q, idx, o, lse, ws, L, err, st);
