@@ -51,21 +51,72 @@ __device__ __forceinline__ bool sub_has_keys(int64_t j, int64_t own, int64_t t, 
 }
 
 // ------------------------------------------------------------------ index inversion
-__global__ void invert_count_kernel(const int32_t* __restrict__ idx, int* __restrict__ counts,
-                                    int* err, Geom g, int64_t n) {
-  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (e >= n) return;
-  const int64_t row = e / g.topk;                // (b*hkv + gg)*S + t
-  const int64_t t = row % g.S, bg = row / g.S;
-  const int64_t j = idx[e];
-  if (j == -1) return;
-  const int64_t own = t / g.block;
-  if (j < -1 || j >= g.nb || j > own) {
-    set_device_error(err, MSA_DEVERR_IDX_RANGE);
-    return;
+// Counting and filling run per CTA over a range of kInvTokens tokens of one (sequence,
+// group): entries are first counted in a shared-memory histogram over that group's
+// segments, so the global atomics are one per non-empty segment per CTA instead of one
+// per entry.  The fill reserves each segment's range with one atomic and places its
+// entries with shared-memory atomics.  The order of entries inside a segment is not
+// defined; no row's arithmetic depends on it.
+constexpr int kInvTokens = 2048;
+constexpr int kInvThreads = 512;
+
+__device__ __forceinline__ bool sub_has_keys32(int j, int own, int t, int sub, const Geom& g) {
+  const int64_t lo = (int64_t)j * g.block + (int64_t)sub * kSegKeys;
+  if ((int64_t)sub * kSegKeys >= g.block || lo >= g.S) return false;
+  return j < own || lo <= t;
+}
+
+// FILL = false: add the CTA's counts to counts[]; FILL = true: write entries[].
+template <bool FILL>
+__global__ void __launch_bounds__(kInvThreads)
+invert_hist_kernel(const int32_t* __restrict__ idx, int* __restrict__ counts,
+                   int* __restrict__ cursor, int* __restrict__ entries, int* err, Geom g) {
+  extern __shared__ int hist[];                       // nb * nsub counters
+  const int nbs = (int)g.nb * g.nsub;
+  const int t0 = blockIdx.x * kInvTokens;
+  const int bg = blockIdx.y;                          // sequence * hkv + group
+  const int t1 = (int)min((int64_t)t0 + kInvTokens, g.S);
+  const int own_max = (t1 - 1) / (int)g.block;        // segments beyond it stay empty
+  const int used = min(nbs, (own_max + 1) * g.nsub);
+  for (int i = threadIdx.x; i < used; i += kInvThreads) hist[i] = 0;
+  __syncthreads();
+  const int32_t* irow = idx + ((int64_t)bg * g.S + t0) * g.topk;
+  const int n = (t1 - t0) * g.topk;
+  for (int e = threadIdx.x; e < n; e += kInvThreads) {
+    const int j = irow[e];
+    if (j == -1) continue;
+    const int t = t0 + e / g.topk;
+    const int own = t / (int)g.block;
+    if (j < -1 || j >= g.nb || j > own) {
+      if (!FILL) set_device_error(err, MSA_DEVERR_IDX_RANGE);
+      continue;
+    }
+    for (int sub = 0; sub < g.nsub; ++sub)
+      if (sub_has_keys32(j, own, t, sub, g)) atomicAdd(&hist[j * g.nsub + sub], 1);
   }
-  for (int sub = 0; sub < g.nsub; ++sub)
-    if (sub_has_keys(j, own, t, sub, g)) atomicAdd(&counts[(bg * g.nb + j) * g.nsub + sub], 1);
+  __syncthreads();
+  int* gcount = (FILL ? cursor : counts) + (int64_t)bg * nbs;
+  for (int i = threadIdx.x; i < used; i += kInvThreads) {
+    const int c = hist[i];
+    if (c == 0) continue;
+    const int base = atomicAdd(&gcount[i], c);        // FILL: reserve [base, base + c)
+    if (FILL) hist[i] = base;
+  }
+  if (!FILL) return;
+  __syncthreads();
+  for (int e = threadIdx.x; e < n; e += kInvThreads) {
+    const int j = irow[e];
+    if (j < 0 || j >= g.nb) continue;
+    const int t = t0 + e / g.topk;
+    const int own = t / (int)g.block;
+    if (j > own) continue;
+    const int slot = e % g.topk;
+    for (int sub = 0; sub < g.nsub; ++sub)
+      if (sub_has_keys32(j, own, t, sub, g)) {
+        const int pos = atomicAdd(&hist[j * g.nsub + sub], 1);
+        entries[pos] = (t << 6) | (slot * g.nsub + sub);
+      }
+  }
 }
 
 // Single-CTA exclusive scans: seg_off (entries), tile_off (tiles of tpt entries).
@@ -94,24 +145,6 @@ invert_scan_kernel(const int* __restrict__ counts, int* __restrict__ seg_off,
   }
   if (tid == 1023) { seg_off[nseg] = (int)s_e[1023]; tile_off[nseg] = (int)s_t[1023];
                      *n_tiles = (int)s_t[1023]; }
-}
-
-__global__ void invert_fill_kernel(const int32_t* __restrict__ idx, int* __restrict__ cursor,
-                                   int* __restrict__ entries, Geom g, int64_t n) {
-  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (e >= n) return;
-  const int slot = (int)(e % g.topk);
-  const int64_t row = e / g.topk;
-  const int64_t t = row % g.S, bg = row / g.S;
-  const int64_t j = idx[e];
-  if (j < 0 || j >= g.nb) return;
-  const int64_t own = t / g.block;
-  if (j > own) return;
-  for (int sub = 0; sub < g.nsub; ++sub)
-    if (sub_has_keys(j, own, t, sub, g)) {
-      const int pos = atomicAdd(&cursor[(bg * g.nb + j) * g.nsub + sub], 1);
-      entries[pos] = (int)((t << 6) | (slot * g.nsub + sub));
-    }
 }
 
 __global__ void tile_table_kernel(const int* __restrict__ counts, const int* __restrict__ seg_off,
@@ -572,36 +605,47 @@ attn_tiles_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
 }
 
 // ------------------------------------------------------------------ merge partials
-// One row = (sequence, group, token); G*16 threads per row, 8 output elements each.
+// One row = (sequence, group, token); G*8 threads per row, 16 output elements (32 bytes)
+// each.  One pass over the row's partials with a running max, four loads in flight.
+__device__ __forceinline__ void ld_global_nc_v8(const void* p, uint32_t* r) {
+  asm volatile("ld.global.nc.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                 "=r"(r[6]), "=r"(r[7])
+               : "l"(p));
+}
+
 template <int G>
-__global__ void merge_partials_kernel(const int32_t* __restrict__ idx,
-                                      const __nv_bfloat16* __restrict__ po,
-                                      const float* __restrict__ plse, __nv_bfloat16* __restrict__ o,
-                                      float* __restrict__ lse, Geom g, int64_t n_rows) {
-  constexpr int TPR = G * 16;
+__global__ void __launch_bounds__(128)
+merge_partials_kernel(const int32_t* __restrict__ idx, const __nv_bfloat16* __restrict__ po,
+                      const float* __restrict__ plse, __nv_bfloat16* __restrict__ o,
+                      float* __restrict__ lse, Geom g, int64_t n_rows) {
+  constexpr int TPR = G * 8;
   constexpr int RPC = 128 / TPR;
   const int64_t row = (int64_t)blockIdx.x * RPC + threadIdx.x / TPR;
   if (row >= n_rows) return;
   const int lt = threadIdx.x % TPR;
-  const int h = lt / 16;
-  const int64_t t = row % g.S, bg = row / g.S;
+  const int h = lt / 8;
+  const int t = (int)(row % g.S);
+  const int64_t bg = row / g.S;
   const int64_t gg = bg % g.hkv, b = bg / g.hkv;
-  const int64_t own = t / g.block;
+  const int own = t / (int)g.block;
   const int32_t* irow = idx + row * g.topk;
   const float* lrow = plse + row * g.kslots * G;
-  const __nv_bfloat16* prow = po + row * g.kslots * G * kD;
+  const __nv_bfloat16* prow = po + row * g.kslots * G * kD + lt * 16;
   float mx = -CUDART_INF_F, den = 0.f;
-  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  float acc[16];
+#pragma unroll
+  for (int e = 0; e < 16; ++e) acc[e] = 0.f;
   int ps_list[4];
   int np = 0;
   auto flush = [&]() {
     float lv[4];
-    uint4 raw[4];
+    uint32_t raw[4][8];
 #pragma unroll
     for (int u = 0; u < 4; ++u)
       if (u < np) {
         lv[u] = lrow[ps_list[u] * G + h];
-        raw[u] = ldg16(prow + (int64_t)ps_list[u] * G * kD + lt * 8);
+        ld_global_nc_v8(prow + (int64_t)ps_list[u] * G * kD, raw[u]);
       }
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
@@ -609,33 +653,38 @@ __global__ void merge_partials_kernel(const int32_t* __restrict__ idx,
       const float mn = fmaxf(mx, lv[u]);
       const float sc = exp2f((mx - mn) * kLog2e);
       const float wgt = exp2f((lv[u] - mn) * kLog2e);
-      float f[8];
-      Vec16<__nv_bfloat16>::unpack(raw[u], f);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[e] = fmaf(wgt, f[e], acc[e] * sc);
+      for (int e = 0; e < 8; ++e) {
+        acc[2 * e] = fmaf(wgt, bf16lo_to_f32(raw[u][e]), acc[2 * e] * sc);
+        acc[2 * e + 1] = fmaf(wgt, bf16hi_to_f32(raw[u][e]), acc[2 * e + 1] * sc);
+      }
       den = den * sc + wgt;
       mx = mn;
     }
     np = 0;
   };
-  for (int s = 0; s < g.topk; ++s) {
-    const int64_t j = irow[s];
+  for (int sl = 0; sl < g.topk; ++sl) {
+    const int j = irow[sl];
     if (j < 0 || j >= g.nb || j > own) continue;
     for (int sub = 0; sub < g.nsub; ++sub) {
-      if (!sub_has_keys(j, own, t, sub, g)) continue;
-      ps_list[np++] = s * g.nsub + sub;
+      if (!sub_has_keys32(j, own, t, sub, g)) continue;
+      ps_list[np++] = sl * g.nsub + sub;
       if (np == 4) flush();
     }
   }
   if (np > 0) flush();
   const float inv = den > 0.f ? 1.f / den : 0.f;
-  uint4 out;
-  out.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
-  out.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
-  out.z = pack_bf16x2(acc[4] * inv, acc[5] * inv);
-  out.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
-  *reinterpret_cast<uint4*>(o + ((b * g.S + t) * g.hq + gg * G) * kD + lt * 8) = out;
-  if (lse != nullptr && (lt % 16) == 0)
+  uint32_t out[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) out[e] = pack_bf16x2(acc[2 * e] * inv, acc[2 * e + 1] * inv);
+  __nv_bfloat16* dst = o + ((b * g.S + t) * g.hq + gg * G) * kD + lt * 16;
+  if ((reinterpret_cast<uintptr_t>(o) & 31) == 0) {   // the ABI only promises 16 bytes
+    st_global_v8(dst, out);
+  } else {
+    reinterpret_cast<uint4*>(dst)[0] = make_uint4(out[0], out[1], out[2], out[3]);
+    reinterpret_cast<uint4*>(dst)[1] = make_uint4(out[4], out[5], out[6], out[7]);
+  }
+  if (lse != nullptr && (lt % 8) == 0)
     lse[(b * g.hq + gg * G + h) * g.S + t] = den > 0.f ? mx + logf(den) : -CUDART_INF_F;
 }
 
@@ -694,7 +743,7 @@ cudaError_t run_tc(const Shape& s, const Geom& g, const CUtensorMap& mk, const C
       (const int*)(ws + L.entries), (__nv_bfloat16*)(ws + L.po), (float*)(ws + L.plse), err, g);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const int64_t rows = s.batch * s.hkv * s.seq;
-  const int rpc = 128 / (G * 16);
+  const int rpc = 128 / (G * 8);
   merge_partials_kernel<G><<<(unsigned)((rows + rpc - 1) / rpc), 128, 0, st>>>(
       idx, (const __nv_bfloat16*)(ws + L.po), (const float*)(ws + L.plse), (__nv_bfloat16*)o,
       lse, g, rows);
@@ -714,6 +763,7 @@ bool tc_attn_supported(const Shape& s) {
   if (s.seq >= ((int64_t)1 << 25)) return false;              // token fits 25 bits
   if (s.batch * s.hkv * s.seq * s.topk * nsub >= ((int64_t)1 << 31)) return false;
   if (s.batch * s.seq >= ((int64_t)1 << 31)) return false;    // TMA row coordinate
+  if (s.nb * nsub > 48 * 1024) return false;                  // inversion histogram in smem
   return true;
 }
 
@@ -732,13 +782,22 @@ cudaError_t launch_attn_prefill_tc(const Shape& s, const void* q, const void* k,
   cudaError_t e = cudaMemsetAsync(ws + L.counts, 0, g.nseg * 4, st);
   if (e != cudaSuccess) return e;
   const int64_t n_sel = s.batch * s.hkv * s.seq * s.topk;
-  const unsigned gb = (unsigned)((n_sel + 255) / 256);
-  invert_count_kernel<<<gb, 256, 0, st>>>(idx, (int*)(ws + L.counts), err, g, n_sel);
+  const size_t hsmem = (size_t)g.nb * g.nsub * sizeof(int);
+  if ((e = cudaFuncSetAttribute(invert_hist_kernel<false>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hsmem)) !=
+          cudaSuccess ||
+      (e = cudaFuncSetAttribute(invert_hist_kernel<true>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hsmem)) !=
+          cudaSuccess)
+    return e;
+  const dim3 hgrid((unsigned)((s.seq + kInvTokens - 1) / kInvTokens), (unsigned)(s.batch * s.hkv));
+  invert_hist_kernel<false><<<hgrid, kInvThreads, hsmem, st>>>(
+      idx, (int*)(ws + L.counts), nullptr, nullptr, err, g);
   invert_scan_kernel<<<1, 1024, 0, st>>>((const int*)(ws + L.counts), (int*)(ws + L.seg_off),
                                          (int*)(ws + L.cursor), (int*)(ws + L.tile_off),
                                          (int*)(ws + L.n_tiles), g.nseg, g.tpt);
-  invert_fill_kernel<<<gb, 256, 0, st>>>(idx, (int*)(ws + L.cursor), (int*)(ws + L.entries), g,
-                                         n_sel);
+  invert_hist_kernel<true><<<hgrid, kInvThreads, hsmem, st>>>(
+      idx, nullptr, (int*)(ws + L.cursor), (int*)(ws + L.entries), err, g);
   const int64_t n_tiles_max = n_sel * g.nsub / g.tpt + g.nseg + 1;
   tile_table_kernel<<<(unsigned)((n_tiles_max + 255) / 256), 256, 0, st>>>(
       (const int*)(ws + L.counts), (const int*)(ws + L.seg_off), (const int*)(ws + L.tile_off),

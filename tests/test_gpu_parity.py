@@ -169,6 +169,31 @@ def test_out_of_range_index_sets_error_word_and_skips(msa):
     assert torch.equal(o_bad[0, :w.seq - 1, :w.hq // w.hkv], o_ref[0, :w.seq - 1, :w.hq // w.hkv])
 
 
+def test_output_with_16_byte_alignment_only(msa):
+    """The ABI promises 16-byte alignment; an output that is not 32-byte aligned must
+    give the same result."""
+    w = SMALL[1]
+    q, k, v = _inputs(w)
+    kbar = msa.pool_keys(k, w.block)
+    idx = msa.topk_select(q, kbar, w.block, w.topk, w.hkv)
+    o_ref, lse_ref = msa.sparse_attn_fwd(q, k, v, idx, w.block, w.scale)
+    buf = torch.empty(q.numel() + 8, dtype=q.dtype, device="cuda")
+    o = buf[8:].view(q.shape)                       # 16 bytes past a 32-byte boundary
+    assert o.data_ptr() % 32 == 16
+    p = msa.params(batch=1, seq=w.seq, hq=w.hq, hkv=w.hkv, d=w.d, block=w.block, topk=w.topk,
+                   scale=w.scale, dtype=q.dtype)
+    ws = msa.workspace(p, msa.OP_SPARSE_ATTN)
+    import ctypes
+    from block_sparse_top_mean_b200 import _lib
+    P = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
+    st = _lib.load().msa_sparse_attn_fwd(ctypes.byref(p), P(q), P(k), P(v), P(idx), P(o), None,
+                                         P(ws), ws.numel(),
+                                         ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == 0
+    torch.cuda.synchronize()
+    assert torch.equal(o, o_ref)
+
+
 def test_prefill_is_deterministic(msa):
     w = SMALL[3]
     q, k, v = _inputs(w)
