@@ -188,7 +188,10 @@ class PrefillRunner:
         self.ptr = {k: P(getattr(self, k)) for k in ("q", "k", "v", "kbar", "khi", "klo", "idx", "o",
                                                      "lse", "ws")}
         self.pp = ctypes.byref(self.p)
-        self.launches_per_step = 3
+        # own kernels per step (memsets excluded): pool 1; selection: tensor-core pass +
+        # exact pass over flagged tiles = 2; attention: count, scan, fill, tile table,
+        # tiles, merge = 6
+        self.launches_per_step = 9
 
     def step(self, events=None):
         s = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
@@ -211,11 +214,122 @@ class PrefillRunner:
             events[3].record()
 
 
+class DecodeRunner:
+    """Decode of n_query queries against a bank resident in HBM, through the C ABI.  The
+    bank's pooled keys are computed once up front (offline encoding, not timed)."""
+
+    def __init__(self, w: mi.Workload, seed: int):
+        import block_sparse_top_mean_b200 as msa
+        from block_sparse_top_mean_b200 import _lib
+        self.msa, self.lib, self.w = msa, _lib.load(), w
+        self.q, self.k, self.v = mi.decode_inputs(w, device="cuda", seed=seed)
+        # the bank's routing keys as bf16 hi/lo planes (the tensor-core scan's input)
+        _, self.khi, self.klo = (t[0] for t in msa.pool_keys(self.k[None], w.block, split=True))
+        dev = self.q.device
+        self.p = msa.params(batch=1, seq=w.seq, hq=w.hq, hkv=w.hkv, d=w.d, block=w.block,
+                            topk=w.topk, scale=w.scale, dtype=self.q.dtype)
+        self.o = torch.empty_like(self.q)
+        self.lse = torch.empty(w.n_query, w.hq, dtype=torch.float32, device=dev)
+        self.idx = torch.empty(w.n_query, w.hkv, w.topk, dtype=torch.int32, device=dev)
+        n = self.lib.msa_workspace_bytes(ctypes.byref(self.p), _lib.OP_DECODE, w.n_query)
+        self.ws = torch.zeros(n, dtype=torch.uint8, device=dev)
+        self.check = _lib.check
+        P = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
+        self.ptr = {k: P(getattr(self, k)) for k in ("q", "k", "v", "khi", "klo", "idx", "o",
+                                                     "lse", "ws")}
+        self.pp = ctypes.byref(self.p)
+        self.launches_per_step = 4          # bank scan, list merge, attention rows, combine
+
+    def step(self, events=None):
+        s = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+        P, w = self.ptr, self.w
+        if events:
+            events[0].record()
+        self.check("msa_decode_fwd", self.lib.msa_decode_fwd(
+            self.pp, w.n_query, P["q"], None, P["khi"], P["klo"], P["k"], P["v"], P["idx"],
+            P["o"], P["lse"], P["ws"], self.ws.numel(), s))
+        if events:
+            events[1].record()
+
+
+def run_decode(args, world, rank, local):
+    w = mi.WORKLOADS[args.workload]
+    from block_sparse_top_mean_b200 import build
+    if rank == 0:
+        build.build()
+    barrier(world)
+    r = DecodeRunner(w, seed=rank)
+    work = decode_work(w)
+    for _ in range(args.warmup):
+        r.step()
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # the bank (41 GB) is far larger than L2; the pooled keys (0.6 GB) too
+    with ClockSampler(local) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        start.record()
+        for i in range(args.steps):
+            r.step(ev[i])
+        end.record()
+        torch.cuda.synchronize()
+        barrier(world)
+    ms = max_over_ranks(start.elapsed_time(end) / args.steps, world)
+    peaks, peak_src = load_peaks()
+    # bytes the step must move at least: the pooled-key bank once at 4 bytes per element
+    # (bf16 hi + lo planes, as exact as fp32 for the selection), the selected K/V blocks
+    # once per (query, group)
+    kbar_bytes = float(w.nb * w.hkv * w.d * 4)
+    alg_bytes = kbar_bytes + work["attn_bytes"]
+    gbs = alg_bytes / (ms * 1e-3) / 1e9
+    roof = {"bound": "hbm", "kernel": "decode step (scan + merge + attention + combine)",
+            "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": round(gbs / peaks["hbm_gbs"], 4), "peak_source": f"hbm_gbs of {peak_src}",
+            "traffic": None, "algorithmic_per_launch": alg_bytes}
+    e2e = None
+    if not args.no_e2e:
+        hq_ = r.q.cpu().pin_memory()
+        ho = torch.empty(r.o.shape, dtype=r.o.dtype).pin_memory()
+
+        def one():
+            r.q.copy_(hq_, non_blocking=True)
+            r.step()
+            ho.copy_(r.o, non_blocking=True)
+        for _ in range(args.warmup):
+            one()
+        torch.cuda.synchronize()
+        s_, e_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s_.record()
+        for _ in range(args.steps):
+            one()
+        e_.record()
+        torch.cuda.synchronize()
+        ems = max_over_ranks(s_.elapsed_time(e_) / args.steps, world)
+        e2e = {"value": round(ems * 1e3, 1), "unit": "us/step", "ms_per_step": round(ems, 4),
+               "h2d_bytes_per_step": hq_.numel() * hq_.element_size(),
+               "d2h_bytes_per_step": ho.numel() * ho.element_size()}
+    line = {
+        "metric": "decode us/step", "value": round(ms * 1e3, 1), "unit": "us/step",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms, 4), "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": {"workload": w.name, "n_query": w.n_query, "bank_tokens": w.seq, "hq": w.hq,
+                   "hkv": w.hkv, "d": w.d, "block": w.block, "topk": w.topk,
+                   "l2": "bank and pooled keys larger than L2, no flush",
+                   "parallelism": f"{world} independent banks, one per GPU"},
+        "roofline": roof, "cpu_baseline": None, "e2e": e2e,
+        "gpu_launches": r.launches_per_step * args.steps, "clocks": clk.summary(),
+        "device_error_bits": r.msa.read_device_error(r.ws),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def run_ours(args, world, rank, local):
     w = mi.WORKLOADS[args.workload]
     if w.kind != "prefill":
-        raise SystemExit("decode workloads: use --workload with a prefill name (decode bench "
-                         "is reported in the extra field)")
+        return run_decode(args, world, rank, local)
     from block_sparse_top_mean_b200 import build
     if rank == 0:
         build.build()
@@ -357,12 +471,56 @@ def cpu_baseline_prefill(w, r, flops, n_blocks=64, n_tokens=96):
             "kind": "oracle", "sample": sample, "extrapolated_s_per_step": round(t_full, 1)}
 
 
+def run_reference_decode(args, world, w):
+    """Oracle decode on the host: a sample of the queries per step, extrapolated to all
+    n_query.  The bank's pooled keys are an input of the step (offline encoding); random
+    values of the right shape stand in for them, since only time is measured here."""
+    import oracle
+    from threadpoolctl import threadpool_limits
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from parity_util import HostView
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    q, kb, vb = mi.decode_inputs(w, device=dev, seed=0)
+    kbar = mi.normal((w.nb, w.hkv, w.d), 7, 7, "cpu", torch.float32).numpy().astype(np.float64)
+    Qd = q.float().cpu().numpy()
+    K, V = HostView(kb), HostView(vb)
+    n_s = 2
+    times = []
+    for s_ in range(args.warmup + args.steps):
+        qs = [(s_ * n_s + i) % w.n_query for i in range(n_s)]
+        with threadpool_limits(limits=1):
+            t0 = time.perf_counter()
+            oracle.decode_rows(Qd, kbar, K, V, w.seq, w.block, w.topk, w.scale, queries=qs)
+            t1 = time.perf_counter()
+        if s_ >= args.warmup:
+            times.append((t1 - t0) / n_s * w.n_query)
+    t = statistics.mean(times)
+    sample = (f"{n_s} of {w.n_query} queries (all {w.hkv} groups) per step, extrapolated to "
+              f"{w.n_query}; numpy fp64, 1 thread")
+    line = {
+        "impl": "reference", "metric": "decode us/step", "value": t * 1e6, "unit": "us/step",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3,
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": w.name, "n_query": w.n_query, "bank_tokens": w.seq, "hq": w.hq,
+                   "hkv": w.hkv, "d": w.d, "block": w.block, "topk": w.topk,
+                   "parallelism": "host oracle, rank 0 only"},
+        "cpu_baseline": {"value": t * 1e6, "unit": "us/step", "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": t * 1e6, "unit": "us/step", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
 def run_reference(args, world, rank):
     """The base contract's reference arm for this method: the fp64 CPU oracle, timed on the
     host cores on a bounded sample of the same workload."""
     if rank != 0:
         return
     w = mi.WORKLOADS[args.workload]
+    if w.kind == "decode":
+        return run_reference_decode(args, world, w)
     attn, score = prefill_flops(w)
     # inputs generated on the host in the same way (bounded: only what the sample touches)
     dev = "cuda" if torch.cuda.is_available() else "cpu"
@@ -403,8 +561,7 @@ def main():
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="prefill_1m_b256_k16",
-                    choices=[n for n, w in mi.WORKLOADS.items() if w.kind == "prefill"])
+    ap.add_argument("--workload", default="prefill_1m_b256_k16", choices=list(mi.WORKLOADS))
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

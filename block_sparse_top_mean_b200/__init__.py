@@ -148,8 +148,10 @@ def prefill_fwd(q, k, v, block: int, topk: int, scale=None, want_lse=True, ws=No
 
 
 def decode_fwd(q, kbar, k_bank, v_bank, block: int, topk: int, scale=None, kbar_hi=None,
-               want_lse=True, ws=None, out=None):
-    """Decode of q [n_query, hq, d] against a bank (k/v [S, hkv, d], kbar [nb, hkv, d]).
+               kbar_lo=None, want_lse=True, ws=None, out=None):
+    """Decode of q [n_query, hq, d] against a bank (k/v [S, hkv, d], pooled keys
+    [nb, hkv, d]: fp32 kbar and/or the bf16 hi/lo planes; with both planes and bf16 q,
+    d = 128, the tensor-core scan runs and kbar may be None).
     Returns (o, lse or None, idx [n_query, hkv, topk])."""
     nq, hq, d = q.shape
     S, hkv, _ = k_bank.shape
@@ -164,13 +166,13 @@ def decode_fwd(q, kbar, k_bank, v_bank, block: int, topk: int, scale=None, kbar_
     if ws is None:
         ws = workspace(p, OP_DECODE, nq, device=q.device)
     _lib.check("msa_decode_fwd", _lib.load().msa_decode_fwd(
-        ctypes.byref(p), nq, _ptr(q), _ptr(kbar), _ptr(kbar_hi), _ptr(k_bank), _ptr(v_bank),
-        _ptr(idx), _ptr(o), _ptr(lse), _ptr(ws), ws.numel(), _stream(q.device)))
+        ctypes.byref(p), nq, _ptr(q), _ptr(kbar), _ptr(kbar_hi), _ptr(kbar_lo), _ptr(k_bank),
+        _ptr(v_bank), _ptr(idx), _ptr(o), _ptr(lse), _ptr(ws), ws.numel(), _stream(q.device)))
     return o, lse, idx
 
 
 def decode_fwd_static(q, kbar, k_bank, v_bank, block: int, topk: int, scale=None,
-                      kbar_hi=None, want_lse=True, out=None):
+                      kbar_hi=None, kbar_lo=None, want_lse=True, out=None):
     """decode_fwd without a workspace: the library's fixed device scratch is used (for
     callers that cannot allocate device memory; see msa_decode_fwd_static in msa.h)."""
     nq, hq, d = q.shape
@@ -184,8 +186,8 @@ def decode_fwd_static(q, kbar, k_bank, v_bank, block: int, topk: int, scale=None
         lse = torch.empty(nq, hq, dtype=torch.float32, device=q.device) if want_lse else None
         idx = torch.empty(nq, hkv, topk, dtype=torch.int32, device=q.device)
     _lib.check("msa_decode_fwd_static", _lib.load().msa_decode_fwd_static(
-        ctypes.byref(p), nq, _ptr(q), _ptr(kbar), _ptr(kbar_hi), _ptr(k_bank), _ptr(v_bank),
-        _ptr(idx), _ptr(o), _ptr(lse), _stream(q.device)))
+        ctypes.byref(p), nq, _ptr(q), _ptr(kbar), _ptr(kbar_hi), _ptr(kbar_lo), _ptr(k_bank),
+        _ptr(v_bank), _ptr(idx), _ptr(o), _ptr(lse), _stream(q.device)))
     return o, lse, idx
 
 

@@ -104,6 +104,14 @@ size_t decode_select_ws_bytes(const Shape& s, int64_t n_query);
 cudaError_t launch_topk_decode(const Shape& s, int64_t n_query, const void* q, const float* kbar,
                                int32_t* idx, void* ws, cudaStream_t st);
 
+// Tensor-core decode selection (bf16 queries, d = 128); see topk_decode_tc.cu.  Needs the
+// bank's pooled keys as bf16 hi/lo planes; workspace: per-CTA candidate lists.
+bool tc_decode_supported(const Shape& s);
+size_t topk_decode_tc_ws_bytes(const Shape& s, int64_t n_query);
+cudaError_t launch_topk_decode_tc(const Shape& s, int64_t n_query, const void* q,
+                                  const void* kbar_hi, const void* kbar_lo, int32_t* idx,
+                                  void* ws, int* err, cudaStream_t st);
+
 // Query-centric attention over selected blocks (SIMT, fp32 math).
 size_t decode_attn_ws_bytes(const Shape& s, int64_t n_query);
 cudaError_t launch_attn_prefill_rows(const Shape& s, const void* q, const void* k, const void* v,

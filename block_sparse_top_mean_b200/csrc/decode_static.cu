@@ -46,9 +46,9 @@ msa_status scratch_address(void** out) {
 
 extern "C" msa_status msa_decode_fwd_static(const msa_params* p, int64_t n_query, const void* q,
                                             const float* kbar, const void* kbar_hi,
-                                            const void* k_bank, const void* v_bank,
-                                            int32_t* idx, void* o, float* lse,
-                                            msa_stream_t stream) {
+                                            const void* kbar_lo, const void* k_bank,
+                                            const void* v_bank, int32_t* idx, void* o,
+                                            float* lse, msa_stream_t stream) {
   if (p == nullptr || n_query < 0) return MSA_ERR_INVALID_ARG;
   if (n_query == 0 || p->seq == 0) return MSA_OK;
   const size_t need = msa_workspace_bytes(p, MSA_OP_DECODE, n_query);
@@ -60,6 +60,6 @@ extern "C" msa_status msa_decode_fwd_static(const msa_params* p, int64_t n_query
   // Only the device error word must start at zero; the rest is written before it is read.
   if (cudaMemsetAsync(scratch, 0, msa::kWsHeader, (cudaStream_t)stream) != cudaSuccess)
     return MSA_ERR_CUDA;
-  return msa_decode_fwd(p, n_query, q, kbar, kbar_hi, k_bank, v_bank, idx, o, lse, scratch,
-                        kMsaDecodeStaticScratch, stream);
+  return msa_decode_fwd(p, n_query, q, kbar, kbar_hi, kbar_lo, k_bank, v_bank, idx, o, lse,
+                        scratch, kMsaDecodeStaticScratch, stream);
 }

@@ -55,6 +55,17 @@ size_t kbar_split_bytes(const Shape& s) {
   return msa::tc_topk_supported(s) ? (size_t)s.batch * s.nb * s.hkv * s.d * 2 : 0;
 }
 
+// Decode selection scratch: enough for the SIMT scan and, where it applies, the
+// tensor-core scan (which of the two runs depends on the planes the caller passes).
+size_t decode_sel_ws(const Shape& s, int64_t n_query) {
+  size_t n = msa::decode_select_ws_bytes(s, n_query);
+  if (msa::tc_decode_supported(s)) {
+    const size_t t = msa::topk_decode_tc_ws_bytes(s, n_query);
+    if (t > n) n = t;
+  }
+  return n;
+}
+
 size_t ws_bytes_for(const Shape& s, int op, int64_t n_query) {
   switch (op) {
     case MSA_OP_TOPK_SELECT:
@@ -66,7 +77,7 @@ size_t ws_bytes_for(const Shape& s, int op, int64_t n_query) {
              topk_flag_ws(s) +
              (msa::tc_attn_supported(s) ? round256(msa::tc_attn_ws_bytes(s)) : 0);
     case MSA_OP_DECODE:
-      return msa::kWsHeader + round256(msa::decode_select_ws_bytes(s, n_query)) +
+      return msa::kWsHeader + round256(decode_sel_ws(s, n_query)) +
              round256(msa::decode_attn_ws_bytes(s, n_query));
     default:
       return 0;
@@ -217,27 +228,31 @@ msa_status msa_prefill_fwd(const msa_params* p, const void* q, const void* k, co
 }
 
 msa_status msa_decode_fwd(const msa_params* p, int64_t n_query, const void* q, const float* kbar,
-                          const void* kbar_hi, const void* k_bank, const void* v_bank,
-                          int32_t* idx, void* o, float* lse, void* ws, size_t ws_bytes,
-                          msa_stream_t stream) {
-  (void)kbar_hi;
+                          const void* kbar_hi, const void* kbar_lo, const void* k_bank,
+                          const void* v_bank, int32_t* idx, void* o, float* lse, void* ws,
+                          size_t ws_bytes, msa_stream_t stream) {
   Shape s;
   msa_status st = check_params(p, true, &s);
   if (st != MSA_OK) return st;
   if (n_query < 0) return MSA_ERR_INVALID_ARG;
   if (n_query == 0 || s.seq == 0) return MSA_OK;
   if (n_query > 65535 * 64) return MSA_ERR_UNSUPPORTED;
-  if (q == nullptr || kbar == nullptr || k_bank == nullptr || v_bank == nullptr ||
+  // the tensor-core scan reads the bf16 planes; the SIMT scan the fp32 pooled keys
+  const bool tc = kbar_hi != nullptr && kbar_lo != nullptr && msa::tc_decode_supported(s);
+  if (q == nullptr || (!tc && kbar == nullptr) || k_bank == nullptr || v_bank == nullptr ||
       idx == nullptr || o == nullptr)
     return MSA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(kbar) || !aligned16(k_bank) || !aligned16(v_bank) ||
-      !aligned16(o))
+  if (!aligned16(q) || !aligned16(kbar) || !aligned16(kbar_hi) || !aligned16(kbar_lo) ||
+      !aligned16(k_bank) || !aligned16(v_bank) || !aligned16(o))
     return MSA_ERR_INVALID_ARG;
   if ((st = check_ws(s, MSA_OP_DECODE, n_query, ws, ws_bytes)) != MSA_OK) return st;
   cudaStream_t cs = (cudaStream_t)stream;
   char* sel_ws = ws_body(ws);
-  char* att_ws = sel_ws + round256(msa::decode_select_ws_bytes(s, n_query));
-  cudaError_t e = msa::launch_topk_decode(s, n_query, q, kbar, idx, sel_ws, cs);
+  char* att_ws = sel_ws + round256(decode_sel_ws(s, n_query));
+  cudaError_t e =
+      tc ? msa::launch_topk_decode_tc(s, n_query, q, kbar_hi, kbar_lo, idx, sel_ws, err_word(ws),
+                                      cs)
+         : msa::launch_topk_decode(s, n_query, q, kbar, idx, sel_ws, cs);
   if (e == cudaSuccess)
     e = msa::launch_attn_decode(s, n_query, q, k_bank, v_bank, idx, o, lse, att_ws, err_word(ws),
                                 cs);

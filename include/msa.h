@@ -162,13 +162,16 @@ MSA_API msa_status msa_prefill_fwd(const msa_params* p, const void* q, const voi
  * is attended; [MiniMax] per query and GQA group top-k):  for each query n and group g,
  * idx[n,g,:] = top-`topk` of all nb bank blocks by (score desc, index asc), ascending;
  * then exact attention of the group's heads over those blocks' keys, no mask.
- * p->seq is the number of bank tokens, p->batch is ignored.  kbar is the bank's pooled
- * keys from msa_pool_keys (fp32, required); kbar_hi may be NULL.
- * ws: msa_workspace_bytes(p, MSA_OP_DECODE, n_query). */
-MSA_API msa_status msa_decode_fwd(const msa_params* p, int64_t n_query, const void* q, const float* kbar,
-                          const void* kbar_hi, const void* k_bank, const void* v_bank,
-                          int32_t* idx, void* o, float* lse, void* ws, size_t ws_bytes,
-                          msa_stream_t stream);
+ * p->seq is the number of bank tokens, p->batch is ignored.  The bank's pooled keys come
+ * from msa_pool_keys, computed once when the bank is written ([MSA-DE]: offline):
+ *   - kbar_hi and kbar_lo (bf16 split planes, [nb, hkv, d]) both given, with bf16 queries
+ *     and d = 128: the tensor-core scan reads only the planes and kbar may be NULL;
+ *   - otherwise kbar (fp32) is required and the fp32 SIMT scan runs.
+ * ws: msa_workspace_bytes(p, MSA_OP_DECODE, n_query) (covers both scans). */
+MSA_API msa_status msa_decode_fwd(const msa_params* p, int64_t n_query, const void* q,
+                                  const float* kbar, const void* kbar_hi, const void* kbar_lo,
+                                  const void* k_bank, const void* v_bank, int32_t* idx, void* o,
+                                  float* lse, void* ws, size_t ws_bytes, msa_stream_t stream);
 
 /* Bytes of the fixed device scratch used by msa_decode_fwd_static (32 MiB). */
 #define MSA_DECODE_STATIC_SCRATCH_BYTES ((size_t)32 << 20)
@@ -193,8 +196,9 @@ MSA_API msa_status msa_decode_fwd(const msa_params* p, int64_t n_query, const vo
  *   - Device error bits are not reported to the caller (they live in the shared array). */
 MSA_API msa_status msa_decode_fwd_static(const msa_params* p, int64_t n_query, const void* q,
                                          const float* kbar, const void* kbar_hi,
-                                         const void* k_bank, const void* v_bank, int32_t* idx,
-                                         void* o, float* lse, msa_stream_t stream);
+                                         const void* kbar_lo, const void* k_bank,
+                                         const void* v_bank, int32_t* idx, void* o, float* lse,
+                                         msa_stream_t stream);
 
 /* Copies the workspace's device error word to *bits after synchronising `stream`;
  * returns MSA_ERR_DEVICE when any bit is set, else MSA_OK. */

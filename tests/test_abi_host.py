@@ -109,7 +109,7 @@ def test_empty_inputs_are_noops(lib):
         assert lib.msa_pool_keys(ctypes.byref(p), None, None, None, None, None) == _lib.MSA_OK
     p = _p()
     assert lib.msa_decode_fwd(ctypes.byref(p), 0, None, None, None, None, None, None, None,
-                              None, None, 0, None) == _lib.MSA_OK
+                              None, None, None, 0, None) == _lib.MSA_OK
 
 
 def test_status_strings(lib):

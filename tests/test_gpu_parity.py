@@ -220,6 +220,74 @@ def test_decode_small(msa, w):
     check_decode(q, kbar_np, kb, vb, w.block, w.topk, w.scale, idx, o, lse)
 
 
+# Tensor-core bank scan (bf16 hi/lo planes of the pooled keys): several chunks per CTA,
+# CTAs that span two groups, ragged last chunk, query tiles beyond 64, G = 1 / 2 / 4 / 8,
+# topk below 32 and a bank with fewer blocks than topk.
+DECODE_TC = [
+    mi.Workload("dtc_b50k_g4", "decode", 1, 50_000, 32, 8, 128, 64, 32, "bf16", n_query=8),
+    mi.Workload("dtc_b300k_q100", "decode", 1, 300_000, 32, 8, 128, 64, 32, "bf16",
+                n_query=100),
+    mi.Workload("dtc_g1_k7", "decode", 1, 200_003, 8, 8, 128, 64, 7, "bf16", n_query=65),
+    mi.Workload("dtc_g2_b128", "decode", 1, 400_000, 16, 8, 128, 128, 16, "bf16", n_query=33),
+    mi.Workload("dtc_g8_hkv4", "decode", 1, 1_000_000, 32, 4, 128, 64, 32, "bf16", n_query=64),
+    mi.Workload("dtc_tiny_bank", "decode", 1, 1000, 32, 8, 128, 64, 32, "bf16", n_query=5),
+]
+
+
+@pytest.mark.parametrize("w", DECODE_TC, ids=lambda w: w.name)
+def test_decode_tc_scan(msa, w):
+    q, kb, vb = mi.decode_inputs(w, device="cuda")
+    kbar, khi, klo = (t[0] for t in msa.pool_keys(kb[None], w.block, split=True))
+    o, lse, idx = msa.decode_fwd(q, None, kb, vb, w.block, w.topk, w.scale, kbar_hi=khi,
+                                 kbar_lo=klo)
+    torch.cuda.synchronize()
+    kbar_np = pool_keys_chunked(kb[None], w.block)[0]
+    qs = list(range(w.n_query)) if w.n_query <= 16 else list(range(0, w.n_query, 3))
+    check_decode(q, kbar_np, kb, vb, w.block, w.topk, w.scale, idx, o, lse, queries=qs)
+
+
+def test_decode_tc_scan_exact_ties(msa):
+    # zero queries: every score is exactly 0, so the lowest block indices win
+    w = mi.Workload("dtc_ties", "decode", 1, 100_000, 32, 8, 128, 64, 32, "bf16", n_query=4)
+    _, kb, vb = mi.decode_inputs(w, device="cuda")
+    q = torch.zeros(w.n_query, w.hq, w.d, dtype=torch.bfloat16, device="cuda")
+    _, khi, klo = (t[0] for t in msa.pool_keys(kb[None], w.block, split=True))
+    _, _, idx = msa.decode_fwd(q, None, kb, vb, w.block, w.topk, w.scale, kbar_hi=khi,
+                               kbar_lo=klo)
+    want = torch.arange(w.topk, dtype=torch.int32, device="cuda").expand_as(idx)
+    assert torch.equal(idx, want)
+
+
+def test_decode_tc_scan_rising_scores(msa):
+    # pooled keys that grow along the bank: for queries aligned with the drift every
+    # block beats the running 32nd best, so every chunk refills the candidate lists
+    w = mi.Workload("dtc_rising", "decode", 1, 250_000, 32, 8, 128, 64, 32, "bf16", n_query=6)
+    q, kb, vb = mi.decode_inputs(w, device="cuda")
+    u = mi.normal((w.hkv, w.d), 5, mi.STREAM_PLANT, "cuda", torch.float32)
+    u = u / u.norm(dim=-1, keepdim=True)
+    ramp = (torch.arange(w.seq, device="cuda", dtype=torch.float32) // w.block) * 2e-3
+    kb = (kb.float() + ramp[:, None, None] * u[None]).to(torch.bfloat16)
+    q = (q.float() + 0.5 * u.repeat_interleave(w.hq // w.hkv, 0)[None]).to(torch.bfloat16)
+    kbar, khi, klo = (t[0] for t in msa.pool_keys(kb[None], w.block, split=True))
+    o, lse, idx = msa.decode_fwd(q, None, kb, vb, w.block, w.topk, w.scale, kbar_hi=khi,
+                                 kbar_lo=klo)
+    torch.cuda.synchronize()
+    kbar_np = pool_keys_chunked(kb[None], w.block)[0]
+    check_decode(q, kbar_np, kb, vb, w.block, w.topk, w.scale, idx, o, lse)
+
+
+def test_decode_tc_matches_fp32_scan(msa):
+    w = DECODE_TC[1]
+    q, kb, vb = mi.decode_inputs(w, device="cuda")
+    kbar, khi, klo = (t[0] for t in msa.pool_keys(kb[None], w.block, split=True))
+    _, _, i_tc = msa.decode_fwd(q, None, kb, vb, w.block, w.topk, w.scale, kbar_hi=khi,
+                                kbar_lo=klo)
+    _, _, i_f32 = msa.decode_fwd(q, kbar, kb, vb, w.block, w.topk, w.scale)
+    # both exact up to fp32 rounding of near-ties: nearly every row agrees
+    agree = (i_tc == i_f32).all(dim=-1).float().mean().item()
+    assert agree > 0.95, agree
+
+
 # ------------------------------------------------------------------ full-size workloads
 
 FULL_PREFILL = ["prefill_tiny_s1k_f32", "prefill_32k_b512_k8", "prefill_128k_b128_k16_planted",
@@ -245,11 +313,16 @@ def test_prefill_full_size_sampled(msa, name):
     assert torch.isfinite(o.float()).all()
 
 
-def test_decode_full_size_sampled(msa):
+@pytest.mark.parametrize("scan", ["tc", "fp32"])
+def test_decode_full_size_sampled(msa, scan):
     w = mi.WORKLOADS["decode_bank10m_b64_k32"]
     q, kb, vb = mi.decode_inputs(w, device="cuda")
-    kbar = msa.pool_keys(kb[None], w.block)[0]
-    o, lse, idx = msa.decode_fwd(q, kbar, kb, vb, w.block, w.topk, w.scale)
+    kbar, khi, klo = (t[0] for t in msa.pool_keys(kb[None], w.block, split=True))
+    if scan == "tc":
+        o, lse, idx = msa.decode_fwd(q, None, kb, vb, w.block, w.topk, w.scale, kbar_hi=khi,
+                                     kbar_lo=klo)
+    else:
+        o, lse, idx = msa.decode_fwd(q, kbar, kb, vb, w.block, w.topk, w.scale)
     torch.cuda.synchronize()
     kbar_np = pool_keys_chunked(kb[None], w.block, tokens_per_chunk=1 << 21)[0]
     rep = check_decode(q, kbar_np, kb, vb, w.block, w.topk, w.scale, idx, o, lse,

@@ -25,20 +25,24 @@ def test_static_scratch_decode_matches_workspace_decode():
     w = mi.Workload("decode_static_check", "decode", 1, 60_000, 32, 8, 128, 64, 32, "bf16",
                     n_query=16)
     _, kb, vb = mi.decode_inputs(w, device="cuda")
-    kbar = msa.pool_keys(kb[None], w.block)[0]
+    kbar, khi, klo = (t[0] for t in msa.pool_keys(kb[None], w.block, split=True))
     p = msa.params(batch=1, seq=w.seq, hq=w.hq, hkv=w.hkv, d=w.d, block=w.block, topk=w.topk,
                    scale=w.scale, dtype=torch.bfloat16)
     assert lib.msa_workspace_bytes(ctypes.byref(p), _lib.OP_DECODE, w.n_query) <= 32 << 20
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     P = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
-    for call, seed in enumerate((11, 12)):          # two calls in a row, different queries
+    # two calls in a row with different queries: the fp32 scan, then the tensor-core scan
+    for call, (seed, split) in enumerate(((11, False), (12, True))):
         q = mi.normal((w.n_query, w.hq, w.d), seed, mi.STREAM_DECODE_Q, "cuda", torch.bfloat16)
-        o_ref, lse_ref, idx_ref = msa.decode_fwd(q, kbar, kb, vb, w.block, w.topk, w.scale)
+        hi, lo = (khi, klo) if split else (None, None)
+        o_ref, lse_ref, idx_ref = msa.decode_fwd(q, kbar, kb, vb, w.block, w.topk, w.scale,
+                                                 kbar_hi=hi, kbar_lo=lo)
         o = torch.empty_like(q)
         lse = torch.empty(w.n_query, w.hq, dtype=torch.float32, device="cuda")
         idx = torch.empty(w.n_query, w.hkv, w.topk, dtype=torch.int32, device="cuda")
-        st = lib.msa_decode_fwd_static(ctypes.byref(p), w.n_query, P(q), P(kbar), None, P(kb),
-                                       P(vb), P(idx), P(o), P(lse), stream)
+        Pn = lambda t: None if t is None else P(t)  # noqa: E731
+        st = lib.msa_decode_fwd_static(ctypes.byref(p), w.n_query, P(q), P(kbar), Pn(hi), Pn(lo),
+                                       P(kb), P(vb), P(idx), P(o), P(lse), stream)
         assert st == _lib.MSA_OK, (call, st)
         torch.cuda.synchronize()
         assert torch.equal(idx, idx_ref), call
@@ -55,6 +59,6 @@ def test_static_scratch_rejects_sizes_beyond_the_limit():
     n_query = 4096                                   # needs far more than 32 MiB
     assert lib.msa_workspace_bytes(ctypes.byref(p), _lib.OP_DECODE, n_query) > 32 << 20
     fake = ctypes.c_void_p(4096)
-    st = lib.msa_decode_fwd_static(ctypes.byref(p), n_query, fake, fake, None, fake, fake, fake,
-                                   fake, None, None)
+    st = lib.msa_decode_fwd_static(ctypes.byref(p), n_query, fake, fake, None, None, fake, fake,
+                                   fake, fake, None, None)
     assert st == _lib.MSA_ERR_WORKSPACE
