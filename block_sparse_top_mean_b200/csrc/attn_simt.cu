@@ -268,9 +268,11 @@ cudaError_t launch_attn_decode(const Shape& s, int64_t n_query, const void* q, c
   a.po = reinterpret_cast<float*>(ws);
   a.plse = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) +
                                     ((np * s.d * sizeof(float) + 255) / 256) * 256);
-  if (a.nsplit == 1) { a.o = o; a.lse = lse; }
-  cudaError_t e = dispatch(s, a, st);
-  if (e != cudaSuccess || a.nsplit == 1) return e;
+  const bool tc = tc_decode_attn_supported(s) && decode_attn_tc_nsplit(s) == a.nsplit;
+  if (a.nsplit == 1 && !tc) { a.o = o; a.lse = lse; }
+  cudaError_t e = tc ? launch_attn_decode_tc(s, n_query, q, k, v, idx, a.po, a.plse, err, st)
+                     : dispatch(s, a, st);
+  if (e != cudaSuccess || (a.nsplit == 1 && !tc)) return e;
   const int64_t tasks = a.n_rows * G;
   const unsigned grid = (unsigned)((tasks + 3) / 4);
   if (s.dtype == MSA_BF16) {

@@ -112,6 +112,15 @@ cudaError_t launch_topk_decode_tc(const Shape& s, int64_t n_query, const void* q
                                   const void* kbar_hi, const void* kbar_lo, int32_t* idx,
                                   void* ws, int* err, cudaStream_t st);
 
+// Decode attention streamed through shared memory on mma.sync (bf16, d = 128,
+// block % 64 == 0); see attn_decode_tc.cu.  Writes per-split partials (normalised O and
+// lse, the same layout as the SIMT decode rows) for combine_splits_kernel.
+bool tc_decode_attn_supported(const Shape& s);
+int decode_attn_tc_nsplit(const Shape& s);
+cudaError_t launch_attn_decode_tc(const Shape& s, int64_t n_query, const void* q, const void* k,
+                                  const void* v, const int32_t* idx, float* po, float* plse,
+                                  int* err, cudaStream_t st);
+
 // Query-centric attention over selected blocks (SIMT, fp32 math).
 size_t decode_attn_ws_bytes(const Shape& s, int64_t n_query);
 cudaError_t launch_attn_prefill_rows(const Shape& s, const void* q, const void* k, const void* v,

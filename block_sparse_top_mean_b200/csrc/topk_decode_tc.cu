@@ -42,7 +42,7 @@ constexpr int kD = 128;
 constexpr int kM = 128;                   // bank blocks per chunk (MMA M, TMEM lanes)
 constexpr int kN = 64;                    // queries per CTA (MMA N)
 constexpr int kStages = 3;                // TMA ring of half-chunks (64 dims, hi + lo)
-constexpr int kAcc = 4;                   // TMEM accumulators of kN columns
+constexpr int kAcc = 8;                   // TMEM accumulators of kN columns (all 512)
 constexpr int kList = 32;                 // running list length per query (>= topk)
 constexpr int kPend = 160;                // pending keys per query: < 32 kept + 128 new
 constexpr int kEpiWarps = 8;
@@ -351,22 +351,28 @@ topk_decode_tc_kernel(const __grid_constant__ CUtensorMap tmHi,
           const int nq_here = nqv - qh * 32;       // valid queries of this warp's 32
           if (!valid || nq_here <= 0) pm = 0u;
           else if (nq_here < 32) pm &= (1u << nq_here) - 1u;
-          const uint32_t any = __reduce_or_sync(0xffffffffu, pm);
-          if (any != 0u) {
+          if (__any_sync(0xffffffffu, pm != 0u)) {
+            // lane n takes query 32*qh + n: transpose the 32x32 pass matrix (lanes =
+            // blocks, bits = queries), reserve that query's slots with one atomic per
+            // lane, then every block stores its keys at base + rank among the passes
+            uint32_t mt = pm;
+#pragma unroll
+            for (int sh = 16; sh > 0; sh >>= 1) {
+              const uint32_t lo = sh == 16 ? 0x0000ffffu : sh == 8 ? 0x00ff00ffu
+                                : sh == 4 ? 0x0f0f0f0fu : sh == 2 ? 0x33333333u : 0x55555555u;
+              const uint32_t o = __shfl_xor_sync(0xffffffffu, mt, sh);
+              mt = (lane & sh) ? ((mt & ~lo) | ((o >> sh) & lo)) : ((mt & lo) | ((o << sh) & ~lo));
+            }
+            const int nmine = __popc(mt);
+            int base = 0;
+            if (nmine > 0) base = atomicAdd(&cnt[qh * 32 + lane], nmine);
 #pragma unroll
             for (int n = 0; n < 32; ++n) {
-              if ((any >> n) & 1u) {
-                const bool pass = (pm >> n) & 1u;
-                const uint32_t m = __ballot_sync(0xffffffffu, pass);
-                const int leader = __ffs(m) - 1;
-                const int qn = qh * 32 + n;
-                int at = 0;
-                if (lane == leader) at = atomicAdd(&cnt[qn], __popc(m));
-                at = __shfl_sync(0xffffffffu, at, leader);
-                if (pass)
-                  pend[(size_t)qn * kPend + at + __popc(m & lt_mask)] =
-                      make_key(__uint_as_float(v[n]), j);
-              }
+              const uint32_t mn = __shfl_sync(0xffffffffu, mt, n);
+              const int bn = __shfl_sync(0xffffffffu, base, n);
+              if ((pm >> n) & 1u)
+                pend[(size_t)(qh * 32 + n) * kPend + bn + __popc(mn & lt_mask)] =
+                    make_key(__uint_as_float(v[n]), j);
             }
           }
         }
