@@ -63,7 +63,8 @@ struct __align__(8) DBars {
 struct DecGeom {
   int64_t nb;        // bank blocks
   int64_t n_query;
-  int64_t nch;       // chunks per group
+  int64_t nch;       // units (chunks visited) per group in this pass
+  int64_t stride;    // chunk index of unit c is c * stride (1, or the sample stride)
   int64_t per;       // units (group, chunk) per CTA along x
   int64_t nq_pad;    // query tiles * kN
   int hq, hkv, G, topk, ns_max, ncta_x;
@@ -152,7 +153,8 @@ __device__ __forceinline__ void joint_drain(uint64_t (&y)[kOwned], float (&T)[kO
       __syncwarp();
     }
     c[i] = rem > 0 ? rem : 0;
-    T[i] = key_score(__shfl_sync(0xffffffffu, y[i], kList - 1));
+    // never below a starting bound the list has not reached yet
+    T[i] = fmaxf(T[i], key_score(__shfl_sync(0xffffffffu, y[i], kList - 1)));
   }
 }
 
@@ -160,8 +162,8 @@ template <int G>
 __global__ void __launch_bounds__(kThreads, 1)
 topk_decode_tc_kernel(const __grid_constant__ CUtensorMap tmHi,
                       const __grid_constant__ CUtensorMap tmLo,
-                      const __nv_bfloat16* __restrict__ q, uint64_t* __restrict__ cand, int* err,
-                      DecGeom g) {
+                      const __nv_bfloat16* __restrict__ q, const float* __restrict__ tinit,
+                      uint64_t* __restrict__ cand, int* err, DecGeom g) {
   const int64_t total = (int64_t)g.hkv * g.nch;
   const int64_t u0 = (int64_t)blockIdx.x * g.per;
   const int64_t u1 = u0 + g.per < total ? u0 + g.per : total;
@@ -211,7 +213,7 @@ topk_decode_tc_kernel(const __grid_constant__ CUtensorMap tmHi,
       int64_t step = 0;
       for (int64_t u = u0; u < u1 && !*abort_flag; ++u) {
         const int gg = (int)(u / g.nch);
-        const int y = (int)((u % g.nch) * kM);
+        const int y = (int)((u % g.nch) * g.stride * kM);
         for (int hf = 0; hf < 2; ++hf, ++step) {
           const int st = (int)(step % kStages);
           if (step >= kStages &&
@@ -320,6 +322,16 @@ topk_decode_tc_kernel(const __grid_constant__ CUtensorMap tmHi,
       }
       fence_proxy_async_smem();
       mbar_arrive(&bars->q_full);
+      if (tinit != nullptr) {
+        // a valid starting bound: 32 sampled blocks of this group score at least T0
+#pragma unroll
+        for (int i = 0; i < kOwned; ++i) {
+          const int n = warp + kEpiWarps * i;
+          T[i] = n < nqv ? tinit[(qt * kN + n) * g.hkv + gg] : -CUDART_INF_F;
+          if (lane == 0) Ts[n] = T[i];
+        }
+      }
+      asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
 
       for (; u < ue; ++u, ++tile) {
         const int a = (int)(tile % kAcc);
@@ -333,10 +345,7 @@ topk_decode_tc_kernel(const __grid_constant__ CUtensorMap tmHi,
           uint32_t v[32];
           tmem_ld32(lane_base + a * kN, v);
           tmem_ld_wait();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&bars->acc_empty[a]);
-          const int64_t j = (u % g.nch) * kM + quarter * 32 + lane;
+          const int64_t j = (u % g.nch) * g.stride * kM + quarter * 32 + lane;
           const bool valid = j < g.nb;
           // bit n: this block reaches T of query 32*qh + n
           uint32_t pm = 0u;
@@ -366,15 +375,24 @@ topk_decode_tc_kernel(const __grid_constant__ CUtensorMap tmHi,
             const int nmine = __popc(mt);
             int base = 0;
             if (nmine > 0) base = atomicAdd(&cnt[qh * 32 + lane], nmine);
-#pragma unroll
-            for (int n = 0; n < 32; ++n) {
-              const uint32_t mn = __shfl_sync(0xffffffffu, mt, n);
+            uint32_t any = __ballot_sync(0xffffffffu, nmine > 0);   // queries with passes
+            while (any != 0u) {
+              // the score column of query n is re-read from TMEM (a uniform column index)
+              const int n = __ffs(any) - 1;
+              any &= any - 1u;
+              const bool pass = (pm >> n) & 1u;
+              const uint32_t mn = __ballot_sync(0xffffffffu, pass);
               const int bn = __shfl_sync(0xffffffffu, base, n);
-              if ((pm >> n) & 1u)
+              const uint32_t sv = tmem_ld1(lane_base + a * kN + n);
+              tmem_ld_wait();
+              if (pass)
                 pend[(size_t)(qh * 32 + n) * kPend + bn + __popc(mn & lt_mask)] =
-                    make_key(__uint_as_float(v[n]), j);
+                    make_key(__uint_as_float(sv), j);
             }
           }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars->acc_empty[a]);
         }
         // every warp's appends of this chunk are in; owners merge, then republish T
         asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
@@ -441,7 +459,8 @@ topk_decode_tc_kernel(const __grid_constant__ CUtensorMap tmHi,
 // One warp per (query, group): merges the sorted lists of the CTAs that covered the
 // group, then writes the best `topk` block indices ascending (-1 padded).
 __global__ void topk_decode_merge_kernel(const uint64_t* __restrict__ cand,
-                                         int32_t* __restrict__ idx, DecGeom g) {
+                                         int32_t* __restrict__ idx, float* __restrict__ tout,
+                                         DecGeom g) {
   const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / 32;
   const int lane = threadIdx.x % 32;
   if (w >= g.n_query * g.hkv) return;
@@ -454,6 +473,12 @@ __global__ void topk_decode_merge_kernel(const uint64_t* __restrict__ cand,
   for (int64_t c = c_first; c <= c_last; ++c) {
     const int64_t row = ((int64_t)gg * g.ns_max + (c - c_first)) * g.nq_pad + n;
     y = warp_merge_desc(y, cand[row * kList + lane], lane);
+  }
+  if (tout != nullptr) {
+    // threshold mode: the 32nd best score of this pass (-inf when fewer were seen)
+    const uint64_t last = __shfl_sync(0xffffffffu, y, kList - 1);
+    if (lane == 0) tout[w] = key_score(last);
+    return;
   }
   // the best topk, ascending by block index (empty entries sort last)
   int j = (lane < g.topk && y != 0ull) ? key_block(y) : 0x7fffffff;
@@ -469,11 +494,17 @@ __global__ void topk_decode_merge_kernel(const uint64_t* __restrict__ cand,
   if (lane < g.topk) idx[w * g.topk + lane] = j == 0x7fffffff ? -1 : j;
 }
 
-DecGeom make_dgeom(const Shape& s, int64_t n_query) {
+// Sample pass: every kSampleStride-th chunk, when the bank has at least kSampleMinChunks
+// chunks per group (the sample then holds >= 16 chunks, 2048 blocks, per group).
+constexpr int64_t kSampleStride = 16;
+constexpr int64_t kSampleMinChunks = 256;
+
+DecGeom make_dgeom(const Shape& s, int64_t n_query, int64_t stride) {
   DecGeom g{};
   g.nb = s.nb;
   g.n_query = n_query;
-  g.nch = (s.nb + kM - 1) / kM;
+  g.stride = stride;
+  g.nch = ((s.nb + kM - 1) / kM + stride - 1) / stride;
   const int64_t qtiles = (n_query + kN - 1) / kN;
   g.nq_pad = qtiles * kN;
   const int sms = sm_count();
@@ -493,16 +524,19 @@ DecGeom make_dgeom(const Shape& s, int64_t n_query) {
   return g;
 }
 
+bool use_sample(const Shape& s) { return (s.nb + kM - 1) / kM >= kSampleMinChunks; }
+
 template <int G>
 cudaError_t run_scan(const DecGeom& g, const CUtensorMap& mh, const CUtensorMap& ml,
-                     const void* q, uint64_t* cand, int* err, cudaStream_t st) {
+                     const void* q, const float* tinit, uint64_t* cand, int* err,
+                     cudaStream_t st) {
   const size_t smem = smem_bytes();
   cudaError_t e = cudaFuncSetAttribute(topk_decode_tc_kernel<G>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const dim3 grid((unsigned)g.ncta_x, (unsigned)(g.nq_pad / kN));
-  topk_decode_tc_kernel<G><<<grid, kThreads, smem, st>>>(mh, ml, (const __nv_bfloat16*)q, cand,
-                                                         err, g);
+  topk_decode_tc_kernel<G><<<grid, kThreads, smem, st>>>(mh, ml, (const __nv_bfloat16*)q, tinit,
+                                                         cand, err, g);
   return cudaGetLastError();
 }
 
@@ -518,30 +552,54 @@ bool tc_decode_supported(const Shape& s) {
   return true;
 }
 
-size_t topk_decode_tc_ws_bytes(const Shape& s, int64_t n_query) {
-  const DecGeom g = make_dgeom(s, n_query);
+// Workspace: candidate lists [hkv][CTA slot][query][32] (sized for the larger of the two
+// passes), then the sample pass's thresholds [query][hkv].
+size_t cand_bytes(const DecGeom& g) {
   return (size_t)g.hkv * g.ns_max * g.nq_pad * kList * sizeof(uint64_t);
+}
+
+size_t topk_decode_tc_ws_bytes(const Shape& s, int64_t n_query) {
+  size_t c = cand_bytes(make_dgeom(s, n_query, 1));
+  if (use_sample(s)) {
+    const size_t c2 = cand_bytes(make_dgeom(s, n_query, kSampleStride));
+    if (c2 > c) c = c2;
+  }
+  return (c + 255) / 256 * 256 + (size_t)n_query * s.hkv * sizeof(float);
 }
 
 cudaError_t launch_topk_decode_tc(const Shape& s, int64_t n_query, const void* q,
                                   const void* kbar_hi, const void* kbar_lo, int32_t* idx,
                                   void* ws, int* err, cudaStream_t st) {
-  const DecGeom g = make_dgeom(s, n_query);
   CUtensorMap mh, ml;
   if (!make_bf16_2d_map(&mh, kbar_hi, s.nb, s.hkv * kD, kM) ||
       !make_bf16_2d_map(&ml, kbar_lo, s.nb, s.hkv * kD, kM))
     return cudaErrorInvalidValue;
+  const DecGeom g = make_dgeom(s, n_query, 1);
+  const bool sample = use_sample(s);
+  const DecGeom gs = make_dgeom(s, n_query, kSampleStride);
+  size_t c = cand_bytes(g);
+  if (sample && cand_bytes(gs) > c) c = cand_bytes(gs);
   uint64_t* cand = reinterpret_cast<uint64_t*>(ws);
-  cudaError_t e;
-  switch (g.G) {
-    case 1: e = run_scan<1>(g, mh, ml, q, cand, err, st); break;
-    case 2: e = run_scan<2>(g, mh, ml, q, cand, err, st); break;
-    case 4: e = run_scan<4>(g, mh, ml, q, cand, err, st); break;
-    default: e = run_scan<8>(g, mh, ml, q, cand, err, st); break;
-  }
-  if (e != cudaSuccess) return e;
+  float* tinit = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + (c + 255) / 256 * 256);
+  auto scan = [&](const DecGeom& gg, const float* t0) {
+    switch (gg.G) {
+      case 1: return run_scan<1>(gg, mh, ml, q, t0, cand, err, st);
+      case 2: return run_scan<2>(gg, mh, ml, q, t0, cand, err, st);
+      case 4: return run_scan<4>(gg, mh, ml, q, t0, cand, err, st);
+      default: return run_scan<8>(gg, mh, ml, q, t0, cand, err, st);
+    }
+  };
   const int64_t warps = n_query * s.hkv;
-  topk_decode_merge_kernel<<<(unsigned)((warps + 7) / 8), 256, 0, st>>>(cand, idx, g);
+  const unsigned mgrid = (unsigned)((warps + 7) / 8);
+  cudaError_t e;
+  if (sample) {
+    // every 16th chunk first: its exact 32nd best per (query, group) starts the full scan
+    if ((e = scan(gs, nullptr)) != cudaSuccess) return e;
+    topk_decode_merge_kernel<<<mgrid, 256, 0, st>>>(cand, nullptr, tinit, gs);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  if ((e = scan(g, sample ? tinit : nullptr)) != cudaSuccess) return e;
+  topk_decode_merge_kernel<<<mgrid, 256, 0, st>>>(cand, idx, nullptr, g);
   return cudaGetLastError();
 }
 

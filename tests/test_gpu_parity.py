@@ -231,6 +231,9 @@ DECODE_TC = [
     mi.Workload("dtc_g2_b128", "decode", 1, 400_000, 16, 8, 128, 128, 16, "bf16", n_query=33),
     mi.Workload("dtc_g8_hkv4", "decode", 1, 1_000_000, 32, 4, 128, 64, 32, "bf16", n_query=64),
     mi.Workload("dtc_tiny_bank", "decode", 1, 1000, 32, 8, 128, 64, 32, "bf16", n_query=5),
+    # >= 256 chunks of 128 blocks per group: a 1/16 sample pass seeds the thresholds
+    mi.Workload("dtc_sampled_2p5m", "decode", 1, 2_500_000, 8, 2, 128, 64, 32, "bf16",
+                n_query=40),
 ]
 
 
@@ -258,14 +261,17 @@ def test_decode_tc_scan_exact_ties(msa):
     assert torch.equal(idx, want)
 
 
-def test_decode_tc_scan_rising_scores(msa):
+@pytest.mark.parametrize("seq,hkv", [(250_000, 8), (2_500_000, 2)])
+def test_decode_tc_scan_rising_scores(msa, seq, hkv):
     # pooled keys that grow along the bank: for queries aligned with the drift every
     # block beats the running 32nd best, so every chunk refills the candidate lists
-    w = mi.Workload("dtc_rising", "decode", 1, 250_000, 32, 8, 128, 64, 32, "bf16", n_query=6)
+    # (the longer bank also runs the sample pass, whose thresholds then lag far behind)
+    w = mi.Workload("dtc_rising", "decode", 1, seq, 4 * hkv, hkv, 128, 64, 32, "bf16",
+                    n_query=6)
     q, kb, vb = mi.decode_inputs(w, device="cuda")
     u = mi.normal((w.hkv, w.d), 5, mi.STREAM_PLANT, "cuda", torch.float32)
     u = u / u.norm(dim=-1, keepdim=True)
-    ramp = (torch.arange(w.seq, device="cuda", dtype=torch.float32) // w.block) * 2e-3
+    ramp = (torch.arange(w.seq, device="cuda", dtype=torch.float32) // w.block) * (8.0 / w.nb)
     kb = (kb.float() + ramp[:, None, None] * u[None]).to(torch.bfloat16)
     q = (q.float() + 0.5 * u.repeat_interleave(w.hq // w.hkv, 0)[None]).to(torch.bfloat16)
     kbar, khi, klo = (t[0] for t in msa.pool_keys(kb[None], w.block, split=True))
