@@ -238,7 +238,9 @@ class DecodeRunner:
         self.ptr = {k: P(getattr(self, k)) for k in ("q", "k", "v", "khi", "klo", "idx", "o",
                                                      "lse", "ws")}
         self.pp = ctypes.byref(self.p)
-        self.launches_per_step = 4          # bank scan, list merge, attention rows, combine
+        # own kernels per step: sample scan, sample threshold, bank scan, list merge,
+        # attention, combine
+        self.launches_per_step = 6
 
     def step(self, events=None):
         s = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
@@ -283,7 +285,8 @@ def run_decode(args, world, rank, local):
     kbar_bytes = float(w.nb * w.hkv * w.d * 4)
     alg_bytes = kbar_bytes + work["attn_bytes"]
     gbs = alg_bytes / (ms * 1e-3) / 1e9
-    roof = {"bound": "hbm", "kernel": "decode step (scan + merge + attention + combine)",
+    roof = {"bound": "hbm", "kernel": "decode step (sample scan + threshold + scan + merge + "
+                                      "attention + combine)",
             "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": round(gbs / peaks["hbm_gbs"], 4), "peak_source": f"hbm_gbs of {peak_src}",
             "traffic": None, "algorithmic_per_launch": alg_bytes}

@@ -25,6 +25,9 @@
 //   - At the end of a group's range the owner flushes its lists, sorted, to the candidate
 //     array; topk_decode_merge_kernel merges the lists of the CTAs that shared the group
 //     and writes the selection ascending.
+// Long banks first run a sample pass over every 8th chunk that only records, per query,
+// the maximum score of each 32-block group; the 32nd largest of those maxima (32
+// different blocks reach it) seeds T for the full scan, so few blocks get appended.
 // Keys are 64-bit: order-preserving bits of the score above the complement of the block
 // index, so a larger key is a better block; key 0 is "empty".
 #include <cudaTypedefs.h>
@@ -75,16 +78,20 @@ constexpr size_t smem_bytes() {
          (size_t)kN * 8 + sizeof(DBars);
 }
 
-__device__ __forceinline__ uint64_t make_key(float s, int64_t j) {
+// Order-preserving unsigned bits of a (finite) score; 0 is below every score.
+__device__ __forceinline__ uint32_t score_ord(float s) {
   const uint32_t b = __float_as_uint(s + 0.0f);            // -0 -> +0
-  const uint32_t ord = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-  return ((uint64_t)ord << 32) | (uint32_t)(~(uint32_t)j);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
-__device__ __forceinline__ float key_score(uint64_t key) {
-  const uint32_t ord = (uint32_t)(key >> 32);
-  if (ord == 0u) return -CUDART_INF_F;                      // empty entry
-  const uint32_t b = (ord & 0x80000000u) ? (ord & 0x7fffffffu) : ~ord;
-  return __uint_as_float(b);
+__device__ __forceinline__ float ord_score(uint32_t ord) {
+  if (ord == 0u) return -CUDART_INF_F;
+  return __uint_as_float((ord & 0x80000000u) ? (ord & 0x7fffffffu) : ~ord);
+}
+__device__ __forceinline__ uint64_t make_key(float s, int64_t j) {
+  return ((uint64_t)score_ord(s) << 32) | (uint32_t)(~(uint32_t)j);
+}
+__device__ __forceinline__ float key_score(uint64_t key) {   // -inf for an empty entry
+  return ord_score((uint32_t)(key >> 32));
 }
 __device__ __forceinline__ int key_block(uint64_t key) {
   return (int)(~(uint32_t)key);
@@ -158,12 +165,16 @@ __device__ __forceinline__ void joint_drain(uint64_t (&y)[kOwned], float (&T)[kO
   }
 }
 
-template <int G>
+// GMAX: the sample pass.  Instead of candidate lists the epilogue writes, per query,
+// the maximum score of every 32-block group (its order-preserving bits) to gmax
+// [query][group][sampled group index].
+template <int G, bool GMAX>
 __global__ void __launch_bounds__(kThreads, 1)
 topk_decode_tc_kernel(const __grid_constant__ CUtensorMap tmHi,
                       const __grid_constant__ CUtensorMap tmLo,
                       const __nv_bfloat16* __restrict__ q, const float* __restrict__ tinit,
-                      uint64_t* __restrict__ cand, int* err, DecGeom g) {
+                      uint64_t* __restrict__ cand, uint32_t* __restrict__ gmax, int* err,
+                      DecGeom g) {
   const int64_t total = (int64_t)g.hkv * g.nch;
   const int64_t u0 = (int64_t)blockIdx.x * g.per;
   const int64_t u1 = u0 + g.per < total ? u0 + g.per : total;
@@ -340,6 +351,29 @@ topk_decode_tc_kernel(const __grid_constant__ CUtensorMap tmHi,
           fail();
           aborted = true;
         }
+        if constexpr (GMAX) {
+          if (!aborted) {
+            tc_fence_after();
+            uint32_t v[32];
+            tmem_ld32(lane_base + a * kN, v);
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->acc_empty[a]);
+            const int64_t j = (u % g.nch) * g.stride * kM + quarter * 32 + lane;
+            const bool valid = j < g.nb;
+            uint32_t mine = 0u;                   // lane n: group max of query 32*qh + n
+#pragma unroll
+            for (int n = 0; n < 32; ++n) {
+              const uint32_t m = __reduce_max_sync(0xffffffffu, valid ? score_ord(__uint_as_float(v[n])) : 0u);
+              if (lane == n) mine = m;
+            }
+            const int qn = qh * 32 + lane;
+            if (qn < nqv)
+              gmax[((qt * kN + qn) * g.hkv + gg) * (g.nch * 4) + (u % g.nch) * 4 + quarter] = mine;
+          }
+          continue;
+        }
         if (!aborted) {
           tc_fence_after();
           uint32_t v[32];
@@ -421,6 +455,7 @@ topk_decode_tc_kernel(const __grid_constant__ CUtensorMap tmHi,
         }
         asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
       }
+      if constexpr (GMAX) continue;
       // end of this group's range: flush the lists to this CTA's slot of group gg
       if (!aborted) {
         int any = 0;
@@ -459,8 +494,7 @@ topk_decode_tc_kernel(const __grid_constant__ CUtensorMap tmHi,
 // One warp per (query, group): merges the sorted lists of the CTAs that covered the
 // group, then writes the best `topk` block indices ascending (-1 padded).
 __global__ void topk_decode_merge_kernel(const uint64_t* __restrict__ cand,
-                                         int32_t* __restrict__ idx, float* __restrict__ tout,
-                                         DecGeom g) {
+                                         int32_t* __restrict__ idx, DecGeom g) {
   const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / 32;
   const int lane = threadIdx.x % 32;
   if (w >= g.n_query * g.hkv) return;
@@ -473,12 +507,6 @@ __global__ void topk_decode_merge_kernel(const uint64_t* __restrict__ cand,
   for (int64_t c = c_first; c <= c_last; ++c) {
     const int64_t row = ((int64_t)gg * g.ns_max + (c - c_first)) * g.nq_pad + n;
     y = warp_merge_desc(y, cand[row * kList + lane], lane);
-  }
-  if (tout != nullptr) {
-    // threshold mode: the 32nd best score of this pass (-inf when fewer were seen)
-    const uint64_t last = __shfl_sync(0xffffffffu, y, kList - 1);
-    if (lane == 0) tout[w] = key_score(last);
-    return;
   }
   // the best topk, ascending by block index (empty entries sort last)
   int j = (lane < g.topk && y != 0ull) ? key_block(y) : 0x7fffffff;
@@ -494,10 +522,29 @@ __global__ void topk_decode_merge_kernel(const uint64_t* __restrict__ cand,
   if (lane < g.topk) idx[w * g.topk + lane] = j == 0x7fffffff ? -1 : j;
 }
 
+// One warp per (query, group): T0 = the 32nd largest of the sampled 32-block group maxima
+// (a valid bound: 32 different blocks score at least T0), found bit by bit on the
+// order-preserving bits; -inf when fewer than 32 groups were sampled.
+__global__ void sample_threshold_kernel(const uint32_t* __restrict__ gmax, float* __restrict__ tout,
+                                        int64_t rows, int ngroups) {
+  const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / 32;
+  const int lane = threadIdx.x % 32;
+  if (w >= rows) return;
+  const uint32_t* vals = gmax + w * ngroups;
+  uint32_t prefix = 0u;
+  for (int bit = 31; bit >= 0; --bit) {
+    const uint32_t cand = prefix | (1u << bit);
+    int c = 0;
+    for (int i = lane; i < ngroups; i += 32) c += __ldg(vals + i) >= cand;
+    if (__reduce_add_sync(0xffffffffu, (uint32_t)c) >= 32u) prefix = cand;
+  }
+  if (lane == 0) tout[w] = ord_score(prefix);
+}
+
 // Sample pass: every kSampleStride-th chunk, when the bank has at least kSampleMinChunks
-// chunks per group (the sample then holds >= 16 chunks, 2048 blocks, per group).
-constexpr int64_t kSampleStride = 16;
-constexpr int64_t kSampleMinChunks = 256;
+// chunks per group (the sample then holds >= 16 chunks, 64 block groups, per group).
+constexpr int64_t kSampleStride = 8;
+constexpr int64_t kSampleMinChunks = 128;
 
 DecGeom make_dgeom(const Shape& s, int64_t n_query, int64_t stride) {
   DecGeom g{};
@@ -526,17 +573,17 @@ DecGeom make_dgeom(const Shape& s, int64_t n_query, int64_t stride) {
 
 bool use_sample(const Shape& s) { return (s.nb + kM - 1) / kM >= kSampleMinChunks; }
 
-template <int G>
+template <int G, bool GMAX>
 cudaError_t run_scan(const DecGeom& g, const CUtensorMap& mh, const CUtensorMap& ml,
-                     const void* q, const float* tinit, uint64_t* cand, int* err,
+                     const void* q, const float* tinit, uint64_t* cand, uint32_t* gmax, int* err,
                      cudaStream_t st) {
   const size_t smem = smem_bytes();
-  cudaError_t e = cudaFuncSetAttribute(topk_decode_tc_kernel<G>,
+  cudaError_t e = cudaFuncSetAttribute(topk_decode_tc_kernel<G, GMAX>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const dim3 grid((unsigned)g.ncta_x, (unsigned)(g.nq_pad / kN));
-  topk_decode_tc_kernel<G><<<grid, kThreads, smem, st>>>(mh, ml, (const __nv_bfloat16*)q, tinit,
-                                                         cand, err, g);
+  topk_decode_tc_kernel<G, GMAX><<<grid, kThreads, smem, st>>>(
+      mh, ml, (const __nv_bfloat16*)q, tinit, cand, gmax, err, g);
   return cudaGetLastError();
 }
 
@@ -558,13 +605,26 @@ size_t cand_bytes(const DecGeom& g) {
   return (size_t)g.hkv * g.ns_max * g.nq_pad * kList * sizeof(uint64_t);
 }
 
-size_t topk_decode_tc_ws_bytes(const Shape& s, int64_t n_query) {
-  size_t c = cand_bytes(make_dgeom(s, n_query, 1));
+// Workspace: candidate lists [hkv][CTA slot][query][32], the sample thresholds
+// [query][hkv] and the sampled group maxima [query][hkv][group].
+struct DecWs {
+  size_t cand, tinit, gmax, total;
+};
+DecWs dec_ws(const Shape& s, int64_t n_query) {
+  DecWs w{};
+  w.cand = 0;
+  w.tinit = (cand_bytes(make_dgeom(s, n_query, 1)) + 255) / 256 * 256;
+  w.gmax = w.tinit + ((size_t)n_query * s.hkv * sizeof(float) + 255) / 256 * 256;
+  w.total = w.gmax;
   if (use_sample(s)) {
-    const size_t c2 = cand_bytes(make_dgeom(s, n_query, kSampleStride));
-    if (c2 > c) c = c2;
+    const DecGeom gs = make_dgeom(s, n_query, kSampleStride);
+    w.total += (size_t)n_query * s.hkv * gs.nch * 4 * sizeof(uint32_t);
   }
-  return (c + 255) / 256 * 256 + (size_t)n_query * s.hkv * sizeof(float);
+  return w;
+}
+
+size_t topk_decode_tc_ws_bytes(const Shape& s, int64_t n_query) {
+  return dec_ws(s, n_query).total;
 }
 
 cudaError_t launch_topk_decode_tc(const Shape& s, int64_t n_query, const void* q,
@@ -576,30 +636,38 @@ cudaError_t launch_topk_decode_tc(const Shape& s, int64_t n_query, const void* q
     return cudaErrorInvalidValue;
   const DecGeom g = make_dgeom(s, n_query, 1);
   const bool sample = use_sample(s);
-  const DecGeom gs = make_dgeom(s, n_query, kSampleStride);
-  size_t c = cand_bytes(g);
-  if (sample && cand_bytes(gs) > c) c = cand_bytes(gs);
-  uint64_t* cand = reinterpret_cast<uint64_t*>(ws);
-  float* tinit = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + (c + 255) / 256 * 256);
-  auto scan = [&](const DecGeom& gg, const float* t0) {
-    switch (gg.G) {
-      case 1: return run_scan<1>(gg, mh, ml, q, t0, cand, err, st);
-      case 2: return run_scan<2>(gg, mh, ml, q, t0, cand, err, st);
-      case 4: return run_scan<4>(gg, mh, ml, q, t0, cand, err, st);
-      default: return run_scan<8>(gg, mh, ml, q, t0, cand, err, st);
-    }
-  };
-  const int64_t warps = n_query * s.hkv;
-  const unsigned mgrid = (unsigned)((warps + 7) / 8);
+  const DecWs L = dec_ws(s, n_query);
+  char* base = reinterpret_cast<char*>(ws);
+  uint64_t* cand = reinterpret_cast<uint64_t*>(base + L.cand);
+  float* tinit = reinterpret_cast<float*>(base + L.tinit);
+  uint32_t* gmax = reinterpret_cast<uint32_t*>(base + L.gmax);
   cudaError_t e;
   if (sample) {
-    // every 16th chunk first: its exact 32nd best per (query, group) starts the full scan
-    if ((e = scan(gs, nullptr)) != cudaSuccess) return e;
-    topk_decode_merge_kernel<<<mgrid, 256, 0, st>>>(cand, nullptr, tinit, gs);
+    // every 8th chunk first: the 32nd largest of its 32-block group maxima per
+    // (query, group) is a valid bound that starts the full scan
+    const DecGeom gs = make_dgeom(s, n_query, kSampleStride);
+    switch (gs.G) {
+      case 1: e = run_scan<1, true>(gs, mh, ml, q, nullptr, nullptr, gmax, err, st); break;
+      case 2: e = run_scan<2, true>(gs, mh, ml, q, nullptr, nullptr, gmax, err, st); break;
+      case 4: e = run_scan<4, true>(gs, mh, ml, q, nullptr, nullptr, gmax, err, st); break;
+      default: e = run_scan<8, true>(gs, mh, ml, q, nullptr, nullptr, gmax, err, st); break;
+    }
+    if (e != cudaSuccess) return e;
+    const int64_t rows = n_query * s.hkv;
+    sample_threshold_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(gmax, tinit, rows,
+                                                                       (int)(gs.nch * 4));
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  if ((e = scan(g, sample ? tinit : nullptr)) != cudaSuccess) return e;
-  topk_decode_merge_kernel<<<mgrid, 256, 0, st>>>(cand, idx, nullptr, g);
+  const float* t0 = sample ? tinit : nullptr;
+  switch (g.G) {
+    case 1: e = run_scan<1, false>(g, mh, ml, q, t0, cand, nullptr, err, st); break;
+    case 2: e = run_scan<2, false>(g, mh, ml, q, t0, cand, nullptr, err, st); break;
+    case 4: e = run_scan<4, false>(g, mh, ml, q, t0, cand, nullptr, err, st); break;
+    default: e = run_scan<8, false>(g, mh, ml, q, t0, cand, nullptr, err, st); break;
+  }
+  if (e != cudaSuccess) return e;
+  const int64_t warps = n_query * s.hkv;
+  topk_decode_merge_kernel<<<(unsigned)((warps + 7) / 8), 256, 0, st>>>(cand, idx, g);
   return cudaGetLastError();
 }
 
