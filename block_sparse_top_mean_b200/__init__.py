@@ -20,7 +20,8 @@ from ._lib import (  # noqa: F401
 
 __all__ = [
     "params", "workspace", "pool_keys", "block_scores", "topk_select", "sparse_attn_fwd",
-    "prefill_fwd", "decode_fwd", "decode_fwd_static", "read_device_error",
+    "prefill_fwd", "decode_fwd", "decode_fwd_static", "encode_bank", "decode_fwd_tiled",
+    "read_device_error",
     "clear_device_error", "version",
     "MsaError", "MsaParams",
 ]
@@ -188,6 +189,51 @@ def decode_fwd_static(q, kbar, k_bank, v_bank, block: int, topk: int, scale=None
     _lib.check("msa_decode_fwd_static", _lib.load().msa_decode_fwd_static(
         ctypes.byref(p), nq, _ptr(q), _ptr(kbar), _ptr(kbar_hi), _ptr(kbar_lo), _ptr(k_bank),
         _ptr(v_bank), _ptr(idx), _ptr(o), _ptr(lse), _stream(q.device)))
+    return o, lse, idx
+
+
+def _bank_params(q, seq, hkv, block, topk, scale):
+    nq, hq, d = q.shape
+    return params(batch=1, seq=seq, hq=hq, hkv=hkv, d=d, block=block, topk=topk,
+                  scale=scale if scale is not None else d ** -0.5, dtype=q.dtype)
+
+
+def encode_bank(k_bank, v_bank, kbar_hi, kbar_lo, block: int):
+    """Encoded images of a bank (see msa_encode_bank): returns (k_tiles, v_tiles,
+    kbar_tiles) as uint8 CUDA tensors."""
+    S, hkv, d = k_bank.shape
+    p = params(batch=1, seq=S, hq=hkv, hkv=hkv, d=d, block=block, topk=1, scale=1.0,
+               dtype=k_bank.dtype)
+    lib = _lib.load()
+    nkv, nkb = lib.msa_bank_tiles_bytes(ctypes.byref(p), 0), lib.msa_bank_tiles_bytes(ctypes.byref(p), 1)
+    if nkv == 0 or nkb == 0:
+        raise MsaError("msa_bank_tiles_bytes", _lib.MSA_ERR_INVALID_ARG, "invalid shapes")
+    dev = k_bank.device
+    kt = torch.empty(nkv, dtype=torch.uint8, device=dev)
+    vt = torch.empty(nkv, dtype=torch.uint8, device=dev)
+    bt = torch.empty(nkb, dtype=torch.uint8, device=dev)
+    _lib.check("msa_encode_bank", lib.msa_encode_bank(
+        ctypes.byref(p), _ptr(k_bank), _ptr(v_bank), _ptr(kbar_hi), _ptr(kbar_lo), _ptr(kt),
+        _ptr(vt), _ptr(bt), _stream(dev)))
+    return kt, vt, bt
+
+
+def decode_fwd_tiled(q, kbar_tiles, k_tiles, v_tiles, seq: int, hkv: int, block: int, topk: int,
+                     scale=None, want_lse=True, ws=None, out=None):
+    """decode_fwd over an encoded bank of `seq` tokens (images from encode_bank)."""
+    nq, hq, d = q.shape
+    p = _bank_params(q, seq, hkv, block, topk, scale)
+    if out is not None:
+        o, lse, idx = out
+    else:
+        o = torch.empty_like(q)
+        lse = torch.empty(nq, hq, dtype=torch.float32, device=q.device) if want_lse else None
+        idx = torch.empty(nq, hkv, topk, dtype=torch.int32, device=q.device)
+    if ws is None:
+        ws = workspace(p, OP_DECODE, nq, device=q.device)
+    _lib.check("msa_decode_fwd_tiled", _lib.load().msa_decode_fwd_tiled(
+        ctypes.byref(p), nq, _ptr(q), _ptr(kbar_tiles), _ptr(k_tiles), _ptr(v_tiles), _ptr(idx),
+        _ptr(o), _ptr(lse), _ptr(ws), ws.numel(), _stream(q.device)))
     return o, lse, idx
 
 

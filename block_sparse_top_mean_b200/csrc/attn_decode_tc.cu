@@ -4,18 +4,19 @@
 // Decode is HBM-bound: every selected K/V byte is read once per (query, group) and the
 // arithmetic is ~2 FLOP per byte.  The kernel is shaped around the stream:
 //   - persistent CTAs (one per SM) take work units round-robin; a unit is one
-//     (query, group) and 4 consecutive selection slots (a split);
+//     (query, group) and 8 consecutive selection slots (a split);
 //   - a producer warp walks the same unit/slot sequence as the consumers and TMA-loads
-//     each selected 64-key tile of K and V (128-byte swizzle, 2 x 8 KB each) into a
-//     5-stage ring; the first tile of a unit also carries the group's G query rows
-//     (one bulk copy);
+//     each selected 64-key tile of K and V (128-byte swizzle, 2 x 8 KB each; with an
+//     encoded bank, one 16 KB bulk copy each, see bank_tiles.cu) into a
+//     6-stage ring; the first tile of a unit also carries the group's G query rows
+//     (one bulk copy); both roles load a unit's selection entries one unit ahead;
 //   - four consumer warps split each tile's 64 keys (16 each) and run the contractions
 //     on mma.sync m16n8k16 (bf16 in, fp32 accumulate) with the G heads as the M rows
 //     (padded to 16): S = Q K^T from ldmatrix'ed K, an online softmax in base 2 per
 //     head, P (bf16) reused in registers as the A operand of O += P V with ldmatrix.trans'ed V;
-//   - at the end of a unit the four warps' (max, sum, O) are merged through shared
-//     memory into one normalised partial and its log-sum-exp; combine_splits_kernel
-//     merges the splits of a (query, group).
+//   - at the end of a unit each warp writes its own normalised partial and log-sum-exp
+//     (no cross-warp merge, no barrier); combine_splits_kernel merges the 4 x nsplit
+//     partials of a (query, group).
 #include <cudaTypedefs.h>
 #include <math_constants.h>
 
@@ -29,10 +30,10 @@ using namespace sm100;
 
 constexpr int kD = 128;
 constexpr int kTileKeys = 64;               // keys per stage (one TMA box of rows)
-constexpr int kStages = 5;
+constexpr int kStages = 6;
 constexpr int kConsumers = 4;               // warps 0-3
 constexpr int kThreads = 32 * kConsumers + 32;   // + producer warp 4
-constexpr int kSlotsPerUnit = 4;            // selection slots per work unit (a split)
+constexpr int kSlotsPerUnit = 8;            // selection slots per work unit (a split)
 constexpr uint32_t kHalfBytes = kTileKeys * 128;        // 64 keys x 64 dims (bf16)
 constexpr uint32_t kKVBytes = 4 * kHalfBytes;           // K halves, V halves (32 KB)
 constexpr uint32_t kQBytesMax = 8 * kD * 2;             // up to 8 heads of one group
@@ -48,6 +49,7 @@ struct __align__(8) ABars {
 
 struct DecAttnGeom {
   int64_t S, nb, block, n_rows;   // bank tokens, bank blocks, block size, n_query * hkv
+  int64_t ntiles;                 // 64-key tiles per head of an encoded bank
   int hq, hkv, topk, nsplit, tiles_per_block;
   float scale_log2;
 };
@@ -73,13 +75,35 @@ __device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
-                                          uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
-          "r"(smem_u32(dst)),
-      "l"(src), "r"(bytes), "r"(smem_u32(bar))
-      : "memory");
+
+// The kSlotsPerUnit selection entries of unit u (-1 beyond topk), one vector load when
+// the row is 16-byte aligned.
+struct Slots {
+  int4 a, b;
+};
+__device__ __forceinline__ int4 load4(const int32_t* p, int s0, int topk) {
+  if ((topk & 3) == 0 && s0 + 4 <= topk) return __ldg(reinterpret_cast<const int4*>(p));
+  int4 r;
+  r.x = s0 + 0 < topk ? __ldg(p + 0) : -1;
+  r.y = s0 + 1 < topk ? __ldg(p + 1) : -1;
+  r.z = s0 + 2 < topk ? __ldg(p + 2) : -1;
+  r.w = s0 + 3 < topk ? __ldg(p + 3) : -1;
+  return r;
+}
+__device__ __forceinline__ Slots unit_slots(const int32_t* __restrict__ idx, int64_t u,
+                                            const DecAttnGeom& g) {
+  const int64_t row = u / g.nsplit;
+  const int s0 = (int)(u % g.nsplit) * kSlotsPerUnit;
+  const int32_t* p = idx + row * g.topk + s0;
+  Slots r;
+  r.a = load4(p, s0, g.topk);
+  r.b = s0 + 4 < g.topk ? load4(p + 4, s0 + 4, g.topk) : make_int4(-1, -1, -1, -1);
+  return r;
+}
+__device__ __forceinline__ int slot_of(const Slots& v, int i) {
+  const int4& h = i < 4 ? v.a : v.b;
+  const int k = i & 3;
+  return k == 0 ? h.x : k == 1 ? h.y : k == 2 ? h.z : h.w;
 }
 
 // Byte offset of 16-byte chunk c (0..15, 8 dims each) of key row r inside a K or V tile.
@@ -93,15 +117,14 @@ __device__ __forceinline__ uint32_t tile_off(int r, int c) {
 template <int G>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                      const unsigned char* __restrict__ ktiles,
+                      const unsigned char* __restrict__ vtiles,
                       const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ idx,
                       float* __restrict__ po, float* __restrict__ plse, int* err, DecAttnGeom g) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* base = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float* red = reinterpret_cast<float*>(base + kStages * kStageStride);   // [4][G][kD] + m, l
-  float* red_m = red + kConsumers * G * kD;
-  float* red_l = red_m + kConsumers * G;
-  ABars* bars = reinterpret_cast<ABars*>(red_l + kConsumers * G);
+  ABars* bars = reinterpret_cast<ABars*>(base + kStages * kStageStride);
 
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   if (tid == 0) {
@@ -120,19 +143,23 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
   if (warp == kConsumers) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      prefetch_tmap(&tmK);
-      prefetch_tmap(&tmV);
+      const bool tiled = ktiles != nullptr;
+      if (!tiled) {
+        prefetch_tmap(&tmK);
+        prefetch_tmap(&tmV);
+      }
       int64_t step = 0;
+      Slots nxt{};
+      if (blockIdx.x < n_units) nxt = unit_slots(idx, blockIdx.x, g);
       for (int64_t u = blockIdx.x; u < n_units && !*abort_flag; u += gridDim.x) {
+        const Slots cur = nxt;                          // the next unit's slots load meanwhile
+        if (u + gridDim.x < n_units) nxt = unit_slots(idx, u + gridDim.x, g);
         const int64_t row = u / g.nsplit;
-        const int split = (int)(u % g.nsplit);
         const int64_t n = row / g.hkv;
         const int gg = (int)(row % g.hkv);
-        const int s0 = split * kSlotsPerUnit;
-        const int s1 = min(g.topk, s0 + kSlotsPerUnit);
         bool first = true;
-        for (int sl = s0; sl < s1 && !*abort_flag; ++sl) {
-          const int64_t j = idx[row * g.topk + sl];
+        for (int sl = 0; sl < kSlotsPerUnit && !*abort_flag; ++sl) {
+          const int64_t j = slot_of(cur, sl);
           if (j == -1) continue;
           if (j < -1 || j >= g.nb) { set_device_error(err, MSA_DEVERR_IDX_RANGE); continue; }
           for (int t = 0; t < g.tiles_per_block; ++t, ++step) {
@@ -147,10 +174,17 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
             unsigned char* dst = base + st * kStageStride;
             const uint32_t qb = first ? (uint32_t)(G * kD * 2) : 0u;
             mbar_arrive_expect_tx(&bars->full[st], kKVBytes + qb);
-            for (int hf = 0; hf < 2; ++hf) {
-              const int x = gg * kD + hf * 64;
-              tma_load_2d(dst + hf * kHalfBytes, &tmK, &bars->full[st], x, (int)key0);
-              tma_load_2d(dst + (2 + hf) * kHalfBytes, &tmV, &bars->full[st], x, (int)key0);
+            if (tiled) {
+              // encoded bank: the (group, 64-key tile) is one contiguous 16 KB image
+              const size_t off = ((size_t)gg * g.ntiles + (size_t)(key0 / kTileKeys)) * 2 * kHalfBytes;
+              bulk_load(dst, ktiles + off, 2 * kHalfBytes, &bars->full[st]);
+              bulk_load(dst + 2 * kHalfBytes, vtiles + off, 2 * kHalfBytes, &bars->full[st]);
+            } else {
+              for (int hf = 0; hf < 2; ++hf) {
+                const int x = gg * kD + hf * 64;
+                tma_load_2d(dst + hf * kHalfBytes, &tmK, &bars->full[st], x, (int)key0);
+                tma_load_2d(dst + (2 + hf) * kHalfBytes, &tmV, &bars->full[st], x, (int)key0);
+              }
             }
             if (first) bulk_load(dst + kKVBytes, q + (n * g.hq + (int64_t)gg * G) * kD, qb,
                                  &bars->full[st]);
@@ -167,11 +201,13 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
   const float c2 = g.scale_log2;
   int64_t step = 0;
   bool aborted = false;
+  Slots nxt{};
+  if (blockIdx.x < n_units) nxt = unit_slots(idx, blockIdx.x, g);
   for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x) {
+    const Slots cur = nxt;
+    if (u + gridDim.x < n_units) nxt = unit_slots(idx, u + gridDim.x, g);
     const int64_t row = u / g.nsplit;
     const int split = (int)(u % g.nsplit);
-    const int s0 = split * kSlotsPerUnit;
-    const int s1 = min(g.topk, s0 + kSlotsPerUnit);
     float m_run = -CUDART_INF_F, l_run = 0.f;       // head gr (valid when gr < G)
     float o[16][4];
 #pragma unroll
@@ -180,8 +216,8 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
       for (int e = 0; e < 4; ++e) o[dt][e] = 0.f;
     uint32_t qa[8][2];                              // A fragments of Q (rows gr; +8 rows are 0)
     bool first = true;
-    for (int sl = s0; sl < s1; ++sl) {
-      const int64_t j = idx[row * g.topk + sl];
+    for (int sl = 0; sl < kSlotsPerUnit; ++sl) {
+      const int64_t j = slot_of(cur, sl);
       if (j < 0 || j >= g.nb) continue;
       for (int t = 0; t < g.tiles_per_block; ++t, ++step) {
         const int64_t key0 = j * g.block + (int64_t)t * kTileKeys;
@@ -262,65 +298,39 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
         if (lane == 0) mbar_arrive(&bars->empty[st]);
       }
     }
-    // merge the four warps' partials of this unit into one normalised partial
+    // this warp's partial over its 16-key slices of the unit's tiles, normalised, with its
+    // log-sum-exp: one split of the (query, group) for combine_splits_kernel
     float lsum = l_run;
     lsum += __shfl_xor_sync(0xffffffffu, lsum, 1);
     lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
     if (gr < G) {
-      if (t4 == 0) {
-        red_m[warp * G + gr] = m_run;
-        red_l[warp * G + gr] = lsum;
-      }
+      const int64_t pi = ((row * g.nsplit + split) * kConsumers + warp) * G + gr;
+      const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+      float* dst = po + pi * kD + 2 * t4;
 #pragma unroll
-      for (int dt = 0; dt < 16; ++dt) {
-        red[(warp * G + gr) * kD + dt * 8 + 2 * t4] = o[dt][0];
-        red[(warp * G + gr) * kD + dt * 8 + 2 * t4 + 1] = o[dt][1];
-      }
+      for (int dt = 0; dt < 16; ++dt)
+        *reinterpret_cast<float2*>(dst + dt * 8) = make_float2(o[dt][0] * inv, o[dt][1] * inv);
+      if (t4 == 0) plse[pi] = lsum > 0.f ? (m_run + log2f(lsum)) * kLn2 : -CUDART_INF_F;
     }
-    asm volatile("bar.sync 1, %0;" ::"n"(32 * kConsumers) : "memory");
-    {
-      const int d = tid;                               // 128 consumer threads = 128 dims
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        float M = -CUDART_INF_F;
-#pragma unroll
-        for (int w = 0; w < kConsumers; ++w) M = fmaxf(M, red_m[w * G + h]);
-        float L = 0.f, acc = 0.f;
-        if (M != -CUDART_INF_F) {
-#pragma unroll
-          for (int w = 0; w < kConsumers; ++w) {
-            const float wt = exp2f(red_m[w * G + h] - M);
-            L += wt * red_l[w * G + h];
-            acc += wt * red[(w * G + h) * kD + d];
-          }
-        }
-        const int64_t pi = (row * g.nsplit + split) * G + h;
-        po[pi * kD + d] = L > 0.f ? acc / L : 0.f;
-        if (d == 0) plse[pi] = L > 0.f ? (M + log2f(L)) * kLn2 : -CUDART_INF_F;
-      }
-    }
-    asm volatile("bar.sync 1, %0;" ::"n"(32 * kConsumers) : "memory");
   }
 }
 
-size_t smem_bytes(int G) {
-  return 1024 + (size_t)kStages * kStageStride + (size_t)kConsumers * G * (kD + 2) * 4 +
-         sizeof(ABars);
-}
+size_t smem_bytes() { return 1024 + (size_t)kStages * kStageStride + sizeof(ABars); }
 
 template <int G>
 cudaError_t run_dec_attn(const DecAttnGeom& g, const CUtensorMap& mk, const CUtensorMap& mv,
-                         const void* q, const int32_t* idx, float* po, float* plse, int* err,
-                         cudaStream_t st) {
-  const size_t smem = smem_bytes(G);
+                         const void* kt, const void* vt, const void* q, const int32_t* idx,
+                         float* po, float* plse, int* err, cudaStream_t st) {
+  const size_t smem = smem_bytes();
   cudaError_t e = cudaFuncSetAttribute(attn_decode_tc_kernel<G>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int64_t units = g.n_rows * g.nsplit;
   int grid = sm_count();
   if (units < grid) grid = (int)units;
-  attn_decode_tc_kernel<G><<<grid, kThreads, smem, st>>>(mk, mv, (const __nv_bfloat16*)q, idx, po,
-                                                         plse, err, g);
+  attn_decode_tc_kernel<G><<<grid, kThreads, smem, st>>>(
+      mk, mv, (const unsigned char*)kt, (const unsigned char*)vt, (const __nv_bfloat16*)q, idx,
+      po, plse, err, g);
   return cudaGetLastError();
 }
 
@@ -338,25 +348,28 @@ bool tc_decode_attn_supported(const Shape& s) {
 int decode_attn_tc_nsplit(const Shape& s) {
   return (int)((s.topk + kSlotsPerUnit - 1) / kSlotsPerUnit);
 }
+int decode_attn_tc_partials(const Shape& s) { return decode_attn_tc_nsplit(s) * kConsumers; }
 
 cudaError_t launch_attn_decode_tc(const Shape& s, int64_t n_query, const void* q, const void* k,
-                                  const void* v, const int32_t* idx, float* po, float* plse,
-                                  int* err, cudaStream_t st) {
-  CUtensorMap mk, mv;
-  if (!make_bf16_2d_map(&mk, k, s.seq, s.hkv * kD, kTileKeys) ||
-      !make_bf16_2d_map(&mv, v, s.seq, s.hkv * kD, kTileKeys))
+                                  const void* v, const void* k_tiles, const void* v_tiles,
+                                  const int32_t* idx, float* po, float* plse, int* err,
+                                  cudaStream_t st) {
+  CUtensorMap mk{}, mv{};
+  if (k_tiles == nullptr && (!make_bf16_2d_map(&mk, k, s.seq, s.hkv * kD, kTileKeys) ||
+                             !make_bf16_2d_map(&mv, v, s.seq, s.hkv * kD, kTileKeys)))
     return cudaErrorInvalidValue;
   DecAttnGeom g{};
+  g.ntiles = (s.seq + kTileKeys - 1) / kTileKeys;
   g.S = s.seq; g.nb = s.nb; g.block = s.block; g.n_rows = n_query * s.hkv;
   g.hq = (int)s.hq; g.hkv = (int)s.hkv; g.topk = (int)s.topk;
   g.nsplit = decode_attn_tc_nsplit(s);
   g.tiles_per_block = (int)(s.block / kTileKeys);
   g.scale_log2 = s.scale * kLog2e;
   switch (s.hq / s.hkv) {
-    case 1: return run_dec_attn<1>(g, mk, mv, q, idx, po, plse, err, st);
-    case 2: return run_dec_attn<2>(g, mk, mv, q, idx, po, plse, err, st);
-    case 4: return run_dec_attn<4>(g, mk, mv, q, idx, po, plse, err, st);
-    default: return run_dec_attn<8>(g, mk, mv, q, idx, po, plse, err, st);
+    case 1: return run_dec_attn<1>(g, mk, mv, k_tiles, v_tiles, q, idx, po, plse, err, st);
+    case 2: return run_dec_attn<2>(g, mk, mv, k_tiles, v_tiles, q, idx, po, plse, err, st);
+    case 4: return run_dec_attn<4>(g, mk, mv, k_tiles, v_tiles, q, idx, po, plse, err, st);
+    default: return run_dec_attn<8>(g, mk, mv, k_tiles, v_tiles, q, idx, po, plse, err, st);
   }
 }
 

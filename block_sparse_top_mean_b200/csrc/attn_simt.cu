@@ -250,27 +250,37 @@ cudaError_t launch_attn_prefill_rows(const Shape& s, const void* q, const void* 
   return dispatch(s, a, st);
 }
 
+// Partials per (query, group): the SIMT rows write one per split, the streamed kernel one
+// per split and consumer warp.
+int decode_partials(const Shape& s) {
+  return tc_decode_attn_supported(s) ? decode_attn_tc_partials(s) : decode_nsplit_attn(s);
+}
+
 size_t decode_attn_ws_bytes(const Shape& s, int64_t n_query) {
   const int G = (int)(s.hq / s.hkv);
-  const size_t np = (size_t)n_query * s.hkv * decode_nsplit_attn(s) * G;
+  const size_t np = (size_t)n_query * s.hkv * decode_partials(s) * G;
   return ((np * s.d * sizeof(float) + 255) / 256) * 256 + np * sizeof(float) + 256;
 }
 
 cudaError_t launch_attn_decode(const Shape& s, int64_t n_query, const void* q, const void* k,
-                               const void* v, const int32_t* idx, void* o, float* lse, void* ws,
-                               int* err, cudaStream_t st) {
+                               const void* v, const void* k_tiles, const void* v_tiles,
+                               const int32_t* idx, void* o, float* lse, void* ws, int* err,
+                               cudaStream_t st) {
   RowsArgs a = base_args(s);
   const int G = (int)(s.hq / s.hkv);
   a.q = q; a.k = k; a.v = v; a.idx = idx; a.err = err;
   a.n_rows = n_query * s.hkv;
   a.nsplit = decode_nsplit_attn(s); a.slots_per_split = kDecodeSplitSlots; a.causal = 0;
-  const size_t np = (size_t)a.n_rows * a.nsplit * G;
+  const bool tc = tc_decode_attn_supported(s);
+  const int nparts = tc ? decode_attn_tc_partials(s) : a.nsplit;
+  const size_t np = (size_t)a.n_rows * nparts * G;
   a.po = reinterpret_cast<float*>(ws);
   a.plse = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) +
                                     ((np * s.d * sizeof(float) + 255) / 256) * 256);
-  const bool tc = tc_decode_attn_supported(s) && decode_attn_tc_nsplit(s) == a.nsplit;
+  if (k_tiles != nullptr && !tc) return cudaErrorInvalidValue;   // encoded banks: tc only
   if (a.nsplit == 1 && !tc) { a.o = o; a.lse = lse; }
-  cudaError_t e = tc ? launch_attn_decode_tc(s, n_query, q, k, v, idx, a.po, a.plse, err, st)
+  cudaError_t e = tc ? launch_attn_decode_tc(s, n_query, q, k, v, k_tiles, v_tiles, idx, a.po,
+                                             a.plse, err, st)
                      : dispatch(s, a, st);
   if (e != cudaSuccess || (a.nsplit == 1 && !tc)) return e;
   const int64_t tasks = a.n_rows * G;
@@ -278,17 +288,17 @@ cudaError_t launch_attn_decode(const Shape& s, int64_t n_query, const void* q, c
   if (s.dtype == MSA_BF16) {
     if (s.d == 128)
       combine_splits_kernel<__nv_bfloat16, 128><<<grid, 128, 0, st>>>(
-          a.po, a.plse, (__nv_bfloat16*)o, lse, a.n_rows, G, a.nsplit, (int)s.hkv, (int)s.hq);
+          a.po, a.plse, (__nv_bfloat16*)o, lse, a.n_rows, G, nparts, (int)s.hkv, (int)s.hq);
     else
       combine_splits_kernel<__nv_bfloat16, 64><<<grid, 128, 0, st>>>(
-          a.po, a.plse, (__nv_bfloat16*)o, lse, a.n_rows, G, a.nsplit, (int)s.hkv, (int)s.hq);
+          a.po, a.plse, (__nv_bfloat16*)o, lse, a.n_rows, G, nparts, (int)s.hkv, (int)s.hq);
   } else {
     if (s.d == 128)
       combine_splits_kernel<float, 128><<<grid, 128, 0, st>>>(
-          a.po, a.plse, (float*)o, lse, a.n_rows, G, a.nsplit, (int)s.hkv, (int)s.hq);
+          a.po, a.plse, (float*)o, lse, a.n_rows, G, nparts, (int)s.hkv, (int)s.hq);
     else
       combine_splits_kernel<float, 64><<<grid, 128, 0, st>>>(
-          a.po, a.plse, (float*)o, lse, a.n_rows, G, a.nsplit, (int)s.hkv, (int)s.hq);
+          a.po, a.plse, (float*)o, lse, a.n_rows, G, nparts, (int)s.hkv, (int)s.hq);
   }
   return cudaGetLastError();
 }

@@ -109,17 +109,29 @@ cudaError_t launch_topk_decode(const Shape& s, int64_t n_query, const void* q, c
 bool tc_decode_supported(const Shape& s);
 size_t topk_decode_tc_ws_bytes(const Shape& s, int64_t n_query);
 cudaError_t launch_topk_decode_tc(const Shape& s, int64_t n_query, const void* q,
-                                  const void* kbar_hi, const void* kbar_lo, int32_t* idx,
-                                  void* ws, int* err, cudaStream_t st);
+                                  const void* kbar_hi, const void* kbar_lo,
+                                  const void* kbar_tiles, int32_t* idx, void* ws, int* err,
+                                  cudaStream_t st);
 
 // Decode attention streamed through shared memory on mma.sync (bf16, d = 128,
 // block % 64 == 0); see attn_decode_tc.cu.  Writes per-split partials (normalised O and
 // lse, the same layout as the SIMT decode rows) for combine_splits_kernel.
 bool tc_decode_attn_supported(const Shape& s);
 int decode_attn_tc_nsplit(const Shape& s);
+int decode_attn_tc_partials(const Shape& s);   // partials per (query, group)
 cudaError_t launch_attn_decode_tc(const Shape& s, int64_t n_query, const void* q, const void* k,
-                                  const void* v, const int32_t* idx, float* po, float* plse,
-                                  int* err, cudaStream_t st);
+                                  const void* v, const void* k_tiles, const void* v_tiles,
+                                  const int32_t* idx, float* po, float* plse, int* err,
+                                  cudaStream_t st);
+
+// Encoded decode banks (bank_tiles.cu): K/V as per-head 64-key 16 KB tile images and
+// pooled-key hi/lo planes as per-head 128-block 32 KB chunk images, both in the
+// 128-byte-swizzled shared-memory layout the decode kernels consume.
+size_t bank_kv_tiles_bytes(const Shape& s);
+size_t bank_kbar_tiles_bytes(const Shape& s);
+cudaError_t launch_encode_bank(const Shape& s, const void* k, const void* v, const void* kbar_hi,
+                               const void* kbar_lo, void* k_tiles, void* v_tiles,
+                               void* kbar_tiles, cudaStream_t st);
 
 // Query-centric attention over selected blocks (SIMT, fp32 math).
 size_t decode_attn_ws_bytes(const Shape& s, int64_t n_query);
@@ -127,8 +139,9 @@ cudaError_t launch_attn_prefill_rows(const Shape& s, const void* q, const void* 
                                      const int32_t* idx, void* o, float* lse, int* err,
                                      cudaStream_t st);
 cudaError_t launch_attn_decode(const Shape& s, int64_t n_query, const void* q, const void* k,
-                               const void* v, const int32_t* idx, void* o, float* lse, void* ws,
-                               int* err, cudaStream_t st);
+                               const void* v, const void* k_tiles, const void* v_tiles,
+                               const int32_t* idx, void* o, float* lse, void* ws, int* err,
+                               cudaStream_t st);
 
 // Host helpers (host_util.cu): a 2-D bf16 TMA map over a row-major [rows, cols] tensor
 // with 64-column x box_rows boxes and 128-byte swizzle; the device's SM count.

@@ -250,12 +250,72 @@ msa_status msa_decode_fwd(const msa_params* p, int64_t n_query, const void* q, c
   char* sel_ws = ws_body(ws);
   char* att_ws = sel_ws + round256(decode_sel_ws(s, n_query));
   cudaError_t e =
-      tc ? msa::launch_topk_decode_tc(s, n_query, q, kbar_hi, kbar_lo, idx, sel_ws, err_word(ws),
-                                      cs)
+      tc ? msa::launch_topk_decode_tc(s, n_query, q, kbar_hi, kbar_lo, nullptr, idx, sel_ws,
+                                      err_word(ws), cs)
          : msa::launch_topk_decode(s, n_query, q, kbar, idx, sel_ws, cs);
   if (e == cudaSuccess)
-    e = msa::launch_attn_decode(s, n_query, q, k_bank, v_bank, idx, o, lse, att_ws, err_word(ws),
-                                cs);
+    e = msa::launch_attn_decode(s, n_query, q, k_bank, v_bank, nullptr, nullptr, idx, o, lse,
+                                att_ws, err_word(ws), cs);
+  return cuda_status(e);
+}
+
+size_t msa_bank_tiles_bytes(const msa_params* p, int32_t which) {
+  Shape s;
+  if (check_params(p, true, &s) != MSA_OK) return 0;
+  if (which == 0) return msa::bank_kv_tiles_bytes(s);
+  if (which == 1) return msa::bank_kbar_tiles_bytes(s);
+  return 0;
+}
+
+// Encoded banks need the tensor-core decode path on both steps.
+static bool tiled_decode_supported(const Shape& s) {
+  return msa::tc_decode_supported(s) && msa::tc_decode_attn_supported(s);
+}
+
+msa_status msa_encode_bank(const msa_params* p, const void* k_bank, const void* v_bank,
+                           const void* kbar_hi, const void* kbar_lo, void* k_tiles,
+                           void* v_tiles, void* kbar_tiles, msa_stream_t stream) {
+  Shape s;
+  msa_status st = check_params(p, true, &s);
+  if (st != MSA_OK) return st;
+  if (s.seq == 0) return MSA_OK;
+  if (!tiled_decode_supported(s)) return MSA_ERR_UNSUPPORTED;
+  if ((k_tiles != nullptr && k_bank == nullptr) || (v_tiles != nullptr && v_bank == nullptr) ||
+      (kbar_tiles != nullptr && (kbar_hi == nullptr || kbar_lo == nullptr)))
+    return MSA_ERR_INVALID_ARG;
+  if (!aligned16(k_bank) || !aligned16(v_bank) || !aligned16(kbar_hi) || !aligned16(kbar_lo) ||
+      !aligned16(k_tiles) || !aligned16(v_tiles) || !aligned16(kbar_tiles))
+    return MSA_ERR_INVALID_ARG;
+  return cuda_status(msa::launch_encode_bank(s, k_bank, v_bank, kbar_hi, kbar_lo, k_tiles,
+                                             v_tiles, kbar_tiles, (cudaStream_t)stream));
+}
+
+msa_status msa_decode_fwd_tiled(const msa_params* p, int64_t n_query, const void* q,
+                                const void* kbar_tiles, const void* k_tiles,
+                                const void* v_tiles, int32_t* idx, void* o, float* lse,
+                                void* ws, size_t ws_bytes, msa_stream_t stream) {
+  Shape s;
+  msa_status st = check_params(p, true, &s);
+  if (st != MSA_OK) return st;
+  if (n_query < 0) return MSA_ERR_INVALID_ARG;
+  if (n_query == 0 || s.seq == 0) return MSA_OK;
+  if (n_query > 65535 * 64) return MSA_ERR_UNSUPPORTED;
+  if (!tiled_decode_supported(s)) return MSA_ERR_UNSUPPORTED;
+  if (q == nullptr || kbar_tiles == nullptr || k_tiles == nullptr || v_tiles == nullptr ||
+      idx == nullptr || o == nullptr)
+    return MSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(kbar_tiles) || !aligned16(k_tiles) || !aligned16(v_tiles) ||
+      !aligned16(o))
+    return MSA_ERR_INVALID_ARG;
+  if ((st = check_ws(s, MSA_OP_DECODE, n_query, ws, ws_bytes)) != MSA_OK) return st;
+  cudaStream_t cs = (cudaStream_t)stream;
+  char* sel_ws = ws_body(ws);
+  char* att_ws = sel_ws + round256(decode_sel_ws(s, n_query));
+  cudaError_t e = msa::launch_topk_decode_tc(s, n_query, q, nullptr, nullptr, kbar_tiles, idx,
+                                             sel_ws, err_word(ws), cs);
+  if (e == cudaSuccess)
+    e = msa::launch_attn_decode(s, n_query, q, nullptr, nullptr, k_tiles, v_tiles, idx, o, lse,
+                                att_ws, err_word(ws), cs);
   return cuda_status(e);
 }
 

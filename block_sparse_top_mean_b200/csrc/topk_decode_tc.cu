@@ -70,6 +70,7 @@ struct DecGeom {
   int64_t stride;    // chunk index of unit c is c * stride (1, or the sample stride)
   int64_t per;       // units (group, chunk) per CTA along x
   int64_t nq_pad;    // query tiles * kN
+  int64_t nch_full;  // 128-block chunks per group of the whole bank (encoded-plane stride)
   int hq, hkv, G, topk, ns_max, ncta_x;
 };
 
@@ -172,6 +173,7 @@ template <int G, bool GMAX>
 __global__ void __launch_bounds__(kThreads, 1)
 topk_decode_tc_kernel(const __grid_constant__ CUtensorMap tmHi,
                       const __grid_constant__ CUtensorMap tmLo,
+                      const unsigned char* __restrict__ ktiles,
                       const __nv_bfloat16* __restrict__ q, const float* __restrict__ tinit,
                       uint64_t* __restrict__ cand, uint32_t* __restrict__ gmax, int* err,
                       DecGeom g) {
@@ -219,12 +221,16 @@ topk_decode_tc_kernel(const __grid_constant__ CUtensorMap tmHi,
   if (warp == kEpiWarps) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      prefetch_tmap(&tmHi);
-      prefetch_tmap(&tmLo);
+      const bool tiled = ktiles != nullptr;
+      if (!tiled) {
+        prefetch_tmap(&tmHi);
+        prefetch_tmap(&tmLo);
+      }
       int64_t step = 0;
       for (int64_t u = u0; u < u1 && !*abort_flag; ++u) {
         const int gg = (int)(u / g.nch);
-        const int y = (int)((u % g.nch) * g.stride * kM);
+        const int64_t chunk = (u % g.nch) * g.stride;
+        const int y = (int)(chunk * kM);
         for (int hf = 0; hf < 2; ++hf, ++step) {
           const int st = (int)(step % kStages);
           if (step >= kStages &&
@@ -234,9 +240,17 @@ topk_decode_tc_kernel(const __grid_constant__ CUtensorMap tmHi,
           }
           unsigned char* dst = KS + st * kStageBytes;
           mbar_arrive_expect_tx(&bars->full[st], kStageBytes);
-          const int x = gg * kD + hf * 64;
-          tma_load_2d(dst, &tmHi, &bars->full[st], x, y);
-          tma_load_2d(dst + kPlane, &tmLo, &bars->full[st], x, y);
+          if (tiled) {
+            // encoded planes: [plane][group][chunk][half] images of 16 KB each
+            const size_t plane = (size_t)g.hkv * g.nch_full * 2 * kPlane;
+            const size_t off = (((size_t)gg * g.nch_full + chunk) * 2 + hf) * kPlane;
+            bulk_load(dst, ktiles + off, kPlane, &bars->full[st]);
+            bulk_load(dst + kPlane, ktiles + plane + off, kPlane, &bars->full[st]);
+          } else {
+            const int x = gg * kD + hf * 64;
+            tma_load_2d(dst, &tmHi, &bars->full[st], x, y);
+            tma_load_2d(dst + kPlane, &tmLo, &bars->full[st], x, y);
+          }
         }
       }
     }
@@ -504,9 +518,15 @@ __global__ void topk_decode_merge_kernel(const uint64_t* __restrict__ cand,
   int64_t c_last = (((int64_t)gg + 1) * g.nch - 1) / g.per;
   if (c_last > g.ncta_x - 1) c_last = g.ncta_x - 1;
   uint64_t y = 0ull;
-  for (int64_t c = c_first; c <= c_last; ++c) {
-    const int64_t row = ((int64_t)gg * g.ns_max + (c - c_first)) * g.nq_pad + n;
-    y = warp_merge_desc(y, cand[row * kList + lane], lane);
+  const uint64_t* src = cand + ((int64_t)gg * g.ns_max * g.nq_pad + n) * kList + lane;
+  const int64_t step = g.nq_pad * kList;            // next CTA slot of the group
+  const int nl = (int)(c_last - c_first + 1);
+  // the next list loads while the current one merges
+  uint64_t x = nl > 0 ? __ldg(src) : 0ull;
+  for (int c = 0; c < nl; ++c) {
+    const uint64_t xn = c + 1 < nl ? __ldg(src + (c + 1) * step) : 0ull;
+    y = warp_merge_desc(y, x, lane);
+    x = xn;
   }
   // the best topk, ascending by block index (empty entries sort last)
   int j = (lane < g.topk && y != 0ull) ? key_block(y) : 0x7fffffff;
@@ -525,6 +545,8 @@ __global__ void topk_decode_merge_kernel(const uint64_t* __restrict__ cand,
 // One warp per (query, group): T0 = the 32nd largest of the sampled 32-block group maxima
 // (a valid bound: 32 different blocks score at least T0), found bit by bit on the
 // order-preserving bits; -inf when fewer than 32 groups were sampled.
+constexpr int kThrRegs = 24;                    // register path up to 768 group maxima
+
 __global__ void sample_threshold_kernel(const uint32_t* __restrict__ gmax, float* __restrict__ tout,
                                         int64_t rows, int ngroups) {
   const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / 32;
@@ -532,11 +554,27 @@ __global__ void sample_threshold_kernel(const uint32_t* __restrict__ gmax, float
   if (w >= rows) return;
   const uint32_t* vals = gmax + w * ngroups;
   uint32_t prefix = 0u;
-  for (int bit = 31; bit >= 0; --bit) {
-    const uint32_t cand = prefix | (1u << bit);
-    int c = 0;
-    for (int i = lane; i < ngroups; i += 32) c += __ldg(vals + i) >= cand;
-    if (__reduce_add_sync(0xffffffffu, (uint32_t)c) >= 32u) prefix = cand;
+  if (ngroups <= 32 * kThrRegs) {
+    uint32_t r[kThrRegs];                       // this lane's values, loaded once
+#pragma unroll
+    for (int k = 0; k < kThrRegs; ++k) {
+      const int i = lane + 32 * k;
+      r[k] = i < ngroups ? __ldg(vals + i) : 0u;
+    }
+    for (int bit = 31; bit >= 0; --bit) {
+      const uint32_t cand = prefix | (1u << bit);
+      uint32_t c = 0;
+#pragma unroll
+      for (int k = 0; k < kThrRegs; ++k) c += r[k] >= cand;
+      if (__reduce_add_sync(0xffffffffu, c) >= 32u) prefix = cand;
+    }
+  } else {
+    for (int bit = 31; bit >= 0; --bit) {
+      const uint32_t cand = prefix | (1u << bit);
+      uint32_t c = 0;
+      for (int i = lane; i < ngroups; i += 32) c += __ldg(vals + i) >= cand;
+      if (__reduce_add_sync(0xffffffffu, c) >= 32u) prefix = cand;
+    }
   }
   if (lane == 0) tout[w] = ord_score(prefix);
 }
@@ -551,7 +589,8 @@ DecGeom make_dgeom(const Shape& s, int64_t n_query, int64_t stride) {
   g.nb = s.nb;
   g.n_query = n_query;
   g.stride = stride;
-  g.nch = ((s.nb + kM - 1) / kM + stride - 1) / stride;
+  g.nch_full = (s.nb + kM - 1) / kM;
+  g.nch = (g.nch_full + stride - 1) / stride;
   const int64_t qtiles = (n_query + kN - 1) / kN;
   g.nq_pad = qtiles * kN;
   const int sms = sm_count();
@@ -575,15 +614,15 @@ bool use_sample(const Shape& s) { return (s.nb + kM - 1) / kM >= kSampleMinChunk
 
 template <int G, bool GMAX>
 cudaError_t run_scan(const DecGeom& g, const CUtensorMap& mh, const CUtensorMap& ml,
-                     const void* q, const float* tinit, uint64_t* cand, uint32_t* gmax, int* err,
-                     cudaStream_t st) {
+                     const void* kt, const void* q, const float* tinit, uint64_t* cand,
+                     uint32_t* gmax, int* err, cudaStream_t st) {
   const size_t smem = smem_bytes();
   cudaError_t e = cudaFuncSetAttribute(topk_decode_tc_kernel<G, GMAX>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const dim3 grid((unsigned)g.ncta_x, (unsigned)(g.nq_pad / kN));
   topk_decode_tc_kernel<G, GMAX><<<grid, kThreads, smem, st>>>(
-      mh, ml, (const __nv_bfloat16*)q, tinit, cand, gmax, err, g);
+      mh, ml, (const unsigned char*)kt, (const __nv_bfloat16*)q, tinit, cand, gmax, err, g);
   return cudaGetLastError();
 }
 
@@ -628,12 +667,14 @@ size_t topk_decode_tc_ws_bytes(const Shape& s, int64_t n_query) {
 }
 
 cudaError_t launch_topk_decode_tc(const Shape& s, int64_t n_query, const void* q,
-                                  const void* kbar_hi, const void* kbar_lo, int32_t* idx,
-                                  void* ws, int* err, cudaStream_t st) {
-  CUtensorMap mh, ml;
-  if (!make_bf16_2d_map(&mh, kbar_hi, s.nb, s.hkv * kD, kM) ||
-      !make_bf16_2d_map(&ml, kbar_lo, s.nb, s.hkv * kD, kM))
+                                  const void* kbar_hi, const void* kbar_lo,
+                                  const void* kbar_tiles, int32_t* idx, void* ws, int* err,
+                                  cudaStream_t st) {
+  CUtensorMap mh{}, ml{};
+  if (kbar_tiles == nullptr && (!make_bf16_2d_map(&mh, kbar_hi, s.nb, s.hkv * kD, kM) ||
+                                !make_bf16_2d_map(&ml, kbar_lo, s.nb, s.hkv * kD, kM)))
     return cudaErrorInvalidValue;
+  const void* kt = kbar_tiles;
   const DecGeom g = make_dgeom(s, n_query, 1);
   const bool sample = use_sample(s);
   const DecWs L = dec_ws(s, n_query);
@@ -647,10 +688,10 @@ cudaError_t launch_topk_decode_tc(const Shape& s, int64_t n_query, const void* q
     // (query, group) is a valid bound that starts the full scan
     const DecGeom gs = make_dgeom(s, n_query, kSampleStride);
     switch (gs.G) {
-      case 1: e = run_scan<1, true>(gs, mh, ml, q, nullptr, nullptr, gmax, err, st); break;
-      case 2: e = run_scan<2, true>(gs, mh, ml, q, nullptr, nullptr, gmax, err, st); break;
-      case 4: e = run_scan<4, true>(gs, mh, ml, q, nullptr, nullptr, gmax, err, st); break;
-      default: e = run_scan<8, true>(gs, mh, ml, q, nullptr, nullptr, gmax, err, st); break;
+      case 1: e = run_scan<1, true>(gs, mh, ml, kt, q, nullptr, nullptr, gmax, err, st); break;
+      case 2: e = run_scan<2, true>(gs, mh, ml, kt, q, nullptr, nullptr, gmax, err, st); break;
+      case 4: e = run_scan<4, true>(gs, mh, ml, kt, q, nullptr, nullptr, gmax, err, st); break;
+      default: e = run_scan<8, true>(gs, mh, ml, kt, q, nullptr, nullptr, gmax, err, st); break;
     }
     if (e != cudaSuccess) return e;
     const int64_t rows = n_query * s.hkv;
@@ -660,10 +701,10 @@ cudaError_t launch_topk_decode_tc(const Shape& s, int64_t n_query, const void* q
   }
   const float* t0 = sample ? tinit : nullptr;
   switch (g.G) {
-    case 1: e = run_scan<1, false>(g, mh, ml, q, t0, cand, nullptr, err, st); break;
-    case 2: e = run_scan<2, false>(g, mh, ml, q, t0, cand, nullptr, err, st); break;
-    case 4: e = run_scan<4, false>(g, mh, ml, q, t0, cand, nullptr, err, st); break;
-    default: e = run_scan<8, false>(g, mh, ml, q, t0, cand, nullptr, err, st); break;
+    case 1: e = run_scan<1, false>(g, mh, ml, kt, q, t0, cand, nullptr, err, st); break;
+    case 2: e = run_scan<2, false>(g, mh, ml, kt, q, t0, cand, nullptr, err, st); break;
+    case 4: e = run_scan<4, false>(g, mh, ml, kt, q, t0, cand, nullptr, err, st); break;
+    default: e = run_scan<8, false>(g, mh, ml, kt, q, t0, cand, nullptr, err, st); break;
   }
   if (e != cudaSuccess) return e;
   const int64_t warps = n_query * s.hkv;

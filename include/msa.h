@@ -173,6 +173,36 @@ MSA_API msa_status msa_decode_fwd(const msa_params* p, int64_t n_query, const vo
                                   const void* k_bank, const void* v_bank, int32_t* idx, void* o,
                                   float* lse, void* ws, size_t ws_bytes, msa_stream_t stream);
 
+/* Encoded decode bank ([MSA-DE]: the bank and its routing keys are prepared offline, when
+ * the bank is written).  Same method and results as msa_decode_fwd; only the memory
+ * layout of the bank differs, chosen so that each selected tile is one contiguous run:
+ *   k_tiles, v_tiles  [hkv][ceil(S/64)][2][64][64] bf16: per KV head, 64-key tiles, each
+ *                     as two 64-dim halves of 64 rows x 128 bytes; inside a half, the
+ *                     16-byte chunk c of row r is stored at chunk position c ^ (r % 8);
+ *                     rows past S are zero.  msa_bank_tiles_bytes(p, 0) bytes each.
+ *   kbar_tiles        [2][hkv][ceil(nb/128)][2][128][64] bf16: the hi planes, then the lo
+ *                     planes of the pooled keys, per KV head in 128-block chunks, the
+ *                     same half/row/chunk order and swizzle; rows past nb are zero.
+ *                     msa_bank_tiles_bytes(p, 1) bytes.
+ * Supported: bf16, d = 128, block a multiple of 64, G in {1, 2, 4, 8} (else
+ * MSA_ERR_UNSUPPORTED).  msa_bank_tiles_bytes returns 0 for invalid shapes or `which`. */
+MSA_API size_t msa_bank_tiles_bytes(const msa_params* p, int32_t which);
+
+/* Writes the encoded images of a bank in the natural layout (k_bank, v_bank [S, hkv, d];
+ * kbar_hi, kbar_lo [nb, hkv, d] from msa_pool_keys).  Any of k_tiles, v_tiles,
+ * kbar_tiles may be NULL (that image is skipped); the matching inputs are then unused. */
+MSA_API msa_status msa_encode_bank(const msa_params* p, const void* k_bank, const void* v_bank,
+                                   const void* kbar_hi, const void* kbar_lo, void* k_tiles,
+                                   void* v_tiles, void* kbar_tiles, msa_stream_t stream);
+
+/* msa_decode_fwd over an encoded bank: the same selection (tensor-core scan of the
+ * pooled-key planes) and the same attention, fed by 1-D bulk copies.
+ * ws: msa_workspace_bytes(p, MSA_OP_DECODE, n_query). */
+MSA_API msa_status msa_decode_fwd_tiled(const msa_params* p, int64_t n_query, const void* q,
+                                        const void* kbar_tiles, const void* k_tiles,
+                                        const void* v_tiles, int32_t* idx, void* o, float* lse,
+                                        void* ws, size_t ws_bytes, msa_stream_t stream);
+
 /* Bytes of the fixed device scratch used by msa_decode_fwd_static (32 MiB). */
 #define MSA_DECODE_STATIC_SCRATCH_BYTES ((size_t)32 << 20)
 
@@ -186,7 +216,7 @@ MSA_API msa_status msa_decode_fwd(const msa_params* p, int64_t n_query, const vo
  *     nothing (no cudaMalloc/cudaFree, no allocating library routine).
  *   - Limit: returns MSA_ERR_WORKSPACE, launching nothing, when
  *     msa_workspace_bytes(p, MSA_OP_DECODE, n_query) exceeds that size (64 queries x 32
- *     heads against a 10M-token bank need about 14 MB).
+ *     heads against a 10M-token bank need about 21 MB).
  *   - Set-up: the first call on a device looks up the array's device address with that
  *     device current (cudaGetSymbolAddress) and caches it; make that first call before
  *     any stream capture.

@@ -249,6 +249,48 @@ def test_decode_tc_scan(msa, w):
     check_decode(q, kbar_np, kb, vb, w.block, w.topk, w.scale, idx, o, lse, queries=qs)
 
 
+@pytest.mark.parametrize("w", [DECODE_TC[0], DECODE_TC[2], DECODE_TC[3], DECODE_TC[6]],
+                         ids=lambda w: w.name)
+def test_decode_tiled_bank_matches_natural_layout(msa, w):
+    # the encoded bank changes only where the bytes live: selection and outputs are
+    # bitwise those of the natural layout, which the oracle checks
+    q, kb, vb = mi.decode_inputs(w, device="cuda")
+    _, khi, klo = (t[0] for t in msa.pool_keys(kb[None], w.block, split=True))
+    o, lse, idx = msa.decode_fwd(q, None, kb, vb, w.block, w.topk, w.scale, kbar_hi=khi,
+                                 kbar_lo=klo)
+    kt, vt, bt = msa.encode_bank(kb, vb, khi, klo, w.block)
+    o2, lse2, idx2 = msa.decode_fwd_tiled(q, bt, kt, vt, w.seq, w.hkv, w.block, w.topk, w.scale)
+    torch.cuda.synchronize()
+    assert torch.equal(idx, idx2)
+    assert torch.equal(o, o2)
+    assert torch.equal(lse, lse2)
+    if w.name == "dtc_sampled_2p5m":
+        kbar_np = pool_keys_chunked(kb[None], w.block)[0]
+        check_decode(q, kbar_np, kb, vb, w.block, w.topk, w.scale, idx2, o2, lse2,
+                     queries=list(range(0, w.n_query, 5)))
+
+
+def test_encode_bank_layout(msa):
+    # spot-check the documented image layout against the natural tensors
+    w = mi.Workload("enc", "decode", 1, 1000, 8, 2, 128, 64, 8, "bf16", n_query=1)
+    _, kb, vb = mi.decode_inputs(w, device="cuda")
+    _, khi, klo = (t[0] for t in msa.pool_keys(kb[None], w.block, split=True))
+    kt, vt, bt = msa.encode_bank(kb, vb, khi, klo, w.block)
+    ntile = -(-w.seq // 64)
+    img = kt.view(torch.bfloat16).view(w.hkv, ntile, 2, 64, 8, 8)   # [g][t][half][row][chunk][8]
+    for g, tok, dim in [(0, 0, 0), (1, 5, 77), (0, 999, 127), (1, 640, 8)]:
+        t, r = divmod(tok, 64)
+        h, c, e = dim // 64, (dim % 64) // 8, dim % 8
+        assert img[g, t, h, r, c ^ (r % 8), e].item() == kb[tok, g, dim].item()
+    assert int(img[0, ntile - 1, 0, (w.seq % 64):].abs().sum().float().item()) == 0   # rows past S
+    nch = -(-w.nb // 128)
+    bimg = bt.view(torch.bfloat16).view(2, w.hkv, nch, 2, 128, 8, 8)
+    for g, j, dim in [(0, 0, 0), (1, 15, 100)]:
+        h, c, e, r = dim // 64, (dim % 64) // 8, dim % 8, j % 128
+        assert bimg[0, g, j // 128, h, r, c ^ (r % 8), e].item() == khi[j, g, dim].item()
+        assert bimg[1, g, j // 128, h, r, c ^ (r % 8), e].item() == klo[j, g, dim].item()
+
+
 def test_decode_tc_scan_exact_ties(msa):
     # zero queries: every score is exactly 0, so the lowest block indices win
     w = mi.Workload("dtc_ties", "decode", 1, 100_000, 32, 8, 128, 64, 32, "bf16", n_query=4)
