@@ -227,9 +227,7 @@ class DecodeRunner:
         # the encoded images the decode kernels stream with one bulk copy per tile
         _, khi, klo = (t[0] for t in msa.pool_keys(self.k[None], w.block, split=True))
         self.kt, self.vt, self.bt = msa.encode_bank(self.k, self.v, khi, klo, w.block)
-        del khi, klo
-        self.k = self.v = None                  # the step reads only the encoded bank
-        torch.cuda.empty_cache()
+        del khi, klo                            # the step reads only the encoded bank
         dev = self.q.device
         self.p = msa.params(batch=1, seq=w.seq, hq=w.hq, hkv=w.hkv, d=w.d, block=w.block,
                             topk=w.topk, scale=w.scale, dtype=self.q.dtype)
@@ -248,19 +246,24 @@ class DecodeRunner:
         self.launches_per_step = 6
 
     def step(self, events=None):
+        # msa_decode_fwd_tiled as its two calls, so the phases can be timed apart
         s = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
         P, w = self.ptr, self.w
         if events:
             events[0].record()
-        self.check("msa_decode_fwd_tiled", self.lib.msa_decode_fwd_tiled(
-            self.pp, w.n_query, P["q"], P["bt"], P["kt"], P["vt"], P["idx"], P["o"], P["lse"],
-            P["ws"], self.ws.numel(), s))
+        self.check("msa_decode_select_tiled", self.lib.msa_decode_select_tiled(
+            self.pp, w.n_query, P["q"], P["bt"], P["idx"], P["ws"], self.ws.numel(), s))
         if events:
             events[1].record()
+        self.check("msa_decode_attn_tiled", self.lib.msa_decode_attn_tiled(
+            self.pp, w.n_query, P["q"], P["kt"], P["vt"], P["idx"], P["o"], P["lse"], P["ws"],
+            self.ws.numel(), s))
+        if events:
+            events[2].record()
 
 
 def run_decode(args, world, rank, local):
-    w = mi.WORKLOADS[args.workload]
+    w = workload_of(args)
     from block_sparse_top_mean_b200 import build
     if rank == 0:
         build.build()
@@ -270,7 +273,7 @@ def run_decode(args, world, rank, local):
     for _ in range(args.warmup):
         r.step()
     torch.cuda.synchronize()
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     # the bank (41 GB) is far larger than L2; the pooled keys (0.6 GB) too
     with ClockSampler(local) as clk:
@@ -284,17 +287,34 @@ def run_decode(args, world, rank, local):
         barrier(world)
     ms = max_over_ranks(start.elapsed_time(end) / args.steps, world)
     peaks, peak_src = load_peaks()
-    # bytes the step must move at least: the pooled-key bank once at 4 bytes per element
-    # (bf16 hi + lo planes, as exact as fp32 for the selection), the selected K/V blocks
-    # once per (query, group)
+    sel_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    att_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    # algorithmic bytes: the selection reads the pooled-key bank once at 4 bytes per element
+    # (bf16 hi + lo planes, as exact as fp32 for the selection); the attention reads the
+    # selected K/V blocks once per (query, group)
     kbar_bytes = float(w.nb * w.hkv * w.d * 4)
-    alg_bytes = kbar_bytes + work["attn_bytes"]
-    gbs = alg_bytes / (ms * 1e-3) / 1e9
-    roof = {"bound": "hbm", "kernel": "decode step (sample scan + threshold + scan + merge + "
-                                      "attention + combine)",
-            "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-            "frac": round(gbs / peaks["hbm_gbs"], 4), "peak_source": f"hbm_gbs of {peak_src}",
-            "traffic": None, "algorithmic_per_launch": alg_bytes}
+    phases = {
+        "select": {"ms": sel_ms, "bytes": kbar_bytes,
+                   "kernel": "msa_decode_select_tiled (sample scan + threshold + full "
+                             "tensor-core scan + list merge)",
+                   # DRAM bytes of its scan kernels in one ncu capture of a 1.2M-token bank
+                   # (sample 10.5 MB + scan 79.5 MB for 18,750 blocks), scaled by blocks
+                   "traffic": (10.52e6 + 79.46e6) * w.nb / 18750},
+        "attend": {"ms": att_ms, "bytes": float(work["attn_bytes"]),
+                   "kernel": "msa_decode_attn_tiled (streamed attention + split combine)",
+                   # the attention kernel's DRAM bytes in the same capture (526.3 MB read,
+                   # 16.8 MB written); they depend on the selection, not on the bank size
+                   "traffic": 543.09e6 * w.n_query * w.hkv * w.topk / (64 * 8 * 32)},
+    }
+    dom = max(phases.values(), key=lambda x: x["ms"])
+    gbs = dom["bytes"] / (dom["ms"] * 1e-3) / 1e9
+    roof = {"bound": "hbm", "kernel": dom["kernel"], "achieved": round(gbs, 1),
+            "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
+            "peak_source": f"hbm_gbs of {peak_src}", "traffic": round(dom["traffic"]),
+            "traffic_source": "ncu capture of a 1.2M-token bank, scaled (see profiles/)",
+            "algorithmic_per_launch": dom["bytes"]}
+    phase_line = {k: {"us": round(v["ms"] * 1e3, 1),
+                      "gbs": round(v["bytes"] / (v["ms"] * 1e-3) / 1e9, 1)} for k, v in phases.items()}
     e2e = None
     if not args.no_e2e:
         hq_ = r.q.cpu().pin_memory()
@@ -317,6 +337,9 @@ def run_decode(args, world, rank, local):
         e2e = {"value": round(ems * 1e3, 1), "unit": "us/step", "ms_per_step": round(ems, 4),
                "h2d_bytes_per_step": hq_.numel() * hq_.element_size(),
                "d2h_bytes_per_step": ho.numel() * ho.element_size()}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline_decode(w, r.q, seed=rank)
     line = {
         "metric": "decode us/step", "value": round(ms * 1e3, 1), "unit": "us/step",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -326,7 +349,7 @@ def run_decode(args, world, rank, local):
                    "hkv": w.hkv, "d": w.d, "block": w.block, "topk": w.topk,
                    "l2": "bank and pooled keys larger than L2, no flush",
                    "parallelism": f"{world} independent banks, one per GPU"},
-        "roofline": roof, "cpu_baseline": None, "e2e": e2e,
+        "phases": phase_line, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": r.launches_per_step * args.steps, "clocks": clk.summary(),
         "device_error_bits": r.msa.read_device_error(r.ws),
     }
@@ -335,7 +358,7 @@ def run_decode(args, world, rank, local):
 
 
 def run_ours(args, world, rank, local):
-    w = mi.WORKLOADS[args.workload]
+    w = workload_of(args)
     if w.kind != "prefill":
         return run_decode(args, world, rank, local)
     from block_sparse_top_mean_b200 import build
@@ -479,43 +502,47 @@ def cpu_baseline_prefill(w, r, flops, n_blocks=64, n_tokens=96):
             "kind": "oracle", "sample": sample, "extrapolated_s_per_step": round(t_full, 1)}
 
 
-def run_reference_decode(args, world, w):
-    """Oracle decode on the host: a sample of the queries per step, extrapolated to all
-    n_query.  The bank's pooled keys are an input of the step (offline encoding); random
-    values of the right shape stand in for them, since only time is measured here."""
+def cpu_baseline_decode(w, q, seed=0, n_s=2):
+    """Oracle decode of n_s queries (all groups) on one host core, extrapolated to
+    n_query.  The fp64 pooled keys of a 10M-token bank would take minutes to build on the
+    host; random values of the right shape stand in (only the time is measured), while
+    K and V are the workload's bank, generated block by block as the oracle reads them."""
     import oracle
     from threadpoolctl import threadpool_limits
-    sys.path.insert(0, os.path.join(ROOT, "tests"))
-    from parity_util import HostView
-    dev = "cuda" if torch.cuda.is_available() else "cpu"
-    q, kb, vb = mi.decode_inputs(w, device=dev, seed=0)
     kbar = mi.normal((w.nb, w.hkv, w.d), 7, 7, "cpu", torch.float32).numpy().astype(np.float64)
     Qd = q.float().cpu().numpy()
-    K, V = HostView(kb), HostView(vb)
-    n_s = 2
+    K, V = mi.lazy_decode_bank(w, seed)
+    with threadpool_limits(limits=1):
+        t0 = time.perf_counter()
+        oracle.decode_rows(Qd, kbar, K, V, w.seq, w.block, w.topk, w.scale,
+                           queries=list(range(n_s)))
+        t = (time.perf_counter() - t0) / n_s * w.n_query
+    sample = (f"{n_s} of {w.n_query} queries (all {w.hkv} groups), extrapolated to "
+              f"{w.n_query}; numpy fp64, 1 thread; random stand-in pooled keys")
+    return {"value": round(t * 1e6, 1), "unit": "us/step", "cores": 1, "kind": "oracle",
+            "sample": sample}
+
+
+def run_reference_decode(args, world, w):
+    """The oracle arm for decode: a bounded sample of the queries per step."""
+    q, _, _ = mi.decode_inputs(w, device="cpu", seed=0, bank=False)
     times = []
     for s_ in range(args.warmup + args.steps):
-        qs = [(s_ * n_s + i) % w.n_query for i in range(n_s)]
-        with threadpool_limits(limits=1):
-            t0 = time.perf_counter()
-            oracle.decode_rows(Qd, kbar, K, V, w.seq, w.block, w.topk, w.scale, queries=qs)
-            t1 = time.perf_counter()
+        qs = torch.roll(q, shifts=-2 * s_, dims=0)
+        cb = cpu_baseline_decode(w, qs)
         if s_ >= args.warmup:
-            times.append((t1 - t0) / n_s * w.n_query)
+            times.append(cb["value"] * 1e-6)
     t = statistics.mean(times)
-    sample = (f"{n_s} of {w.n_query} queries (all {w.hkv} groups) per step, extrapolated to "
-              f"{w.n_query}; numpy fp64, 1 thread")
     line = {
-        "impl": "reference", "metric": "decode us/step", "value": t * 1e6, "unit": "us/step",
-        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3,
-        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic",
+        "impl": "reference", "metric": "decode us/step", "value": round(t * 1e6, 1),
+        "unit": "us/step", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": t * 1e3, "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": w.name, "n_query": w.n_query, "bank_tokens": w.seq, "hq": w.hq,
                    "hkv": w.hkv, "d": w.d, "block": w.block, "topk": w.topk,
                    "parallelism": "host oracle, rank 0 only"},
-        "cpu_baseline": {"value": t * 1e6, "unit": "us/step", "cores": 1, "kind": "oracle",
-                         "sample": sample},
-        "e2e": {"value": t * 1e6, "unit": "us/step", "h2d_bytes_per_step": 0,
+        "cpu_baseline": dict(cb, value=round(t * 1e6, 1)),
+        "e2e": {"value": round(t * 1e6, 1), "unit": "us/step", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -526,7 +553,7 @@ def run_reference(args, world, rank):
     host cores on a bounded sample of the same workload."""
     if rank != 0:
         return
-    w = mi.WORKLOADS[args.workload]
+    w = workload_of(args)
     if w.kind == "decode":
         return run_reference_decode(args, world, w)
     attn, score = prefill_flops(w)
@@ -563,6 +590,13 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
+def workload_of(args) -> mi.Workload:
+    w = mi.WORKLOADS[args.workload]
+    if args.seq is not None:
+        w = w.with_(name=f"{w.name}@seq{args.seq}", seq=args.seq)
+    return w
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -572,6 +606,9 @@ def main():
     ap.add_argument("--workload", default="prefill_1m_b256_k16", choices=list(mi.WORKLOADS))
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--seq", type=int, default=None,
+                    help="override the workload's sequence / bank length (small profiling "
+                         "captures only; the JSON line then names the changed workload)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     world, rank, local = dist_setup()

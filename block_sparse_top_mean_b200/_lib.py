@@ -38,6 +38,11 @@ SIGNATURES = {
     "msa_bank_tiles_bytes": (c_size_t, [c_void_p, c_int32]),
     "msa_encode_bank": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                   c_void_p, c_void_p, c_void_p]),
+    "msa_decode_select_tiled": (c_int32, [c_void_p, c_int64, c_void_p, c_void_p, c_void_p,
+                                          c_void_p, c_size_t, c_void_p]),
+    "msa_decode_attn_tiled": (c_int32, [c_void_p, c_int64, c_void_p, c_void_p, c_void_p,
+                                        c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
+                                        c_void_p]),
     "msa_decode_fwd_tiled": (c_int32, [c_void_p, c_int64, c_void_p, c_void_p, c_void_p,
                                        c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                        c_size_t, c_void_p]),

@@ -290,33 +290,59 @@ msa_status msa_encode_bank(const msa_params* p, const void* k_bank, const void* 
                                              v_tiles, kbar_tiles, (cudaStream_t)stream));
 }
 
+// Common checks of the encoded-bank decode calls; sets *empty for a call with no work.
+static msa_status tiled_checks(const msa_params* p, int64_t n_query, const void* q,
+                               const void* const* bufs, int nbufs, const void* ws,
+                               size_t ws_bytes, Shape* s, bool* empty) {
+  msa_status st = check_params(p, true, s);
+  if (st != MSA_OK) return st;
+  if (n_query < 0) return MSA_ERR_INVALID_ARG;
+  *empty = n_query == 0 || s->seq == 0;
+  if (*empty) return MSA_OK;
+  if (n_query > 65535 * 64) return MSA_ERR_UNSUPPORTED;
+  if (!tiled_decode_supported(*s)) return MSA_ERR_UNSUPPORTED;
+  if (q == nullptr || !aligned16(q)) return MSA_ERR_INVALID_ARG;
+  for (int i = 0; i < nbufs; ++i)
+    if (bufs[i] == nullptr || !aligned16(bufs[i])) return MSA_ERR_INVALID_ARG;
+  return check_ws(*s, MSA_OP_DECODE, n_query, ws, ws_bytes);
+}
+
+msa_status msa_decode_select_tiled(const msa_params* p, int64_t n_query, const void* q,
+                                   const void* kbar_tiles, int32_t* idx, void* ws,
+                                   size_t ws_bytes, msa_stream_t stream) {
+  Shape s;
+  bool empty = false;
+  const void* bufs[] = {kbar_tiles, idx};
+  msa_status st = tiled_checks(p, n_query, q, bufs, 2, ws, ws_bytes, &s, &empty);
+  if (st != MSA_OK || empty) return st;
+  return cuda_status(msa::launch_topk_decode_tc(s, n_query, q, nullptr, nullptr, kbar_tiles,
+                                                idx, ws_body(ws), err_word(ws),
+                                                (cudaStream_t)stream));
+}
+
+msa_status msa_decode_attn_tiled(const msa_params* p, int64_t n_query, const void* q,
+                                 const void* k_tiles, const void* v_tiles, const int32_t* idx,
+                                 void* o, float* lse, void* ws, size_t ws_bytes,
+                                 msa_stream_t stream) {
+  Shape s;
+  bool empty = false;
+  const void* bufs[] = {k_tiles, v_tiles, idx, o};
+  msa_status st = tiled_checks(p, n_query, q, bufs, 4, ws, ws_bytes, &s, &empty);
+  if (st != MSA_OK || empty) return st;
+  char* att_ws = ws_body(ws) + round256(decode_sel_ws(s, n_query));
+  return cuda_status(msa::launch_attn_decode(s, n_query, q, nullptr, nullptr, k_tiles, v_tiles,
+                                             idx, o, lse, att_ws, err_word(ws),
+                                             (cudaStream_t)stream));
+}
+
 msa_status msa_decode_fwd_tiled(const msa_params* p, int64_t n_query, const void* q,
                                 const void* kbar_tiles, const void* k_tiles,
                                 const void* v_tiles, int32_t* idx, void* o, float* lse,
                                 void* ws, size_t ws_bytes, msa_stream_t stream) {
-  Shape s;
-  msa_status st = check_params(p, true, &s);
+  msa_status st = msa_decode_select_tiled(p, n_query, q, kbar_tiles, idx, ws, ws_bytes, stream);
   if (st != MSA_OK) return st;
-  if (n_query < 0) return MSA_ERR_INVALID_ARG;
-  if (n_query == 0 || s.seq == 0) return MSA_OK;
-  if (n_query > 65535 * 64) return MSA_ERR_UNSUPPORTED;
-  if (!tiled_decode_supported(s)) return MSA_ERR_UNSUPPORTED;
-  if (q == nullptr || kbar_tiles == nullptr || k_tiles == nullptr || v_tiles == nullptr ||
-      idx == nullptr || o == nullptr)
-    return MSA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(kbar_tiles) || !aligned16(k_tiles) || !aligned16(v_tiles) ||
-      !aligned16(o))
-    return MSA_ERR_INVALID_ARG;
-  if ((st = check_ws(s, MSA_OP_DECODE, n_query, ws, ws_bytes)) != MSA_OK) return st;
-  cudaStream_t cs = (cudaStream_t)stream;
-  char* sel_ws = ws_body(ws);
-  char* att_ws = sel_ws + round256(decode_sel_ws(s, n_query));
-  cudaError_t e = msa::launch_topk_decode_tc(s, n_query, q, nullptr, nullptr, kbar_tiles, idx,
-                                             sel_ws, err_word(ws), cs);
-  if (e == cudaSuccess)
-    e = msa::launch_attn_decode(s, n_query, q, nullptr, nullptr, k_tiles, v_tiles, idx, o, lse,
-                                att_ws, err_word(ws), cs);
-  return cuda_status(e);
+  return msa_decode_attn_tiled(p, n_query, q, k_tiles, v_tiles, idx, o, lse, ws, ws_bytes,
+                               stream);
 }
 
 msa_status msa_read_device_error(const void* ws, int32_t* bits, msa_stream_t stream) {

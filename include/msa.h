@@ -195,6 +195,19 @@ MSA_API msa_status msa_encode_bank(const msa_params* p, const void* k_bank, cons
                                    const void* kbar_hi, const void* kbar_lo, void* k_tiles,
                                    void* v_tiles, void* kbar_tiles, msa_stream_t stream);
 
+/* The two steps of a decode over an encoded bank, for callers that schedule them apart
+ * (msa_decode_fwd_tiled below is the two in sequence).  Both take the same decode
+ * workspace; the selection writes idx [n_query, hkv, topk] as msa_decode_fwd does, the
+ * attention reads it (entries -1 skipped, others must be in [0, nb): an out-of-range
+ * entry is skipped and sets MSA_DEVERR_IDX_RANGE). */
+MSA_API msa_status msa_decode_select_tiled(const msa_params* p, int64_t n_query, const void* q,
+                                           const void* kbar_tiles, int32_t* idx, void* ws,
+                                           size_t ws_bytes, msa_stream_t stream);
+MSA_API msa_status msa_decode_attn_tiled(const msa_params* p, int64_t n_query, const void* q,
+                                         const void* k_tiles, const void* v_tiles,
+                                         const int32_t* idx, void* o, float* lse, void* ws,
+                                         size_t ws_bytes, msa_stream_t stream);
+
 /* msa_decode_fwd over an encoded bank: the same selection (tensor-core scan of the
  * pooled-key planes) and the same attention, fed by 1-D bulk copies.
  * ws: msa_workspace_bytes(p, MSA_OP_DECODE, n_query). */

@@ -25,9 +25,11 @@ from __future__ import annotations
 import math
 from dataclasses import dataclass, field
 
+import numpy as np
 import torch
 
 __all__ = [
+    "LazyBank", "lazy_decode_bank",
     "Workload", "WORKLOADS", "normal", "planted_blocks", "planted_directions",
     "prefill_inputs", "decode_inputs", "STREAM_Q", "STREAM_K", "STREAM_V",
     "STREAM_U", "STREAM_PLANT", "STREAM_DECODE_Q",
@@ -75,7 +77,10 @@ def stream_base(seed: int, stream: int) -> int:
 
 
 def _normal_chunk(base: int, start: int, count: int, device) -> torch.Tensor:
-    i = torch.arange(start, start + count, dtype=torch.int64, device=device)
+    return _normal_idx(base, torch.arange(start, start + count, dtype=torch.int64, device=device))
+
+
+def _normal_idx(base: int, i: torch.Tensor) -> torch.Tensor:
     g = _signed(_GAMMA)
     b = _signed(base)
     a = _mix64_t(b + (2 * i + 1) * g)
@@ -108,6 +113,32 @@ def normal(shape, seed: int, stream: int, device="cpu", dtype=torch.float32,
             x = shift(x, start)
         out[start:start + cnt] = x.to(torch.float32).to(dtype)
     return out.view(shape)
+
+
+class LazyBank:
+    """The bank tensor normal((S, hkv, d), seed, stream) of a decode workload, generated on
+    demand: bank[p, g] returns the rows p (index array) of head g as fp32 numpy values of
+    the `dtype`-rounded elements, identical to the materialised tensor's.  Lets host-side
+    code read a few selected blocks of a 10M-token bank without building 20 GB."""
+
+    def __init__(self, shape, seed: int, stream: int, dtype=torch.bfloat16):
+        self.shape = tuple(int(s) for s in shape)
+        self.base = stream_base(seed, stream)
+        self.dtype = dtype
+
+    def __getitem__(self, key):
+        p, g = key
+        S, hkv, d = self.shape
+        p = torch.as_tensor(np.asarray(p), dtype=torch.int64).reshape(-1)
+        flat = (p[:, None] * hkv + int(g)) * d + torch.arange(d, dtype=torch.int64)[None, :]
+        x = _normal_idx(self.base, flat.reshape(-1)).to(torch.float32).to(self.dtype)
+        return x.float().reshape(len(p), d).numpy()
+
+
+def lazy_decode_bank(w: "Workload", seed: int = 0):
+    """(K, V) of decode_inputs(w, seed=seed) as LazyBank views."""
+    return (LazyBank((w.seq, w.hkv, w.d), seed, STREAM_K, w.torch_dtype),
+            LazyBank((w.seq, w.hkv, w.d), seed, STREAM_V, w.torch_dtype))
 
 
 @dataclass(frozen=True)
