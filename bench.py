@@ -79,12 +79,46 @@ CLOCK_Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active
 
 
 class ClockSampler:
+    """Samples SM clock, power and clock-event reasons of one GPU while the timed region
+    runs: NVML from a host thread every 2 ms (short regions such as a decode step get
+    samples too), else nvidia-smi every 200 ms.  Reads only; changes no setting."""
+
+    # NVML clock-event reason bits
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap"}
+
     def __init__(self, index: int):
         self.index = index
         self.proc = None
+        self.thread = None
+        self.rows = []
         self.path = os.path.join("/tmp", f"msa_clocks_{os.getpid()}.csv")
 
+    def _nvml_loop(self, nv, h):
+        while not self.stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+                pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.rows.append((float(sm), float(mx), pw,
+                                  [name for bit, name in self.REASONS.items() if rs & bit]))
+            except Exception:  # noqa: BLE001 - sampling is best effort
+                pass
+            self.stop.wait(0.002)
+
     def __enter__(self):
+        try:
+            import threading
+            import pynvml as nv
+            nv.nvmlInit()
+            h = nv.nvmlDeviceGetHandleByIndex(self.index)
+            self.stop = threading.Event()
+            self.thread = threading.Thread(target=self._nvml_loop, args=(nv, h), daemon=True)
+            self.thread.start()
+            return self
+        except Exception:  # noqa: BLE001 - fall back to nvidia-smi
+            self.thread = None
         try:
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(
@@ -96,6 +130,9 @@ class ClockSampler:
         return self
 
     def __exit__(self, *a):
+        if self.thread is not None:
+            self.stop.set()
+            self.thread.join(timeout=5)
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -103,28 +140,28 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
             self.f.close()
+            names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+            for line in open(self.path):
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    self.rows.append((float(parts[1]), float(parts[2]), float(parts[3]),
+                                      [names[k] for k, x in enumerate(parts[5:9])
+                                       if x.lower().startswith("active")]))
+                except ValueError:
+                    continue
 
     def summary(self):
-        if self.proc is None:
-            return None
-        rows = []
-        for line in open(self.path):
-            parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[5:9]))
-            except ValueError:
-                continue
+        rows = self.rows
         if not rows:
             return None
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[k] for r in rows for k, x in enumerate(r[3])
-                          if x.lower().startswith("active")})
+        reasons = sorted({n for r in rows for n in r[3]})
         busy = [r[0] for r in rows if r[2] > 300.0] or [r[0] for r in rows]
         return {"sm_mhz": statistics.median(busy), "sm_max_mhz": max(r[1] for r in rows),
                 "reasons": reasons, "samples": len(rows),
-                "power_w_max": max(r[2] for r in rows)}
+                "power_w_max": round(max(r[2] for r in rows), 1),
+                "source": "nvml 2 ms" if self.thread is not None else "nvidia-smi 200 ms"}
 
 
 # ------------------------------------------------------------------ distributed plumbing

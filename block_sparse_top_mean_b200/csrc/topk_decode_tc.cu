@@ -695,7 +695,8 @@ cudaError_t launch_topk_decode_tc(const Shape& s, int64_t n_query, const void* q
     }
     if (e != cudaSuccess) return e;
     const int64_t rows = n_query * s.hkv;
-    sample_threshold_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(gmax, tinit, rows,
+    // two warps per block: the few hundred warps spread over all SMs
+    sample_threshold_kernel<<<(unsigned)((rows + 1) / 2), 64, 0, st>>>(gmax, tinit, rows,
                                                                        (int)(gs.nch * 4));
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
@@ -708,7 +709,7 @@ cudaError_t launch_topk_decode_tc(const Shape& s, int64_t n_query, const void* q
   }
   if (e != cudaSuccess) return e;
   const int64_t warps = n_query * s.hkv;
-  topk_decode_merge_kernel<<<(unsigned)((warps + 7) / 8), 256, 0, st>>>(cand, idx, g);
+  topk_decode_merge_kernel<<<(unsigned)((warps + 1) / 2), 64, 0, st>>>(cand, idx, g);
   return cudaGetLastError();
 }
 
