@@ -574,18 +574,24 @@ attn_tiles_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
       __nv_bfloat16* dst = po + ((((b * g.hkv + gg) * g.S + t) * g.kslots + pslot) * G + h) * kD;
+      // O in two halves of 64 columns, two TMEM loads in flight per wait
 #pragma unroll 1
-      for (int qd = 0; qd < 4; ++qd) {
-        uint32_t ov[32];
-        tmem_ld32(oX + qd * 32, ov);
+      for (int q2 = 0; q2 < 2; ++q2) {
+        uint32_t ov[2][32];
+        tmem_ld32(oX + q2 * 64, ov[0]);
+        tmem_ld32(oX + q2 * 64 + 32, ov[1]);
         tmem_ld_wait();
-        uint32_t ob[16];
 #pragma unroll
-        for (int k = 0; k < 32; k += 2)
-          ob[k / 2] = pack_bf16x2(__uint_as_float(ov[k]) * inv, __uint_as_float(ov[k + 1]) * inv);
-        if (valid) {
-          st_global_v8(dst + qd * 32, ob);
-          st_global_v8(dst + qd * 32 + 16, ob + 8);
+        for (int u = 0; u < 2; ++u) {
+          uint32_t ob[16];
+#pragma unroll
+          for (int k = 0; k < 32; k += 2)
+            ob[k / 2] = pack_bf16x2(__uint_as_float(ov[u][k]) * inv,
+                                    __uint_as_float(ov[u][k + 1]) * inv);
+          if (valid) {
+            st_global_v8(dst + (q2 * 2 + u) * 32, ob);
+            st_global_v8(dst + (q2 * 2 + u) * 32 + 16, ob + 8);
+          }
         }
       }
       tc_fence_before();
