@@ -492,14 +492,19 @@ attn_tiles_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
         if (!mbar_wait_warp(&bars->s_full[X], ph)) { ok = false; break; }
         tc_fence_after();
         const bool full = __all_sync(0xffffffffu, lim == kChunkKeys);
-        // pass 1: row max of the raw scores (two TMEM loads per wait)
-        float mx = -CUDART_INF_F;
+        // One pass over S in two halves of 64 columns.  Each half's max is taken from the
+        // registers just loaded; the exponent reference mref only moves when a half's max
+        // exceeds it by more than 2^8 (always for the first half of a row's first chunk),
+        // and then O, l, and the P already made for this chunk are rescaled.
+        float sum = 0.f;
+        bool o_ready = c == 0;                           // O holds nothing to rescale yet
 #pragma unroll
         for (int hq2 = 0; hq2 < 2; ++hq2) {
           uint32_t sv[2][32];
           tmem_ld32(sX + hq2 * 64, sv[0]);
           tmem_ld32(sX + hq2 * 64 + 32, sv[1]);
           tmem_ld_wait();
+          float mx = -CUDART_INF_F;
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
             const int qd = hq2 * 2 + u;
@@ -512,37 +517,50 @@ attn_tiles_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
                 if (qd * 32 + k < lim) mx = fmaxf(mx, __uint_as_float(sv[u][k]));
             }
           }
-        }
-        const float mc = lim > 0 ? mx * c2 : -CUDART_INF_F;
-        // exponent reference: chunk 0 sets it; a later chunk keeps it unless its max is
-        // more than 2^8 larger, which requires rescaling O (after the earlier PV is done)
-        const bool need = mc > mref + kRescaleLog2;
-        if (c > 0 && __any_sync(0xffffffffu, need)) {
-          if (!mbar_wait_warp(&bars->pv_done[X], chunk_phase(n, c - 1, nch))) { ok = false; break; }
-          tc_fence_after();
-          const float f = need ? fast_exp2(mref - mc) : 1.f;
+          const float mc = lim > hq2 * 64 ? mx * c2 : -CUDART_INF_F;
+          const bool need = mc > mref + kRescaleLog2;
+          if (__any_sync(0xffffffffu, need)) {
+            const float f = need ? fast_exp2(mref - mc) : 1.f;
+            if (!o_ready) {
+              // O must hold every earlier chunk before it is rescaled in TMEM
+              if (!mbar_wait_warp(&bars->pv_done[X], chunk_phase(n, c - 1, nch))) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              o_ready = true;
+            }
+            // (rare) rescale in 16-column pieces, keeping S of this half in registers
+            if (c > 0) {
+#pragma unroll 1
+              for (int qd = 0; qd < 8; ++qd) {
+                uint32_t ov[16];
+                tmem_ld16(oX + qd * 16, ov);
+                tmem_ld_wait();
 #pragma unroll
-          for (int qd = 0; qd < 4; ++qd) {
-            uint32_t ov[32];
-            tmem_ld32(oX + qd * 32, ov);
-            tmem_ld_wait();
+                for (int k = 0; k < 16; ++k) ov[k] = __float_as_uint(__uint_as_float(ov[k]) * f);
+                tmem_st16(oX + qd * 16, ov);
+              }
+              tmem_st_wait();
+            }
+            if (hq2 == 1) {                             // this chunk's first half of P
+              tmem_st_wait();
+#pragma unroll 1
+              for (int qd = 0; qd < 2; ++qd) {
+                uint32_t pv[16];
+                tmem_ld16(sX + qd * 16, pv);
+                tmem_ld_wait();
 #pragma unroll
-            for (int k = 0; k < 32; ++k) ov[k] = __float_as_uint(__uint_as_float(ov[k]) * f);
-            tmem_st32(oX + qd * 32, ov);
+                for (int k = 0; k < 16; ++k)
+                  pv[k] = pack_bf16x2(bf16lo_to_f32(pv[k]) * f, bf16hi_to_f32(pv[k]) * f);
+                tmem_st16(sX + qd * 16, pv);
+              }
+            }
+            l *= f;
+            sum *= f;
+            if (need) mref = mc;
           }
-          tmem_st_wait();
-          l *= f;
-        }
-        if (need) mref = mc;
-        const float mb = mref > -CUDART_INF_F ? mref : 0.f;
-        // pass 2: P = 2^(s*c2 - mref), packed two bf16 per column over S_X
-        float sum = 0.f;
-#pragma unroll
-        for (int hq2 = 0; hq2 < 2; ++hq2) {
-          uint32_t sv[2][32];
-          tmem_ld32(sX + hq2 * 64, sv[0]);
-          tmem_ld32(sX + hq2 * 64 + 32, sv[1]);
-          tmem_ld_wait();
+          const float mb = mref > -CUDART_INF_F ? mref : 0.f;
           uint32_t pk[32];
 #pragma unroll
           for (int u = 0; u < 2; ++u)
@@ -560,8 +578,10 @@ attn_tiles_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
               sum += p0 + p1;
               pk[u * 16 + k / 2] = pack_bf16x2(p0, p1);
             }
+          // P of this half over S columns already consumed
           tmem_st32(sX + hq2 * 32, pk);
         }
+        if (!ok) break;
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&bars->p_full[X]);
