@@ -253,21 +253,47 @@ topk_tc_kernel(const __grid_constant__ CUtensorMap tmHi, const __grid_constant__
       const int rem = own - j0;
       const int lim = rem <= 0 ? 0 : (rem >= 64 ? 64 : rem);
       if (!pass2) {
+        // the 16 group maxima of these 64 columns, sorted (bitonic network), then merged
+        // into the descending list: max against the reversed batch, then a bitonic merge
+        constexpr int kNG = 64 / kGroup;
+        float v[kNG];
 #pragma unroll
-        for (int q4 = 0; q4 < 64 / kGroup; ++q4) {
-          float v = -CUDART_INF_F;
+        for (int q4 = 0; q4 < kNG; ++q4) {
+          v[q4] = -CUDART_INF_F;
 #pragma unroll
           for (int u = 0; u < kGroup; ++u) {
             const int k = q4 * kGroup + u;
-            if (k < lim) v = fmaxf(v, __uint_as_float(sv[k >> 5][k & 31]));
-          }
-#pragma unroll
-          for (int e = 0; e < KM; ++e) {           // bubble v into the descending list
-            const float hi = fmaxf(gm[e], v);
-            v = fminf(gm[e], v);
-            gm[e] = hi;
+            if (k < lim) v[q4] = fmaxf(v[q4], __uint_as_float(sv[k >> 5][k & 31]));
           }
         }
+#pragma unroll
+        for (int kk = 2; kk <= kNG; kk <<= 1)
+#pragma unroll
+          for (int jj = kk >> 1; jj > 0; jj >>= 1)
+#pragma unroll
+            for (int i = 0; i < kNG; ++i) {
+              const int o = i ^ jj;
+              if (o > i) {
+                const float a = v[i], bq = v[o];
+                const bool desc = (i & kk) == 0;
+                v[i] = desc ? fmaxf(a, bq) : fminf(a, bq);
+                v[o] = desc ? fminf(a, bq) : fmaxf(a, bq);
+              }
+            }
+#pragma unroll
+        for (int e = 0; e < KM; ++e)
+          if (KM - 1 - e < kNG) gm[e] = fmaxf(gm[e], v[KM - 1 - e]);
+#pragma unroll
+        for (int jj = KM >> 1; jj > 0; jj >>= 1)
+#pragma unroll
+          for (int i = 0; i < KM; ++i) {
+            const int o = i ^ jj;
+            if (o > i) {
+              const float a = gm[i], bq = gm[o];
+              gm[i] = fmaxf(a, bq);
+              gm[o] = fminf(a, bq);
+            }
+          }
       } else {
 #pragma unroll
         for (int k = 0; k < 64; ++k) {
