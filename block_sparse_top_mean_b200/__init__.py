@@ -20,7 +20,7 @@ from ._lib import (  # noqa: F401
 
 __all__ = [
     "params", "workspace", "pool_keys", "block_scores", "topk_select", "sparse_attn_fwd",
-    "prefill_fwd", "decode_fwd", "decode_fwd_static", "encode_bank", "decode_fwd_tiled",
+    "prefill_fwd", "decode_fwd", "decode_fwd_static", "encode_bank", "decode_fwd_tiled", "decode_select_tiled", "decode_attn_tiled",
     "read_device_error",
     "clear_device_error", "version",
     "MsaError", "MsaParams",
@@ -235,6 +235,37 @@ def decode_fwd_tiled(q, kbar_tiles, k_tiles, v_tiles, seq: int, hkv: int, block:
         ctypes.byref(p), nq, _ptr(q), _ptr(kbar_tiles), _ptr(k_tiles), _ptr(v_tiles), _ptr(idx),
         _ptr(o), _ptr(lse), _ptr(ws), ws.numel(), _stream(q.device)))
     return o, lse, idx
+
+
+def decode_select_tiled(q, kbar_tiles, seq: int, hkv: int, block: int, topk: int, ws=None,
+                        idx=None):
+    """The selection step of decode_fwd_tiled: idx [n_query, hkv, topk]."""
+    nq = q.shape[0]
+    p = _bank_params(q, seq, hkv, block, topk, None)
+    if idx is None:
+        idx = torch.empty(nq, hkv, topk, dtype=torch.int32, device=q.device)
+    if ws is None:
+        ws = workspace(p, OP_DECODE, nq, device=q.device)
+    _lib.check("msa_decode_select_tiled", _lib.load().msa_decode_select_tiled(
+        ctypes.byref(p), nq, _ptr(q), _ptr(kbar_tiles), _ptr(idx), _ptr(ws), ws.numel(),
+        _stream(q.device)))
+    return idx
+
+
+def decode_attn_tiled(q, k_tiles, v_tiles, idx, seq: int, hkv: int, block: int, scale=None,
+                      want_lse=True, ws=None):
+    """The attention step of decode_fwd_tiled for a given idx [n_query, hkv, topk]."""
+    nq, hq, d = q.shape
+    topk = idx.shape[-1]
+    p = _bank_params(q, seq, hkv, block, topk, scale)
+    o = torch.empty_like(q)
+    lse = torch.empty(nq, hq, dtype=torch.float32, device=q.device) if want_lse else None
+    if ws is None:
+        ws = workspace(p, OP_DECODE, nq, device=q.device)
+    _lib.check("msa_decode_attn_tiled", _lib.load().msa_decode_attn_tiled(
+        ctypes.byref(p), nq, _ptr(q), _ptr(k_tiles), _ptr(v_tiles), _ptr(idx), _ptr(o), _ptr(lse),
+        _ptr(ws), ws.numel(), _stream(q.device)))
+    return o, lse
 
 
 def read_device_error(ws: torch.Tensor) -> int:

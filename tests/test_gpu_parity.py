@@ -270,6 +270,44 @@ def test_decode_tiled_bank_matches_natural_layout(msa, w):
                      queries=list(range(0, w.n_query, 5)))
 
 
+def test_decode_attn_tiled_given_selection(msa):
+    # the attention step alone: -1 entries are skipped, an out-of-range entry is skipped
+    # and reported, and every other row is the oracle's attention over its given blocks
+    w = mi.Workload("dattn", "decode", 1, 80_000, 32, 8, 128, 64, 16, "bf16", n_query=6)
+    q, kb, vb = mi.decode_inputs(w, device="cuda")
+    _, khi, klo = (t[0] for t in msa.pool_keys(kb[None], w.block, split=True))
+    kt, vt, bt = msa.encode_bank(kb, vb, khi, klo, w.block)
+    p = msa._bank_params(q, w.seq, w.hkv, w.block, w.topk, w.scale)
+    ws = msa.workspace(p, msa.OP_DECODE, w.n_query)
+    idx = msa.decode_select_tiled(q, bt, w.seq, w.hkv, w.block, w.topk, ws=ws)
+    gen = torch.Generator().manual_seed(3)
+    given = idx.clone()
+    given[0, 0, 5:] = -1                                   # a shorter set, padded
+    given[1, 2] = torch.randperm(w.nb, generator=gen)[:w.topk].sort().values.to(given)
+    o, lse = msa.decode_attn_tiled(q, kt, vt, given, w.seq, w.hkv, w.block, w.scale, ws=ws)
+    torch.cuda.synchronize()
+    assert msa.read_device_error(ws) == 0
+    kbar_np = pool_keys_chunked(kb[None], w.block)[0]
+    Qd = q.float().cpu().numpy()
+    gi = given.cpu().numpy()
+    override = {(n, g): [int(x) for x in gi[n, g]] for n in range(w.n_query) for g in range(w.hkv)}
+    ref = oracle.decode_rows(Qd, kbar_np, HostView(kb), HostView(vb), w.seq, w.block, w.topk,
+                             w.scale, idx_override=override)
+    G = w.hq // w.hkv
+    og, lg = o.float().cpu().numpy(), lse.cpu().numpy()
+    for r in ref:
+        assert np.abs(og[r.n, r.g * G:(r.g + 1) * G] - r.O).max() <= 2e-2, (r.n, r.g)
+        assert np.abs(lg[r.n, r.g * G:(r.g + 1) * G] - r.lse).max() <= 2e-3, (r.n, r.g)
+    bad = given.clone()
+    bad[3, 1, 0] = w.nb + 7
+    o2, _ = msa.decode_attn_tiled(q, kt, vt, bad, w.seq, w.hkv, w.block, w.scale, ws=ws)
+    assert msa.read_device_error(ws) & msa.DEVERR_IDX_RANGE
+    msa.clear_device_error(ws)
+    keep = torch.ones(w.n_query, w.hq, dtype=torch.bool)
+    keep[3, G:2 * G] = False
+    assert torch.equal(o2[keep], o[keep])
+
+
 def test_encode_bank_layout(msa):
     # spot-check the documented image layout against the natural tensors
     w = mi.Workload("enc", "decode", 1, 1000, 8, 2, 128, 64, 8, "bf16", n_query=1)
