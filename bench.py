@@ -226,9 +226,11 @@ class PrefillRunner:
                                                      "lse", "ws")}
         self.pp = ctypes.byref(self.p)
         # own kernels per step (memsets excluded): pool 1; selection: tensor-core pass +
-        # exact pass over flagged tiles = 2; attention: count, scan, fill, tile table,
-        # tiles, merge = 6
-        self.launches_per_step = 9
+        # exact pass over flagged tiles = 2; attention, per token slab: count, scan, fill,
+        # tile table, tiles, merge = 6
+        slab = msa.attn_slab_tokens(self.p, _lib.OP_SPARSE_ATTN, n)
+        self.n_slabs = -(-w.seq // slab)
+        self.launches_per_step = 3 + 6 * self.n_slabs
 
     def step(self, events=None):
         s = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
@@ -452,6 +454,8 @@ def run_ours(args, world, rank, local):
         "config": {"workload": w.name, "batch_per_gpu": w.batch, "seq": w.seq, "hq": w.hq,
                    "hkv": w.hkv, "d": w.d, "block": w.block, "topk": w.topk,
                    "l2": "inputs larger than L2 (Q alone 8 GiB), no flush",
+                   "workspace_gib": round(r.ws.numel() / 2**30, 2),
+                   "attn_token_slabs": r.n_slabs,
                    "parallelism": f"{world} independent sequences, one per GPU"},
         "tokens_per_s": round(tokens_s, 1),
         "flops_per_step": {"attention": attn_flops, "scoring": score_flops},

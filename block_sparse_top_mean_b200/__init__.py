@@ -15,6 +15,7 @@ import torch
 from . import _lib
 from ._lib import (  # noqa: F401
     MsaError, MsaParams, OP_DECODE, OP_PREFILL, OP_SPARSE_ATTN, OP_TOPK_SELECT,
+    OP_SPARSE_ATTN_MIN, OP_PREFILL_MIN,
     DEVERR_IDX_RANGE, DEVERR_TIMEOUT, MSA_F32, MSA_BF16,
 )
 
@@ -62,6 +63,15 @@ def workspace(p: MsaParams, op: int, n_query: int = 0, device="cuda") -> torch.T
     ws = torch.empty(n, dtype=torch.uint8, device=device)
     ws[:256].zero_()
     return ws
+
+
+def attn_slab_tokens(p: MsaParams, op: int, ws_bytes: int) -> int:
+    """Tokens per slab the prefill attention walks with ws_bytes of workspace for `op`
+    (OP_SPARSE_ATTN or OP_PREFILL); p.seq means one pass, 0 means too small."""
+    n = _lib.load().msa_attn_slab_tokens(ctypes.byref(p), op, ws_bytes)
+    if n < 0:
+        raise MsaError("msa_attn_slab_tokens", _lib.MSA_ERR_INVALID_ARG, "invalid shapes or op")
+    return n
 
 
 def _prefill_params(q, k, block, topk, scale):

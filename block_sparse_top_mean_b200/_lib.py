@@ -13,7 +13,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmsa_b200
 MSA_OK, MSA_ERR_INVALID_ARG, MSA_ERR_UNSUPPORTED, MSA_ERR_WORKSPACE, MSA_ERR_CUDA, \
     MSA_ERR_DEVICE = range(6)
 MSA_F32, MSA_BF16 = 0, 1
-OP_TOPK_SELECT, OP_SPARSE_ATTN, OP_PREFILL, OP_DECODE = range(4)
+OP_TOPK_SELECT, OP_SPARSE_ATTN, OP_PREFILL, OP_DECODE, OP_SPARSE_ATTN_MIN, OP_PREFILL_MIN = range(6)
 DEVERR_IDX_RANGE, DEVERR_TIMEOUT = 0x1, 0x2
 
 # Every symbol include/msa.h declares, with (restype, argtypes).
@@ -21,6 +21,7 @@ SIGNATURES = {
     "msa_version": (c_char_p, []),
     "msa_status_string": (c_char_p, [c_int32]),
     "msa_workspace_bytes": (c_size_t, [c_void_p, c_int32, c_int64]),
+    "msa_attn_slab_tokens": (c_int64, [c_void_p, c_int32, c_size_t]),
     "msa_pool_keys": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
     "msa_block_scores": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
     "msa_topk_select": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,

@@ -39,6 +39,7 @@ constexpr float kLn2 = 0.6931471805599453f;
 
 struct Geom {
   int64_t S, nb, block, nseg;
+  int64_t t_base, t_end, slab;   // this call's token slab [t_base, t_end); partial rows per (b, g)
   int hq, hkv, G, topk, nsub, kslots, tpt, nch;
   float scale_log2;
 };
@@ -73,9 +74,9 @@ invert_hist_kernel(const int32_t* __restrict__ idx, int* __restrict__ counts,
                    int* __restrict__ cursor, int* __restrict__ entries, int* err, Geom g) {
   extern __shared__ int hist[];                       // nb * nsub counters
   const int nbs = (int)g.nb * g.nsub;
-  const int t0 = blockIdx.x * kInvTokens;
+  const int t0 = (int)g.t_base + blockIdx.x * kInvTokens;
   const int bg = blockIdx.y;                          // sequence * hkv + group
-  const int t1 = (int)min((int64_t)t0 + kInvTokens, g.S);
+  const int t1 = (int)min((int64_t)t0 + kInvTokens, g.t_end);
   const int own_max = (t1 - 1) / (int)g.block;        // segments beyond it stay empty
   const int used = min(nbs, (own_max + 1) * g.nsub);
   for (int i = threadIdx.x; i < used; i += kInvThreads) hist[i] = 0;
@@ -593,7 +594,8 @@ attn_tiles_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
       }
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
-      __nv_bfloat16* dst = po + ((((b * g.hkv + gg) * g.S + t) * g.kslots + pslot) * G + h) * kD;
+      const int64_t prow = (b * g.hkv + gg) * g.slab + (t - g.t_base);   // partial row of the slab
+      __nv_bfloat16* dst = po + ((prow * g.kslots + pslot) * G + h) * kD;
       // O in two halves of 64 columns, two TMEM loads in flight per wait
 #pragma unroll 1
       for (int q2 = 0; q2 < 2; ++q2) {
@@ -617,7 +619,7 @@ attn_tiles_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
       tc_fence_before();
       mbar_arrive(&bars->o_empty[X]);
       if (valid)
-        plse[(((b * g.hkv + gg) * g.S + t) * g.kslots + pslot) * G + h] =
+        plse[(prow * g.kslots + pslot) * G + h] =
             l > 0.f ? (mref + log2f(l)) * kLn2 : -CUDART_INF_F;
     }
   }
@@ -651,11 +653,13 @@ merge_partials_kernel(const int32_t* __restrict__ idx, const __nv_bfloat16* __re
   if (row >= n_rows) return;
   const int lt = threadIdx.x % TPR;
   const int h = lt / 8;
-  const int t = (int)(row % g.S);
-  const int64_t bg = row / g.S;
+  // partial row `row` of the slab = (sequence*hkv + group, token t_base + row % slab)
+  const int64_t bg = row / g.slab;
+  const int t = (int)(g.t_base + row % g.slab);
+  if (t >= g.t_end) return;
   const int64_t gg = bg % g.hkv, b = bg / g.hkv;
   const int own = t / (int)g.block;
-  const int32_t* irow = idx + row * g.topk;
+  const int32_t* irow = idx + (bg * g.S + t) * g.topk;
   const float* lrow = plse + row * g.kslots * G;
   const __nv_bfloat16* prow = po + row * g.kslots * G * kD + lt * 16;
   float mx = -CUDART_INF_F, den = 0.f;
@@ -731,15 +735,18 @@ Geom make_geom(const Shape& s) {
   g.nch = (int)(((s.block < kSegKeys ? s.block : (int64_t)kSegKeys) + kChunkKeys - 1) / kChunkKeys);
   g.nseg = s.batch * s.hkv * s.nb * g.nsub;
   g.scale_log2 = s.scale * kLog2e;
+  g.t_base = 0; g.t_end = s.seq; g.slab = s.seq;
   return g;
 }
 
-WsLayout layout_for(const Shape& s) {
+// Workspace of one call processing `slab` tokens of every (sequence, group) at a time: the
+// per-segment index of the whole call, the entries and tiles of one slab, and the
+// slab's partials (which dominate: kslots x G x 256 B + 4 B per (token, group)).
+WsLayout layout_for(const Shape& s, int64_t slab) {
   const Geom g = make_geom(s);
-  const int64_t n_sel = s.batch * s.hkv * s.seq * s.topk;
-  const int64_t n_entries = n_sel * g.nsub;
+  const int64_t n_entries = s.batch * s.hkv * slab * s.topk * g.nsub;
   const int64_t n_tiles_max = n_entries / g.tpt + g.nseg + 1;
-  const int64_t rows = s.batch * s.hkv * s.seq;
+  const int64_t rows = s.batch * s.hkv * slab;
   WsLayout L{};
   size_t o = 0;
   L.counts = o;   o += up256(g.nseg * 4);
@@ -755,6 +762,23 @@ WsLayout layout_for(const Shape& s) {
   return L;
 }
 
+// Slabs are whole multiples of the inversion's token range (or the whole sequence).
+constexpr size_t kSlabBudget = (size_t)32 << 30;   // recommended workspace: <= 32 GiB of slab
+int64_t min_slab(const Shape& s) { return s.seq < kInvTokens ? s.seq : kInvTokens; }
+int64_t slab_for(const Shape& s, size_t bytes) {
+  if (layout_for(s, s.seq).total <= bytes) return s.seq;
+  int64_t lo = 1, hi = s.seq / kInvTokens;         // in units of kInvTokens
+  if (hi < 1) return s.seq;
+  while (lo < hi) {                                // largest fitting multiple
+    const int64_t mid = (lo + hi + 1) / 2;
+    if (layout_for(s, mid * kInvTokens).total <= bytes) lo = mid; else hi = mid - 1;
+  }
+  // same number of slabs, evened out (never larger than the largest that fits)
+  const int64_t units = (s.seq + kInvTokens - 1) / kInvTokens;
+  const int64_t n_slabs = (units + lo - 1) / lo;
+  return (units + n_slabs - 1) / n_slabs * kInvTokens;
+}
+
 template <int G>
 cudaError_t run_tc(const Shape& s, const Geom& g, const CUtensorMap& mk, const CUtensorMap& mv,
                    const void* q, const int32_t* idx, void* o, float* lse, char* ws,
@@ -768,7 +792,7 @@ cudaError_t run_tc(const Shape& s, const Geom& g, const CUtensorMap& mk, const C
       mk, mv, (const __nv_bfloat16*)q, (const int4*)(ws + L.tiles), (const int*)(ws + L.n_tiles),
       (const int*)(ws + L.entries), (__nv_bfloat16*)(ws + L.po), (float*)(ws + L.plse), err, g);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  const int64_t rows = s.batch * s.hkv * s.seq;
+  const int64_t rows = s.batch * s.hkv * g.slab;
   const int rpc = 128 / (G * 8);
   merge_partials_kernel<G><<<(unsigned)((rows + rpc - 1) / rpc), 128, 0, st>>>(
       idx, (const __nv_bfloat16*)(ws + L.po), (const float*)(ws + L.plse), (__nv_bfloat16*)o,
@@ -793,22 +817,30 @@ bool tc_attn_supported(const Shape& s) {
   return true;
 }
 
-size_t tc_attn_ws_bytes(const Shape& s) { return layout_for(s).total; }
+size_t tc_attn_ws_bytes(const Shape& s) {
+  return layout_for(s, slab_for(s, kSlabBudget)).total;
+}
+size_t tc_attn_ws_min_bytes(const Shape& s) { return layout_for(s, min_slab(s)).total; }
+int64_t tc_attn_slab_tokens(const Shape& s, size_t ws_body_bytes) {
+  const int64_t slab = slab_for(s, ws_body_bytes);
+  return layout_for(s, slab).total <= ws_body_bytes ? (slab < s.seq ? slab : s.seq) : 0;
+}
 
 cudaError_t launch_attn_prefill_tc(const Shape& s, const void* q, const void* k, const void* v,
                                    const int32_t* idx, void* o, float* lse, void* ws_body,
-                                   int* err, cudaStream_t st) {
-  const Geom g = make_geom(s);
-  const WsLayout L = layout_for(s);
+                                   size_t ws_body_bytes, int* err, cudaStream_t st) {
+  Geom g = make_geom(s);
+  const int64_t slab = slab_for(s, ws_body_bytes);
+  const WsLayout L = layout_for(s, slab);
+  if (L.total > ws_body_bytes) return cudaErrorInvalidValue;
+  g.slab = slab;
   char* ws = reinterpret_cast<char*>(ws_body);
   CUtensorMap mk, mv;
   if (!make_bf16_2d_map(&mk, k, s.batch * s.seq, s.hkv * kD, 128) ||
       !make_bf16_2d_map(&mv, v, s.batch * s.seq, s.hkv * kD, 128))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaMemsetAsync(ws + L.counts, 0, g.nseg * 4, st);
-  if (e != cudaSuccess) return e;
-  const int64_t n_sel = s.batch * s.hkv * s.seq * s.topk;
   const size_t hsmem = (size_t)g.nb * g.nsub * sizeof(int);
+  cudaError_t e;
   if ((e = cudaFuncSetAttribute(invert_hist_kernel<false>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hsmem)) !=
           cudaSuccess ||
@@ -816,26 +848,36 @@ cudaError_t launch_attn_prefill_tc(const Shape& s, const void* q, const void* k,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hsmem)) !=
           cudaSuccess)
     return e;
-  const dim3 hgrid((unsigned)((s.seq + kInvTokens - 1) / kInvTokens), (unsigned)(s.batch * s.hkv));
-  invert_hist_kernel<false><<<hgrid, kInvThreads, hsmem, st>>>(
-      idx, (int*)(ws + L.counts), nullptr, nullptr, err, g);
-  invert_scan_kernel<<<1, 1024, 0, st>>>((const int*)(ws + L.counts), (int*)(ws + L.seg_off),
-                                         (int*)(ws + L.cursor), (int*)(ws + L.tile_off),
-                                         (int*)(ws + L.n_tiles), g.nseg, g.tpt);
-  invert_hist_kernel<true><<<hgrid, kInvThreads, hsmem, st>>>(
-      idx, nullptr, (int*)(ws + L.cursor), (int*)(ws + L.entries), err, g);
-  const int64_t n_tiles_max = n_sel * g.nsub / g.tpt + g.nseg + 1;
-  tile_table_kernel<<<(unsigned)((n_tiles_max + 255) / 256), 256, 0, st>>>(
-      (const int*)(ws + L.counts), (const int*)(ws + L.seg_off), (const int*)(ws + L.tile_off),
-      (const int*)(ws + L.n_tiles), (int4*)(ws + L.tiles), g.nseg, g.tpt,
-      (int64_t)g.nb * g.nsub);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  switch (g.G) {
-    case 1: return run_tc<1>(s, g, mk, mv, q, idx, o, lse, ws, L, err, st);
-    case 2: return run_tc<2>(s, g, mk, mv, q, idx, o, lse, ws, L, err, st);
-    case 4: return run_tc<4>(s, g, mk, mv, q, idx, o, lse, ws, L, err, st);
-    default: return run_tc<8>(s, g, mk, mv, q, idx, o, lse, ws, L, err, st);
+  // one pass per token slab: invert its selections, attend its tiles, merge its rows
+  for (int64_t t0 = 0; t0 < s.seq; t0 += slab) {
+    g.t_base = t0;
+    g.t_end = t0 + slab < s.seq ? t0 + slab : s.seq;
+    if ((e = cudaMemsetAsync(ws + L.counts, 0, g.nseg * 4, st)) != cudaSuccess) return e;
+    const int64_t n_sel = s.batch * s.hkv * (g.t_end - t0) * s.topk;
+    const dim3 hgrid((unsigned)((g.t_end - t0 + kInvTokens - 1) / kInvTokens),
+                     (unsigned)(s.batch * s.hkv));
+    invert_hist_kernel<false><<<hgrid, kInvThreads, hsmem, st>>>(
+        idx, (int*)(ws + L.counts), nullptr, nullptr, err, g);
+    invert_scan_kernel<<<1, 1024, 0, st>>>((const int*)(ws + L.counts), (int*)(ws + L.seg_off),
+                                           (int*)(ws + L.cursor), (int*)(ws + L.tile_off),
+                                           (int*)(ws + L.n_tiles), g.nseg, g.tpt);
+    invert_hist_kernel<true><<<hgrid, kInvThreads, hsmem, st>>>(
+        idx, nullptr, (int*)(ws + L.cursor), (int*)(ws + L.entries), err, g);
+    const int64_t n_tiles_max = n_sel * g.nsub / g.tpt + g.nseg + 1;
+    tile_table_kernel<<<(unsigned)((n_tiles_max + 255) / 256), 256, 0, st>>>(
+        (const int*)(ws + L.counts), (const int*)(ws + L.seg_off), (const int*)(ws + L.tile_off),
+        (const int*)(ws + L.n_tiles), (int4*)(ws + L.tiles), g.nseg, g.tpt,
+        (int64_t)g.nb * g.nsub);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    switch (g.G) {
+      case 1: e = run_tc<1>(s, g, mk, mv, q, idx, o, lse, ws, L, err, st); break;
+      case 2: e = run_tc<2>(s, g, mk, mv, q, idx, o, lse, ws, L, err, st); break;
+      case 4: e = run_tc<4>(s, g, mk, mv, q, idx, o, lse, ws, L, err, st); break;
+      default: e = run_tc<8>(s, g, mk, mv, q, idx, o, lse, ws, L, err, st); break;
+    }
+    if (e != cudaSuccess) return e;
   }
+  return cudaSuccess;
 }
 
 }  // namespace msa

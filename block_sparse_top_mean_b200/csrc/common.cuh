@@ -160,9 +160,12 @@ cudaError_t launch_topk_prefill_tc(const Shape& s, const void* q, const float* k
 
 // Key-centric tensor-core attention (bf16, d = 128); see attn_tc.cu.
 bool tc_attn_supported(const Shape& s);
-size_t tc_attn_ws_bytes(const Shape& s);
+size_t tc_attn_ws_bytes(const Shape& s);       // recommended (whole sequence or a 32 GiB slab)
+size_t tc_attn_ws_min_bytes(const Shape& s);   // one 2048-token slab
+int64_t tc_attn_slab_tokens(const Shape& s, size_t ws_body_bytes);   // 0: too small
+// Runs in token slabs sized to the ws_body_bytes given (>= tc_attn_ws_min_bytes).
 cudaError_t launch_attn_prefill_tc(const Shape& s, const void* q, const void* k, const void* v,
                                    const int32_t* idx, void* o, float* lse, void* ws_body,
-                                   int* err, cudaStream_t st);
+                                   size_t ws_body_bytes, int* err, cudaStream_t st);
 
 }  // namespace msa

@@ -66,16 +66,28 @@ size_t decode_sel_ws(const Shape& s, int64_t n_query) {
   return n;
 }
 
+// Attention scratch: the recommended size, or the smallest the tensor-core path accepts
+// (it then walks the sequence in more, smaller token slabs).
+size_t attn_ws(const Shape& s, bool minimum) {
+  if (!msa::tc_attn_supported(s)) return 0;
+  return round256(minimum ? msa::tc_attn_ws_min_bytes(s) : msa::tc_attn_ws_bytes(s));
+}
+
+// Bytes of the prefill workspace in front of the attention scratch.
+size_t prefill_fixed_ws(const Shape& s) {
+  return round256(kbar_bytes(s)) + 2 * round256(kbar_split_bytes(s)) + topk_flag_ws(s);
+}
+
 size_t ws_bytes_for(const Shape& s, int op, int64_t n_query) {
   switch (op) {
     case MSA_OP_TOPK_SELECT:
       return msa::kWsHeader + topk_flag_ws(s);
     case MSA_OP_SPARSE_ATTN:
-      return msa::kWsHeader + (msa::tc_attn_supported(s) ? round256(msa::tc_attn_ws_bytes(s)) : 0);
+    case MSA_OP_SPARSE_ATTN_MIN:
+      return msa::kWsHeader + attn_ws(s, op == MSA_OP_SPARSE_ATTN_MIN);
     case MSA_OP_PREFILL:
-      return msa::kWsHeader + round256(kbar_bytes(s)) + 2 * round256(kbar_split_bytes(s)) +
-             topk_flag_ws(s) +
-             (msa::tc_attn_supported(s) ? round256(msa::tc_attn_ws_bytes(s)) : 0);
+    case MSA_OP_PREFILL_MIN:
+      return msa::kWsHeader + prefill_fixed_ws(s) + attn_ws(s, op == MSA_OP_PREFILL_MIN);
     case MSA_OP_DECODE:
       return msa::kWsHeader + round256(decode_sel_ws(s, n_query)) +
              round256(msa::decode_attn_ws_bytes(s, n_query));
@@ -84,7 +96,10 @@ size_t ws_bytes_for(const Shape& s, int op, int64_t n_query) {
   }
 }
 
+// The attention-bearing calls accept anything from the minimum size up.
 msa_status check_ws(const Shape& s, int op, int64_t n_query, const void* ws, size_t ws_bytes) {
+  if (op == MSA_OP_SPARSE_ATTN) op = MSA_OP_SPARSE_ATTN_MIN;
+  if (op == MSA_OP_PREFILL) op = MSA_OP_PREFILL_MIN;
   const size_t need = ws_bytes_for(s, op, n_query);
   if (ws == nullptr || ws_bytes < need || !aligned256(ws)) return MSA_ERR_WORKSPACE;
   return MSA_OK;
@@ -105,10 +120,10 @@ cudaError_t launch_selection(const Shape& s, const void* q, const float* kbar,
 // bf16 with d = 128 and 128-multiple blocks runs on the tensor cores (key-centric tiles);
 // everything else on the query-centric SIMT kernel.
 cudaError_t launch_attention(const Shape& s, const void* q, const void* k, const void* v,
-                             const int32_t* idx, void* o, float* lse, char* scratch, int* err,
-                             cudaStream_t st) {
+                             const int32_t* idx, void* o, float* lse, char* scratch,
+                             size_t scratch_bytes, int* err, cudaStream_t st) {
   if (msa::tc_attn_supported(s))
-    return msa::launch_attn_prefill_tc(s, q, k, v, idx, o, lse, scratch, err, st);
+    return msa::launch_attn_prefill_tc(s, q, k, v, idx, o, lse, scratch, scratch_bytes, err, st);
   return msa::launch_attn_prefill_rows(s, q, k, v, idx, o, lse, err, st);
 }
 
@@ -136,6 +151,17 @@ size_t msa_workspace_bytes(const msa_params* p, int32_t op, int64_t n_query) {
   if (check_params(p, op == MSA_OP_DECODE, &s) != MSA_OK) return 0;
   if (op == MSA_OP_DECODE && n_query < 0) return 0;
   return ws_bytes_for(s, op, n_query);
+}
+
+int64_t msa_attn_slab_tokens(const msa_params* p, int32_t op, size_t ws_bytes) {
+  Shape s;
+  if (check_params(p, false, &s) != MSA_OK) return -1;
+  if (op != MSA_OP_SPARSE_ATTN && op != MSA_OP_PREFILL) return -1;
+  if (ws_bytes < ws_bytes_for(s, op == MSA_OP_PREFILL ? MSA_OP_PREFILL_MIN : MSA_OP_SPARSE_ATTN_MIN, 0))
+    return 0;
+  if (!msa::tc_attn_supported(s) || s.seq == 0) return s.seq;
+  const size_t fixed = msa::kWsHeader + (op == MSA_OP_PREFILL ? prefill_fixed_ws(s) : 0);
+  return msa::tc_attn_slab_tokens(s, ws_bytes - fixed);
 }
 
 msa_status msa_pool_keys(const msa_params* p, const void* k, float* kbar, void* kbar_hi,
@@ -193,7 +219,8 @@ msa_status msa_sparse_attn_fwd(const msa_params* p, const void* q, const void* k
     return MSA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return MSA_ERR_INVALID_ARG;
   if ((st = check_ws(s, MSA_OP_SPARSE_ATTN, 0, ws, ws_bytes)) != MSA_OK) return st;
-  return cuda_status(launch_attention(s, q, k, v, idx, o, lse, ws_body(ws), err_word(ws),
+  return cuda_status(launch_attention(s, q, k, v, idx, o, lse, ws_body(ws),
+                                      ws_bytes - msa::kWsHeader, err_word(ws),
                                       (cudaStream_t)stream));
 }
 
@@ -223,7 +250,9 @@ msa_status msa_prefill_fwd(const msa_params* p, const void* q, const void* k, co
   off += topk_flag_ws(s);
   cudaError_t e = msa::launch_pool_keys(s, k, kbar, hi, lo, s.batch, cs);
   if (e == cudaSuccess) e = launch_selection(s, q, kbar, hi, lo, idx, flags, err_word(ws), cs);
-  if (e == cudaSuccess) e = launch_attention(s, q, k, v, idx, o, lse, body + off, err_word(ws), cs);
+  if (e == cudaSuccess)
+    e = launch_attention(s, q, k, v, idx, o, lse, body + off, ws_bytes - msa::kWsHeader - off,
+                         err_word(ws), cs);
   return cuda_status(e);
 }
 

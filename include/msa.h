@@ -88,7 +88,9 @@ typedef enum {
   MSA_OP_TOPK_SELECT = 0,
   MSA_OP_SPARSE_ATTN = 1,
   MSA_OP_PREFILL = 2,
-  MSA_OP_DECODE = 3
+  MSA_OP_DECODE = 3,
+  MSA_OP_SPARSE_ATTN_MIN = 4, /* smallest workspace msa_sparse_attn_fwd accepts */
+  MSA_OP_PREFILL_MIN = 5      /* smallest workspace msa_prefill_fwd accepts */
 } msa_op;
 
 /* Device error bits (msa_read_device_error). */
@@ -119,6 +121,12 @@ MSA_API const char* msa_status_string(msa_status status);
  * word; the rest is scratch whose content between calls is unspecified. */
 MSA_API size_t msa_workspace_bytes(const msa_params* p, int32_t op, int64_t n_query);
 
+/* Tokens per slab that msa_sparse_attn_fwd (op MSA_OP_SPARSE_ATTN) or msa_prefill_fwd
+ * (op MSA_OP_PREFILL) processes at a time when given ws_bytes of workspace: p->seq for one
+ * pass, 0 when ws_bytes is below the minimum, -1 for invalid params or op.  Each slab
+ * is one more round of the attention's six kernel launches.  Host-only. */
+MSA_API int64_t msa_attn_slab_tokens(const msa_params* p, int32_t op, size_t ws_bytes);
+
 /* Step 1, block pooling ([MSA-DE] routing keys; [MoBA] KV blocks):
  *   kbar[b,j,g,:] = (1/n_j) * sum_{t in block j} k[b,t,g,:],  n_j = tokens in block j.
  * kbar (fp32) is required; kbar_hi / kbar_lo (bf16 split planes) may each be NULL.
@@ -146,14 +154,19 @@ MSA_API msa_status msa_topk_select(const msa_params* p, const void* q, const flo
  *   o[b,t,h,:] = sum_{p in U} softmax_p(scale * q[b,t,h,:] . k[b,p,g,:]) v[b,p,g,:],
  *   U = keys of the blocks in idx[b,g,t,:] (entries -1 skipped), keeping p <= t.
  * lse may be NULL.  Entries outside [-1, nb) or after the own block set
- * MSA_DEVERR_IDX_RANGE and are skipped.  ws: msa_workspace_bytes(p, MSA_OP_SPARSE_ATTN). */
+ * MSA_DEVERR_IDX_RANGE and are skipped.  ws: msa_workspace_bytes(p, MSA_OP_SPARSE_ATTN) is
+ * the recommended size (the whole sequence in one pass, or token slabs of about 32 GiB of
+ * partials); any size from msa_workspace_bytes(p, MSA_OP_SPARSE_ATTN_MIN) up is accepted,
+ * and the bf16 d = 128 path then processes the sequence in token slabs (multiples of 2048
+ * tokens) that fit ws_bytes: same results, more launches. */
 MSA_API msa_status msa_sparse_attn_fwd(const msa_params* p, const void* q, const void* k, const void* v,
                                const int32_t* idx, void* o, float* lse, void* ws,
                                size_t ws_bytes, msa_stream_t stream);
 
 /* Whole causal prefill: msa_pool_keys -> msa_topk_select -> msa_sparse_attn_fwd, with the
  * pooled keys kept in the workspace.  idx is written (caller-owned, [b,hkv,S,topk]);
- * lse may be NULL.  ws: msa_workspace_bytes(p, MSA_OP_PREFILL, 0). */
+ * lse may be NULL.  ws: msa_workspace_bytes(p, MSA_OP_PREFILL, 0) recommended, at least
+ * msa_workspace_bytes(p, MSA_OP_PREFILL_MIN, 0) (slabbed attention, as above). */
 MSA_API msa_status msa_prefill_fwd(const msa_params* p, const void* q, const void* k, const void* v,
                            int32_t* idx, void* o, float* lse, void* ws, size_t ws_bytes,
                            msa_stream_t stream);

@@ -101,6 +101,39 @@ def test_workspace_checks(lib):
     assert lib.msa_workspace_bytes(ctypes.byref(p), 99, 0) == 0
 
 
+def test_attention_workspace_bounded_by_token_slabs(lib):
+    """The key-centric attention keeps one partial per (token, group, selected segment);
+    at 1M tokens that is ~140 GB, so the library walks the sequence in token slabs:
+    the recommended size stays near 32 GiB and the minimum is one 2048-token slab."""
+    def ws(op, **kw):
+        return lib.msa_workspace_bytes(ctypes.byref(_p(**kw)), op, 0)
+    big = dict(seq=1_048_576, hq=32, hkv=8, block=256, topk=16)
+    rec, mn = ws(_lib.OP_SPARSE_ATTN, **big), ws(_lib.OP_SPARSE_ATTN_MIN, **big)
+    assert 16 << 30 < rec <= (33 << 30)
+    assert 0 < mn < (1 << 30) and mn < rec
+    # prefill adds the same fixed part (pooled keys, split planes, flags) to both
+    frec, fmn = ws(_lib.OP_PREFILL, **big), ws(_lib.OP_PREFILL_MIN, **big)
+    assert frec - rec == fmn - mn > 0
+    # short sequences: one slab, minimum == recommended
+    assert ws(_lib.OP_SPARSE_ATTN, seq=1500) == ws(_lib.OP_SPARSE_ATTN_MIN, seq=1500)
+    # the slab plan: evened-out slabs of 2048-token multiples, one pass when it all fits
+    p = _p(**big)
+    slab = lib.msa_attn_slab_tokens(ctypes.byref(p), _lib.OP_SPARSE_ATTN, rec)
+    assert slab % 2048 == 0 and 1 < -(-big["seq"] // slab) <= 8
+    assert lib.msa_attn_slab_tokens(ctypes.byref(p), _lib.OP_PREFILL, frec) == slab
+    assert lib.msa_attn_slab_tokens(ctypes.byref(p), _lib.OP_SPARSE_ATTN, mn) == 2048
+    assert lib.msa_attn_slab_tokens(ctypes.byref(p), _lib.OP_SPARSE_ATTN, mn - 1) == 0
+    assert lib.msa_attn_slab_tokens(ctypes.byref(p), _lib.OP_SPARSE_ATTN, 1 << 40) == big["seq"]
+    assert lib.msa_attn_slab_tokens(ctypes.byref(p), _lib.OP_DECODE, 1 << 40) == -1
+    # the minimum is the floor the calls accept
+    st = lib.msa_sparse_attn_fwd(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE,
+                                 mn - 1, None)
+    assert st == _lib.MSA_ERR_WORKSPACE
+    st = lib.msa_prefill_fwd(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE,
+                             fmn - 1, None)
+    assert st == _lib.MSA_ERR_WORKSPACE
+
+
 def test_empty_inputs_are_noops(lib):
     for kw in (dict(seq=0), dict(batch=0)):
         p = _p(**kw)

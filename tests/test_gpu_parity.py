@@ -203,6 +203,31 @@ def test_prefill_is_deterministic(msa):
         assert torch.equal(x, y)
 
 
+@pytest.mark.parametrize("w", [
+    mi.Workload("bf16_slabs_b128", "prefill", 2, 5000, 8, 2, 128, 128, 8, "bf16"),
+    mi.Workload("bf16_slabs_b256_g4", "prefill", 1, 6500, 16, 4, 128, 256, 6, "bf16"),
+], ids=lambda w: w.name)
+def test_attention_in_token_slabs(msa, w):
+    """With the minimum workspace the tensor-core attention walks the sequence in
+    2048-token slabs (the last one ragged); every token's result is bitwise the one-pass
+    result, and both match the oracle."""
+    q, k, v = _inputs(w)
+    o1, lse1, idx = msa.prefill_fwd(q, k, v, w.block, w.topk, w.scale)
+    p = msa._prefill_params(q, k, w.block, w.topk, w.scale)
+    ws_min = msa.workspace(p, msa.OP_PREFILL_MIN, device=q.device)
+    assert ws_min.numel() < msa.workspace(p, msa.OP_PREFILL, device=q.device).numel()
+    o2, lse2, idx2 = msa.prefill_fwd(q, k, v, w.block, w.topk, w.scale, ws=ws_min)
+    a_ws = msa.workspace(p, msa.OP_SPARSE_ATTN_MIN, device=q.device)
+    o3, lse3 = msa.sparse_attn_fwd(q, k, v, idx, w.block, w.scale, ws=a_ws)
+    torch.cuda.synchronize()
+    assert torch.equal(idx, idx2)
+    for o, lse in [(o2, lse2), (o3, lse3)]:
+        assert torch.equal(o, o1)
+        assert torch.equal(lse, lse1)
+    check_prefill(q, k, v, w.block, w.topk, w.scale, idx2, o2, lse2)
+    assert msa.read_device_error(ws_min) == 0
+
+
 DECODE_SMALL = [
     mi.Workload("decode_small_bf16", "decode", 1, 50_000, 32, 8, 128, 64, 32, "bf16", n_query=8),
     mi.Workload("decode_small_f32", "decode", 1, 9_000, 8, 2, 64, 64, 8, "f32", n_query=70),
