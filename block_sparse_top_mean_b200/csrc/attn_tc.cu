@@ -44,13 +44,6 @@ struct Geom {
   float scale_log2;
 };
 
-__device__ __forceinline__ bool sub_has_keys(int64_t j, int64_t own, int64_t t, int sub,
-                                             const Geom& g) {
-  const int64_t lo = j * g.block + (int64_t)sub * kSegKeys;
-  if ((int64_t)sub * kSegKeys >= g.block || lo >= g.S) return false;
-  return j < own || lo <= t;
-}
-
 // ------------------------------------------------------------------ index inversion
 // Counting and filling run per CTA over a range of kInvTokens tokens of one (sequence,
 // group): entries are first counted in a shared-memory histogram over that group's
@@ -188,10 +181,9 @@ struct __align__(8) Bars {
 // chunks, 128 KB of K/V) get 3 stages and 128-key blocks 4 (both fit 227 KB).
 __host__ __device__ constexpr int q_stages(int nch) { return nch == 1 ? 4 : 3; }
 
-constexpr int kThreads3 = 384;       // WG0 warps 0-3, WG1 warps 4-7, issuer 8, gather 9-11
+constexpr int kThreads3 = 320;       // WG0 warps 0-3, WG1 warps 4-7, issuer 8, gather 9
 constexpr int kIssuerWarp = 8;
-constexpr int kGatherWarp0 = 9;
-constexpr int kGatherThreads = 96;
+constexpr int kGatherWarp = 9;
 constexpr float kRescaleLog2 = 8.f;  // chunk-1 max may exceed the reference by 2^8
 
 __device__ __forceinline__ float fast_exp2(float x) {
@@ -215,19 +207,59 @@ __device__ __forceinline__ TileId decode_tile(const int4& tl, const Geom& g) {
   return d;
 }
 
-// 2^x on the FMA pipe, for part of the softmax exponentials: x = n + f with n = floor(x),
-// 2^f from a degree-4 polynomial fitted here to minimise the relative error on [0, 1)
-// (max 2.6e-6), and 2^n added to the exponent field.  Inputs below -126 return 2^-126.
-__device__ __forceinline__ float poly_exp2(float x) {
-  x = fmaxf(x, -126.f);
-  const float n = floorf(x);
-  const float f = x - n;
-  float p = fmaf(0.013534167241300929f, f, 0.052011461907036594f);
-  p = fmaf(p, f, 0.24144275612530167f);
-  p = fmaf(p, f, 0.6930038346109176f);
-  p = fmaf(p, f, 1.0000025933668424f);
-  return __int_as_float(__float_as_int(p) + ((int)n << 23));
+// Packed two-lane fp32 arithmetic (sm_100: one instruction for both lanes).
+__device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, float b0, float b1,
+                                      float c0, float c1) {
+  asm("{\n.reg .b64 a, b, c, d;\nmov.b64 a, {%2, %3};\nmov.b64 b, {%4, %5};\n"
+      "mov.b64 c, {%6, %7};\nfma.rn.f32x2 d, a, b, c;\nmov.b64 {%0, %1}, d;\n}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
 }
+__device__ __forceinline__ void fadd2(float& d0, float& d1, float a0, float a1, float b0,
+                                      float b1) {
+  asm("{\n.reg .b64 a, b, d;\nmov.b64 a, {%2, %3};\nmov.b64 b, {%4, %5};\n"
+      "add.rn.f32x2 d, a, b;\nmov.b64 {%0, %1}, d;\n}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+__device__ __forceinline__ void fmul2(float& d0, float& d1, float a0, float a1, float b0,
+                                      float b1) {
+  asm("{\n.reg .b64 a, b, d;\nmov.b64 a, {%2, %3};\nmov.b64 b, {%4, %5};\n"
+      "mul.rn.f32x2 d, a, b;\nmov.b64 {%0, %1}, d;\n}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x for two lanes on the FMA pipe: adding 1.5 * 2^23 rounds x to the nearest integer n
+// and leaves n in the low mantissa bits; f = x - n lies in [-1/2, 1/2]; 2^f comes from a
+// cubic fitted here for minimal relative error on that interval (7.5e-5, below the bf16
+// rounding P goes through); n is then added to the exponent field.  x is clamped to -126.
+__device__ __forceinline__ void poly_exp2x2(float x0, float x1, float& p0, float& p1) {
+  constexpr float kShift = 12582912.f;            // 1.5 * 2^23
+  x0 = fmaxf(x0, -126.f);
+  x1 = fmaxf(x1, -126.f);
+  float t0, t1, n0, n1, f0, f1;
+  fadd2(t0, t1, x0, x1, kShift, kShift);
+  fadd2(n0, n1, t0, t1, -kShift, -kShift);        // exact: n as a float
+  ffma2(f0, f1, n0, n1, -1.f, -1.f, x0, x1);      // exact: x - n
+  float q0, q1;
+  ffma2(q0, q1, 0.0551716573536396f, 0.0551716573536396f, f0, f1, 0.2426111400127411f,
+        0.2426111400127411f);
+  ffma2(q0, q1, q0, q1, f0, f1, 0.6932609677314758f, 0.6932609677314758f);
+  ffma2(q0, q1, q0, q1, f0, f1, 0.9999280571937561f, 0.9999280571937561f);
+  // the low 9 bits of t's pattern are n's; shifted by 23 only n << 23 remains
+  p0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
+  p1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
+}
+
+#ifndef MSA_POLY_PAIRS
+#define MSA_POLY_PAIRS 0x44                       // pairs (of 8) whose exponentials use the FMA pipe
+#endif
 
 // Phase parity of the per-chunk barriers for chunk c of this CTA's tile n.
 __device__ __forceinline__ uint32_t chunk_phase(int n, int c, int nch) {
@@ -237,7 +269,7 @@ __device__ __forceinline__ uint32_t chunk_phase(int n, int c, int nch) {
 template <int G>
 __global__ void __launch_bounds__(kThreads3, 1)
 attn_tiles_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                  const __nv_bfloat16* __restrict__ q, const int4* __restrict__ tiles,
+                  const __grid_constant__ CUtensorMap tmQ, const int4* __restrict__ tiles,
                   const int* __restrict__ n_tiles_p, const int* __restrict__ entries,
                   __nv_bfloat16* __restrict__ po, float* __restrict__ plse, int* err, Geom g) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -248,8 +280,7 @@ attn_tiles_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
   unsigned char* Qs = base;                                   // nqs stages x 32 KB
   unsigned char* Ks = base + nqs * 2 * kTileBytes;            // nch x 2 halves x 16 KB
   unsigned char* Vs = Ks + nch * 2 * kTileBytes;
-  int* tok_all = reinterpret_cast<int*>(Vs + nch * 2 * kTileBytes);   // [nqs][kRowsT]
-  Bars* bars = reinterpret_cast<Bars*>(tok_all + nqs * kRowsT);
+  Bars* bars = reinterpret_cast<Bars*>(Vs + nch * 2 * kTileBytes);
 
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   const int n_tiles = *n_tiles_p;
@@ -260,7 +291,7 @@ attn_tiles_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
 
   if (tid == 0) {
     for (int s = 0; s < nqs; ++s) {
-      mbar_init(&bars->q_full[s], kGatherThreads);
+      mbar_init(&bars->q_full[s], 1);
       mbar_init(&bars->q_empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
@@ -380,80 +411,66 @@ attn_tiles_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
       }
       if (!ok) fail();
     }
-  } else if (warp >= kGatherWarp0) {
+  } else if (warp == kGatherWarp) {
     // ---------------------------------------------------------------- Q gather
-    // Tile n's copies are issued before waiting for tile n-1's, so two gathers are in
-    // flight; the next tile's record and token ids are loaded while copies run.
-    const int gt = tid - kGatherWarp0 * 32;
-    constexpr int kPerThread = (kRowsT / G + kGatherThreads - 1) / kGatherThreads;
+    // Tensor-map copies: viewed as [b*S*hq, 128], a token's G query heads of group gg are
+    // G consecutive rows, so each (token, 64-dim half) is one box of G rows, landing at
+    // tile rows [G*i, G*i+G) in the 128-byte-swizzled layout the MMA reads.  Each lane
+    // copies its own tokens; one arrive with the tile's byte count publishes the stage.
+    // Tile n+1's token ids and tile n+2's record are loaded while tile n's copies go out.
+    constexpr int kTok = kRowsT / G;                     // tokens per tile
+    constexpr int kPerLane = (kTok + 31) / 32;
+    if (lane == 0 && my_tiles > 0) prefetch_tmap(&tmQ);
     int4 tl_n = my_tiles > 0 ? tiles[tile_lo] : make_int4(0, 0, 0, 0);
-    int ent_n[kPerThread];
+    int4 tl_n1 = my_tiles > 1 ? tiles[tile_lo + 1] : make_int4(0, 0, 0, 0);
+    int ent_n[kPerLane];
 #pragma unroll
-    for (int u = 0; u < kPerThread; ++u) {
-      const int i = gt + u * kGatherThreads;
-      ent_n[u] = (my_tiles > 0 && i < kRowsT / G && i < tl_n.z) ? entries[tl_n.y + i] : -1;
+    for (int u = 0; u < kPerLane; ++u) {
+      const int i = lane + u * 32;
+      ent_n[u] = (my_tiles > 0 && i < kTok && i < tl_n.z) ? entries[tl_n.y + i] : -1;
     }
-    int pending = -1;                                    // tile whose copies are in flight
+    int issued = 0;                                      // tiles whose copies went out
     for (int n = 0; n < my_tiles; ++n) {
       const int st = n % nqs;
-      bool bad = *abort_flag != 0;
-      if (!bad && n >= nqs) {
-        const uint32_t par = ((n / nqs) - 1) & 1;
-        // Never block on a stage while holding an unpublished tile: its consumer may be
-        // what frees the stage (with two key chunks, QK of tile n-1 needs tile n-1's Q
-        // before tile n-2's stage is released).
-        if (pending >= 0 && !mbar_try_wait(&bars->q_empty[st], par)) {
-          cp_async_wait_all();
-          fence_proxy_async_smem();
-          mbar_arrive(&bars->q_full[pending % nqs]);
-          pending = -1;
-        }
-        if (!mbar_wait(&bars->q_empty[st], par)) {
-          fail();
-          bad = true;
-        }
+      if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+      if (n >= nqs && !mbar_wait_warp(&bars->q_empty[st], ((n / nqs) - 1) & 1)) {
+        if (lane == 0) fail();
+        break;
       }
       const int4 tl = tl_n;
-      int* tk = tok_all + st * kRowsT;
+      int ent[kPerLane];
+      int n_valid = 0;
 #pragma unroll
-      for (int u = 0; u < kPerThread; ++u) {
-        const int i = gt + u * kGatherThreads;
-        if (i < kRowsT / G) tk[i] = ent_n[u] >= 0 ? (ent_n[u] >> 6) : -1;
+      for (int u = 0; u < kPerLane; ++u) {
+        ent[u] = ent_n[u];
+        n_valid += __popc(__ballot_sync(0xffffffffu, ent[u] >= 0));
       }
-      // all gather threads leave together: the token list is complete, or all abort
-      if (bar_sync_or<1, kGatherThreads>(bad)) break;
-      if (n + 1 < my_tiles) {                            // prefetch the next tile's record
-        tl_n = tiles[tile_lo + n + 1];
+      if (n + 1 < my_tiles) {                            // tile n+1's token ids
 #pragma unroll
-        for (int u = 0; u < kPerThread; ++u) {
-          const int i = gt + u * kGatherThreads;
-          ent_n[u] = (i < kRowsT / G && i < tl_n.z) ? entries[tl_n.y + i] : -1;
+        for (int u = 0; u < kPerLane; ++u) {
+          const int i = lane + u * 32;
+          ent_n[u] = (i < kTok && i < tl_n1.z) ? entries[tl_n1.y + i] : -1;
         }
+        tl_n = tl_n1;
       }
-      const int64_t b = tl.w / g.hkv, gg = tl.w - b * g.hkv;
+      if (n + 2 < my_tiles) tl_n1 = tiles[tile_lo + n + 2];   // tile n+2's record
+      if (lane == 0) mbar_arrive_expect_tx(&bars->q_full[st], (uint32_t)(n_valid * G * kD * 2));
+      __syncwarp();
+      const int b = tl.w / g.hkv, gg = tl.w - b * g.hkv;
       unsigned char* qb = Qs + st * 2 * kTileBytes;
-      const __nv_bfloat16* qbase = q + (b * g.S * g.hq + gg * G) * kD;
-#pragma unroll 4
-      for (int i = gt; i < kRowsT * 16; i += kGatherThreads) {
-        const int r = i >> 4, c = i & 15;
-        const int t = tk[r / G];
-        const bool valid = t >= 0;
-        const __nv_bfloat16* src = qbase + ((int64_t)(valid ? t : 0) * g.hq + r % G) * kD + c * 8;
-        cp_async16(qb + (c >> 3) * kTileBytes + r * 128 + (((c & 7) ^ (r & 7)) << 4), src, valid);
+#pragma unroll
+      for (int u = 0; u < kPerLane; ++u) {
+        if (ent[u] < 0) continue;
+        const int i = lane + u * 32;
+        const int y = (int)(((int64_t)b * g.S + (ent[u] >> 6)) * g.hq + gg * G);
+        tma_load_2d(qb + i * G * 128, &tmQ, &bars->q_full[st], 0, y);
+        tma_load_2d(qb + kTileBytes + i * G * 128, &tmQ, &bars->q_full[st], 64, y);
       }
-      cp_async_commit();
-      if (pending >= 0) {                                // the previous tile's copies landed
-        cp_async_wait_group1();
-        fence_proxy_async_smem();
-        mbar_arrive(&bars->q_full[pending % nqs]);
-      }
-      pending = n;
+      issued = n + 1;
     }
-    if (pending >= 0) {
-      cp_async_wait_all();
-      fence_proxy_async_smem();
-      mbar_arrive(&bars->q_full[pending % nqs]);
-    }
+    // no copy may still be landing when the CTA exits (normally all were consumed)
+    for (int m = issued > nqs ? issued - nqs : 0; m < issued; ++m)
+      if (!mbar_wait_warp(&bars->q_full[m % nqs], (m / nqs) & 1)) break;
   } else {
     // ---------------------------------------------------------------- softmax + epilogue
     const int X = warp >> 2;                             // this warpgroup's tile parity
@@ -506,13 +523,23 @@ attn_tiles_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
           tmem_ld32(sX + hq2 * 64 + 32, sv[1]);
           tmem_ld_wait();
           float mx = -CUDART_INF_F;
+          if (full) {
+            // eight independent chains of three-input maxima
+            float m8[8];
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int qd = hq2 * 2 + u;
-            if (full) {
+            for (int i = 0; i < 8; ++i) {
+              const uint32_t* v = &sv[i >> 2][(i & 3) * 8];
+              float m = fmax3(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]));
+              m = fmax3(m, __uint_as_float(v[3]), __uint_as_float(v[4]));
+              m = fmax3(m, __uint_as_float(v[5]), __uint_as_float(v[6]));
+              m8[i] = fmaxf(m, __uint_as_float(v[7]));
+            }
+            mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]),
+                       fmaxf(m8[6], m8[7]));
+          } else {
 #pragma unroll
-              for (int k = 0; k < 32; ++k) mx = fmaxf(mx, __uint_as_float(sv[u][k]));
-            } else {
+            for (int u = 0; u < 2; ++u) {
+              const int qd = hq2 * 2 + u;
 #pragma unroll
               for (int k = 0; k < 32; ++k)
                 if (qd * 32 + k < lim) mx = fmaxf(mx, __uint_as_float(sv[u][k]));
@@ -563,22 +590,34 @@ attn_tiles_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
           }
           const float mb = mref > -CUDART_INF_F ? mref : 0.f;
           uint32_t pk[32];
+          // Two lanes per instruction.  The pairs MSA_POLY_PAIRS marks take their
+          // exponentials on the FMA pipe, the rest on the MUFU unit; columns past lim
+          // (ragged or causal rows) become 0.  The arithmetic of a column does not depend
+          // on whether other rows of the warp are ragged.
+          float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
 #pragma unroll
           for (int u = 0; u < 2; ++u)
 #pragma unroll
             for (int k = 0; k < 32; k += 2) {
-              const int kk = (hq2 * 2 + u) * 32 + k;
-              // one exponential in four on the FMA pipe, the rest on the MUFU unit
-              float p0 = fast_exp2(fmaf(__uint_as_float(sv[u][k]), c2, -mb));
-              const float x1 = fmaf(__uint_as_float(sv[u][k + 1]), c2, -mb);
-              float p1 = (k & 3) == 2 ? poly_exp2(x1) : fast_exp2(x1);
+              float x0, x1, p0, p1;
+              ffma2(x0, x1, __uint_as_float(sv[u][k]), __uint_as_float(sv[u][k + 1]), c2, c2,
+                    -mb, -mb);
+              if ((MSA_POLY_PAIRS >> ((k / 2) & 7)) & 1) {
+                poly_exp2x2(x0, x1, p0, p1);
+              } else {
+                p0 = fast_exp2(x0);
+                p1 = fast_exp2(x1);
+              }
               if (!full) {
+                const int kk = (hq2 * 2 + u) * 32 + k;
                 p0 = kk < lim ? p0 : 0.f;
                 p1 = kk + 1 < lim ? p1 : 0.f;
               }
-              sum += p0 + p1;
+              if (u == 0) fadd2(a0, a1, a0, a1, p0, p1);
+              else fadd2(b0, b1, b0, b1, p0, p1);
               pk[u * 16 + k / 2] = pack_bf16x2(p0, p1);
             }
+          sum += (a0 + a1) + (b0 + b1);
           // P of this half over S columns already consumed
           tmem_st32(sX + hq2 * 32, pk);
         }
@@ -607,9 +646,11 @@ attn_tiles_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
         for (int u = 0; u < 2; ++u) {
           uint32_t ob[16];
 #pragma unroll
-          for (int k = 0; k < 32; k += 2)
-            ob[k / 2] = pack_bf16x2(__uint_as_float(ov[u][k]) * inv,
-                                    __uint_as_float(ov[u][k + 1]) * inv);
+          for (int k = 0; k < 32; k += 2) {
+            float y0, y1;
+            fmul2(y0, y1, __uint_as_float(ov[u][k]), __uint_as_float(ov[u][k + 1]), inv, inv);
+            ob[k / 2] = pack_bf16x2(y0, y1);
+          }
           if (valid) {
             st_global_v8(dst + (q2 * 2 + u) * 32, ob);
             st_global_v8(dst + (q2 * 2 + u) * 32 + 16, ob + 8);
@@ -781,15 +822,15 @@ int64_t slab_for(const Shape& s, size_t bytes) {
 
 template <int G>
 cudaError_t run_tc(const Shape& s, const Geom& g, const CUtensorMap& mk, const CUtensorMap& mv,
-                   const void* q, const int32_t* idx, void* o, float* lse, char* ws,
+                   const CUtensorMap& mq, const int32_t* idx, void* o, float* lse, char* ws,
                    const WsLayout& L, int* err, cudaStream_t st) {
-  const size_t smem = 1024 + (size_t)q_stages(g.nch) * (2 * kTileBytes + kRowsT * 4) +
+  const size_t smem = 1024 + (size_t)q_stages(g.nch) * 2 * kTileBytes +
                       (size_t)g.nch * 4 * kTileBytes + sizeof(Bars);
   cudaError_t e = cudaFuncSetAttribute(attn_tiles_kernel<G>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   attn_tiles_kernel<G><<<sm_count(), kThreads3, smem, st>>>(
-      mk, mv, (const __nv_bfloat16*)q, (const int4*)(ws + L.tiles), (const int*)(ws + L.n_tiles),
+      mk, mv, mq, (const int4*)(ws + L.tiles), (const int*)(ws + L.n_tiles),
       (const int*)(ws + L.entries), (__nv_bfloat16*)(ws + L.po), (float*)(ws + L.plse), err, g);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const int64_t rows = s.batch * s.hkv * g.slab;
@@ -811,6 +852,7 @@ bool tc_attn_supported(const Shape& s) {
   const int64_t nsub = (s.block + kSegKeys - 1) / kSegKeys;
   if (s.topk * nsub > 64) return false;                       // pslot fits 6 bits
   if (s.seq >= ((int64_t)1 << 25)) return false;              // token fits 25 bits
+  if (s.batch * s.seq * s.hq >= ((int64_t)1 << 31)) return false;   // q row fits a map coordinate
   if (s.batch * s.hkv * s.seq * s.topk * nsub >= ((int64_t)1 << 31)) return false;
   if (s.batch * s.seq >= ((int64_t)1 << 31)) return false;    // TMA row coordinate
   if (s.nb * nsub > 48 * 1024) return false;                  // inversion histogram in smem
@@ -835,9 +877,10 @@ cudaError_t launch_attn_prefill_tc(const Shape& s, const void* q, const void* k,
   if (L.total > ws_body_bytes) return cudaErrorInvalidValue;
   g.slab = slab;
   char* ws = reinterpret_cast<char*>(ws_body);
-  CUtensorMap mk, mv;
+  CUtensorMap mk, mv, mq;
   if (!make_bf16_2d_map(&mk, k, s.batch * s.seq, s.hkv * kD, 128) ||
-      !make_bf16_2d_map(&mv, v, s.batch * s.seq, s.hkv * kD, 128))
+      !make_bf16_2d_map(&mv, v, s.batch * s.seq, s.hkv * kD, 128) ||
+      !make_bf16_2d_map(&mq, q, s.batch * s.seq * s.hq, kD, g.G))   // G heads per box
     return cudaErrorInvalidValue;
   const size_t hsmem = (size_t)g.nb * g.nsub * sizeof(int);
   cudaError_t e;
@@ -870,10 +913,10 @@ cudaError_t launch_attn_prefill_tc(const Shape& s, const void* q, const void* k,
         (int64_t)g.nb * g.nsub);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     switch (g.G) {
-      case 1: e = run_tc<1>(s, g, mk, mv, q, idx, o, lse, ws, L, err, st); break;
-      case 2: e = run_tc<2>(s, g, mk, mv, q, idx, o, lse, ws, L, err, st); break;
-      case 4: e = run_tc<4>(s, g, mk, mv, q, idx, o, lse, ws, L, err, st); break;
-      default: e = run_tc<8>(s, g, mk, mv, q, idx, o, lse, ws, L, err, st); break;
+      case 1: e = run_tc<1>(s, g, mk, mv, mq, idx, o, lse, ws, L, err, st); break;
+      case 2: e = run_tc<2>(s, g, mk, mv, mq, idx, o, lse, ws, L, err, st); break;
+      case 4: e = run_tc<4>(s, g, mk, mv, mq, idx, o, lse, ws, L, err, st); break;
+      default: e = run_tc<8>(s, g, mk, mv, mq, idx, o, lse, ws, L, err, st); break;
     }
     if (e != cudaSuccess) return e;
   }
