@@ -161,14 +161,14 @@ __global__ void tile_table_kernel(const int* __restrict__ counts, const int* __r
 
 // ------------------------------------------------------------------ the tile kernel
 // Two tiles are in flight: tile n (the n-th of this CTA) uses TMEM set X = n & 1
-// (S_X at columns 128X, O_X at 256 + 128X), Q stage X and softmax warpgroup X.  The issuer
-// walks "rounds" of one or two consecutive tiles of the same block and issues, per key
-// chunk c, QK of both tiles then PV of both, so the tensor core works on one tile while
-// the other tile's warpgroup runs its softmax or epilogue.  MMAs of one thread run in
-// issue order, so a QK may reuse the TMEM of a P that an earlier PV reads; only thread
-// accesses of TMEM (softmax, epilogue) and TMA writes of K/V wait for MMA completion.  One O accumulator per tile:
-// chunk 1 reuses chunk 0's row max as its exponent reference unless the max grew by more
-// than 2^8, in which case that warp rescales O in TMEM after chunk 0's PV completed.
+// (S_X at columns 128X, O_X at 256 + 128X), Q stage n % stages and softmax warpgroup X.
+// The issuer runs the tiles of one block as two interleaved streams (even and odd tiles),
+// so the tensor core works on one tile while the other tile's warpgroup runs its softmax
+// or epilogue.  MMAs of one thread run in issue order, so a QK may reuse the TMEM of a P
+// that an earlier PV reads; only thread accesses of TMEM (softmax, epilogue) and TMA
+// writes of K/V wait for MMA completion.  One O accumulator per tile: chunk 1 reuses
+// chunk 0's row max as its exponent reference unless the max grew by more than 2^8, in
+// which case that warp rescales O in TMEM after chunk 0's PV completed.
 constexpr int kMaxQStages = 4;
 struct __align__(8) Bars {
   uint64_t q_full[kMaxQStages], q_empty[kMaxQStages];
@@ -366,21 +366,27 @@ attn_tiles_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
         umma_commit(&bars->pv_done[X]);
         return true;
       };
-      int n = 0;
-      int4 tl_a = tiles[tile_lo];                                   // tile n
-      int4 tl_b = my_tiles > 1 ? tiles[tile_lo + 1] : make_int4(-1, 0, 0, 0);   // tile n+1
+      // Runs of consecutive tiles share one segment's K/V.  Inside a run the tiles are
+      // two streams (tiles n, n+2, ... and n+1, n+3, ...), issued alternately one unit
+      // at a time, a unit being [wait P] PV(m, c) followed by the stream's next QK: chunk
+      // c+1 of m, or chunk 0 of m+2.  So one tile's MMAs run while the other tile's
+      // warpgroup does its softmax (the two are half a unit apart).
+      auto rec_x = [&](int m) -> int { return m < my_tiles ? tiles[tile_lo + m].x : -1; };
+      int n = 0, last_pv = -1;
       while (n < my_tiles && ok) {
         if (*abort_flag) break;
-        const int4 tl = tl_a;
-        const int pair = (n + 1 < my_tiles && tl_b.x == tl.x) ? 2 : 1;
-        // records of the next round's first two tiles, loaded ahead of time
-        const int nn = n + pair;
-        int4 nx_a = pair == 2 ? (nn < my_tiles ? tiles[tile_lo + nn] : make_int4(-1, 0, 0, 0))
-                              : tl_b;
-        const int4 nx_b = nn + 1 < my_tiles ? tiles[tile_lo + nn + 1] : make_int4(-1, 0, 0, 0);
+        const int4 tl = tiles[tile_lo + n];
+        // the stream whose turn it is (a) and the other (b): tile, next chunk, segment of
+        // the stream's next tile, still active
+        int ma = n, ca = 0, xa = rec_x(n + 2);
+        bool aa = true;
+        int mb = n + 1, cb = 0, xb = -1;
+        bool ab = rec_x(n + 1) == tl.x;
+        if (ab) xb = rec_x(n + 3);
         if (tl.x != prev_seg) {
           // every MMA of earlier tiles must be done before K/V are overwritten
-          if (n > 0 && !mbar_wait(&bars->pv_done[(n - 1) & 1], chunk_phase(n - 1, nch - 1, nch))) {
+          if (last_pv >= 0 &&
+              !mbar_wait(&bars->pv_done[last_pv & 1], chunk_phase(last_pv, nch - 1, nch))) {
             ok = false;
             break;
           }
@@ -389,25 +395,47 @@ attn_tiles_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
                                (int64_t)id.sub * kSegKeys);
           const int64_t gg = id.gg;
           mbar_arrive_expect_tx(&bars->kv_full, (uint32_t)(nch * 4 * kTileBytes));
-          for (int c = 0; c < nch; ++c)
+          for (int cc = 0; cc < nch; ++cc)
             for (int hf = 0; hf < 2; ++hf) {
               const int x = (int)(gg * kD + hf * 64);
-              tma_load_2d(Ks + (c * 2 + hf) * kTileBytes, &tmK, &bars->kv_full, x,
-                          y0 + c * kChunkKeys);
-              tma_load_2d(Vs + (c * 2 + hf) * kTileBytes, &tmV, &bars->kv_full, x,
-                          y0 + c * kChunkKeys);
+              tma_load_2d(Ks + (cc * 2 + hf) * kTileBytes, &tmK, &bars->kv_full, x,
+                          y0 + cc * kChunkKeys);
+              tma_load_2d(Vs + (cc * 2 + hf) * kTileBytes, &tmV, &bars->kv_full, x,
+                          y0 + cc * kChunkKeys);
             }
           if (!mbar_wait(&bars->kv_full, kvn & 1)) { ok = false; break; }
           ++kvn;
           prev_seg = tl.x;
         }
-        for (int c = 0; c < nch && ok; ++c) {
-          for (int i = 0; i < pair && ok; ++i) ok = issue_qk(n + i, c);
-          for (int i = 0; i < pair && ok; ++i) ok = issue_pv(n + i, c);
+        int end = ab ? n + 2 : n + 1;                    // one past the last tile started
+        ok = issue_qk(ma, 0);
+        if (ok && ab) ok = issue_qk(mb, 0);
+        while (ok && (aa || ab)) {
+          if (aa) {
+            if (*abort_flag) { ok = false; break; }
+            ok = issue_pv(ma, ca);
+            last_pv = ma;
+            if (!ok) break;
+            if (ca + 1 < nch) {
+              ++ca;
+              ok = issue_qk(ma, ca);
+            } else if (xa == tl.x) {                     // the stream's next tile, same K/V
+              ma += 2;
+              ca = 0;
+              xa = rec_x(ma + 2);
+              ok = issue_qk(ma, 0);
+              end = ma + 1 > end ? ma + 1 : end;
+            } else {
+              aa = false;
+            }
+          }
+          // the other stream's turn
+          int t_m = ma, t_c = ca, t_x = xa;
+          bool t_a = aa;
+          ma = mb; ca = cb; xa = xb; aa = ab;
+          mb = t_m; cb = t_c; xb = t_x; ab = t_a;
         }
-        n = nn;
-        tl_a = nx_a;
-        tl_b = nx_b;
+        n = end;
       }
       if (!ok) fail();
     }
