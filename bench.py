@@ -453,7 +453,7 @@ def run_ours(args, world, rank, local):
         "data": "synthetic",
         "config": {"workload": w.name, "batch_per_gpu": w.batch, "seq": w.seq, "hq": w.hq,
                    "hkv": w.hkv, "d": w.d, "block": w.block, "topk": w.topk,
-                   "l2": "inputs larger than L2 (Q alone 8 GiB), no flush",
+                   "l2": f"inputs larger than L2 (Q alone {w.batch * w.seq * w.hq * w.d * 2 / 2**30:.2f} GiB), no flush",
                    "workspace_gib": round(r.ws.numel() / 2**30, 2),
                    "attn_token_slabs": r.n_slabs,
                    "parallelism": f"{world} independent sequences, one per GPU"},
