@@ -5,7 +5,8 @@
 // of (token, slot) entries that selected it is built, and one tile = the G query heads
 // of 128/G such tokens (128 rows) against that block's keys.  K/V of a block are loaded
 // once per run of tiles into shared memory with TMA; the tile's query rows are gathered
-// with cp.async into the 128-byte-swizzled K-major layout the MMA reads.
+// with tensor-map boxes (G heads of one token each) into the 128-byte-swizzled K-major
+// layout the MMA reads.
 //
 // Per tile, per 128-key chunk c (a block of 256 keys is 2 chunks; longer blocks are
 // split into 256-key segments, each its own partial slot):
