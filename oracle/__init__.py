@@ -13,3 +13,7 @@ from .msa_oracle import (  # noqa: F401
     select_decode_row, attend_row, prefill_rows, decode_rows, PrefillRow, DecodeRow,
     rel_gap, prefill_keys_of, decode_keys_of,
 )
+from .msa_sharded import (  # noqa: F401
+    shard_blocks, local_candidates, merge_candidates, attend_owned, merge_partials,
+    decode_rows_sharded,
+)
