@@ -17,3 +17,4 @@ from .msa_sharded import (  # noqa: F401
     shard_blocks, local_candidates, merge_candidates, attend_owned, merge_partials,
     decode_rows_sharded,
 )
+from .msa_backward import attend_row_backward, prefill_backward  # noqa: F401
