@@ -40,7 +40,6 @@ constexpr int kCap = 32;                     // candidate buffer per row and col
 constexpr int kFlagTile = 64;                // tokens per fallback flag
 constexpr int kEpiThreads = 256;             // epilogue warps 0-7
 constexpr int kThreads = 288;                // warps 0-7 epilogue, 8 issuer
-constexpr uint32_t kHalf = 16384;            // 128 rows x 128 B (query planes)
 constexpr uint32_t kKHalf = 16384;           // 128 rows x 128 B (pooled-key planes)
 
 constexpr int kStages = 2;                   // pooled-key TMA ring depth
