@@ -21,7 +21,8 @@ from ._lib import (  # noqa: F401
 
 __all__ = [
     "params", "workspace", "pool_keys", "block_scores", "topk_select", "sparse_attn_fwd",
-    "prefill_fwd", "decode_fwd", "decode_fwd_static", "encode_bank", "decode_fwd_tiled", "decode_select_tiled", "decode_attn_tiled",
+    "prefill_fwd", "decode_fwd", "decode_fwd_static", "encode_bank", "decode_fwd_tiled",
+    "decode_select_tiled", "decode_attn_tiled", "attn_slab_tokens",
     "read_device_error",
     "clear_device_error", "version",
     "MsaError", "MsaParams",
