@@ -112,7 +112,7 @@ def _worker(rank, world, port, out):
 @pytest.mark.parametrize("world", [2, 3])
 def test_memory_parallel_protocol_equals_unsharded_decode(world):
     port = _free_port()
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
     mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
     res = dict(out)

@@ -36,7 +36,7 @@ def _worker(rank, world, port, out):
 
 def test_max_over_ranks_gloo():
     port = _free_port()
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
     mp.spawn(_worker, args=(2, port, out), nprocs=2, join=True)
     assert dict(out) == {0: 3.0, 1: 3.0}
