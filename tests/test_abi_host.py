@@ -134,6 +134,68 @@ def test_attention_workspace_bounded_by_token_slabs(lib):
     assert st == _lib.MSA_ERR_WORKSPACE
 
 
+def test_encoded_bank_sizes_closed_form(lib):
+    p = _p(seq=10_000_000, block=64, topk=32)
+    nb = -(-10_000_000 // 64)
+    assert lib.msa_bank_tiles_bytes(ctypes.byref(p), 0) == 8 * (-(-10_000_000 // 64)) * 16384
+    assert lib.msa_bank_tiles_bytes(ctypes.byref(p), 1) == 2 * 8 * (-(-nb // 128)) * 32768
+    assert lib.msa_bank_tiles_bytes(ctypes.byref(p), 2) == 0
+    assert lib.msa_bank_tiles_bytes(ctypes.byref(_p(seq=1000, hq=30)), 0) == 0
+
+
+def test_encoded_bank_entries_check_arguments_before_launch(lib):
+    p = _p(seq=1_000_000, block=64, topk=32)
+    pp = ctypes.byref(p)
+    odd = ctypes.c_void_p(4096 + 8)
+    # encoding: only the tensor-core decode shapes; each image needs its source
+    assert lib.msa_encode_bank(ctypes.byref(_p(seq=1000, block=64, dtype=_lib.MSA_F32)), FAKE,
+                               FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None) == \
+        _lib.MSA_ERR_UNSUPPORTED
+    assert lib.msa_encode_bank(pp, None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None) == \
+        _lib.MSA_ERR_INVALID_ARG
+    assert lib.msa_encode_bank(pp, FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, None) == \
+        _lib.MSA_ERR_INVALID_ARG
+    assert lib.msa_encode_bank(pp, odd, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None) == \
+        _lib.MSA_ERR_INVALID_ARG
+    assert lib.msa_encode_bank(ctypes.byref(_p(seq=0, block=64)), None, None, None, None,
+                               FAKE, FAKE, FAKE, None) == _lib.MSA_OK
+    need = lib.msa_workspace_bytes(pp, _lib.OP_DECODE, 64)
+    assert need > 256
+    sel, att, fwd = lib.msa_decode_select_tiled, lib.msa_decode_attn_tiled, \
+        lib.msa_decode_fwd_tiled
+    # no queries: nothing to do, nothing launched
+    assert sel(pp, 0, None, None, None, None, 0, None) == _lib.MSA_OK
+    assert att(pp, 0, None, None, None, None, None, None, None, 0, None) == _lib.MSA_OK
+    assert fwd(pp, 0, None, None, None, None, None, None, None, None, 0, None) == _lib.MSA_OK
+    assert sel(pp, -1, FAKE, FAKE, FAKE, FAKE, need, None) == _lib.MSA_ERR_INVALID_ARG
+    assert sel(pp, 64, None, FAKE, FAKE, FAKE, need, None) == _lib.MSA_ERR_INVALID_ARG
+    assert sel(pp, 64, FAKE, None, FAKE, FAKE, need, None) == _lib.MSA_ERR_INVALID_ARG
+    assert sel(pp, 64, FAKE, odd, FAKE, FAKE, need, None) == _lib.MSA_ERR_INVALID_ARG
+    assert sel(pp, 64, FAKE, FAKE, FAKE, FAKE, need - 1, None) == _lib.MSA_ERR_WORKSPACE
+    assert att(pp, 64, FAKE, FAKE, None, FAKE, FAKE, None, FAKE, need, None) == \
+        _lib.MSA_ERR_INVALID_ARG
+    assert att(pp, 64, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, need - 1, None) == \
+        _lib.MSA_ERR_WORKSPACE
+    # fp32 banks and d = 64 have no encoded form
+    for bad in (_p(seq=1000, block=64, dtype=_lib.MSA_F32), _p(seq=1000, block=64, d=64)):
+        assert sel(ctypes.byref(bad), 4, FAKE, FAKE, FAKE, FAKE, 1 << 30, None) == \
+            _lib.MSA_ERR_UNSUPPORTED
+
+
+def test_static_decode_rejects_before_touching_the_device(lib):
+    p = _p(seq=10_000_000, block=64, topk=32)
+    st = lib.msa_decode_fwd_static
+    assert st(None, 1, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, None) == \
+        _lib.MSA_ERR_INVALID_ARG
+    assert st(ctypes.byref(p), -1, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None,
+              None) == _lib.MSA_ERR_INVALID_ARG
+    assert st(ctypes.byref(p), 0, None, None, None, None, None, None, None, None, None,
+              None) == _lib.MSA_OK
+    # more queries than the fixed 32 MiB scratch can hold
+    assert st(ctypes.byref(p), 100_000, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None,
+              None) == _lib.MSA_ERR_WORKSPACE
+
+
 def test_empty_inputs_are_noops(lib):
     for kw in (dict(seq=0), dict(batch=0)):
         p = _p(**kw)
