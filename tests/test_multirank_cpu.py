@@ -42,11 +42,14 @@ def test_max_over_ranks_gloo():
     assert dict(out) == {0: 3.0, 1: 3.0}
 
 
-def test_reference_arm_under_torchrun_prints_one_line():
+@pytest.mark.parametrize("workload", [["prefill_tiny_s1k_f32"],
+                                      ["decode_bank10m_b64_k32", "--seq", "100000"]],
+                         ids=["prefill", "decode"])
+def test_reference_arm_under_torchrun_prints_one_line(workload):
     port = _free_port()
     cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node=2",
            "--master-addr", "127.0.0.1", "--master-port", str(port), "bench.py", "--impl",
-           "reference", "--workload", "prefill_tiny_s1k_f32", "--steps", "1", "--warmup", "3",
+           "reference", "--workload", *workload, "--steps", "1", "--warmup", "3",
            "--gpus", "2"]
     r = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=600,
                        env={**os.environ, "CUDA_VISIBLE_DEVICES": ""})
