@@ -68,6 +68,22 @@ def test_sharded_selection_with_exact_ties_across_shards():
         assert [r.idx for r in got] == [r.idx for r in ref] == [tied[:4]] * len(ref)
 
 
+def test_cut_margin_when_one_shard_holds_the_whole_top():
+    """All of the global top-(k+1) lie in one shard: the first left-out score (the margin
+    the parity gate reads) must still be the unsharded one."""
+    S, block, topk = 1024, 16, 8                    # 64 blocks, two shards of 32
+    Qd, K, V, _ = _bank(9, S, 4, 1, 16, block, 3)
+    rng = np.random.default_rng(10)
+    Qd = rng.integers(1, 4, Qd.shape).astype(np.float64)
+    kbar = rng.integers(-3, 4, (S // block, 1, 16)).astype(np.float64)
+    kbar[:topk + 1] = 10.0 + np.arange(topk + 1)[:, None, None]   # blocks 0..k, shard 0
+    ref = oracle.decode_rows(Qd, kbar, K, V, S, block, topk, 0.25)
+    got = oracle.decode_rows_sharded(Qd, kbar, K, V, S, block, topk, 0.25, 2)
+    for a, b in zip(ref, got):
+        assert a.idx == b.idx == list(range(1, topk + 1))
+        assert a.first_left == b.first_left and a.last_taken == b.last_taken
+
+
 def test_merge_partials_is_attention_over_the_union():
     """Attention over a key set split into disjoint parts (one empty) and merged by the
     log-sum-exp rule equals attention over the whole set."""
