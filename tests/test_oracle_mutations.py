@@ -26,6 +26,18 @@ MUTATIONS = [
      "n_take = min(topk, order.shape[0])", PINS),                                    # own block
     ("msa_oracle.py", "logits = scale * (q @ k.T)", "logits = (q @ k.T)", PINS),     # scale
     ("msa_oracle.py", "m[:, 0] + np.log(den[:, 0])", "np.log(den[:, 0])", PINS),     # lse
+    # the parity gate: which rows must match the oracle's selection exactly
+    ("msa_oracle.py", "first_left = float(scores_past[order[n_take]])",
+     "first_left = float(scores_past[order[min(n_take + 1, order.shape[0] - 1)]])",
+     PINS),                                                                          # cut + 1
+    ("msa_oracle.py", "last = float(scores_past[order[n_take - 1]])",
+     "last = float(scores_past[order[max(n_take - 2, 0)]])", PINS),                  # cut - 1
+    ("msa_oracle.py", "first_left = float(scores[order[n_take]])",
+     "first_left = float(scores[order[min(n_take + 1, order.shape[0] - 1)]])",
+     PINS),                                                                          # decode cut
+    ("msa_oracle.py", "den = max(abs(a), abs(b))", "den = abs(a)", PINS),            # gap scale
+    ("msa_oracle.py", "else (a - b) / den", "else 0.0 * (a - b) / den", PINS),       # gap = 0
+    ("msa_oracle.py", 'return float("inf")', "return 0.0", PINS),                    # none left
     ("msa_sharded.py", "lo, topk + 1)", "lo, topk)", SHARDED),                       # k+1 lists
     ("msa_sharded.py", "lo = r * base + min(r, extra)", "lo = r * base", SHARDED),   # ranges
     ("msa_sharded.py", "return O, m + np.log(den)", "return O, m", SHARDED),         # lse merge

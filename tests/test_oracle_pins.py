@@ -294,3 +294,160 @@ def test_planted_blocks_always_selected_after_they_appear():
         for j in pl:
             if j < r.t // w.block:
                 assert j in r.idx, (r.t, r.g, j, r.idx)
+
+
+# ---------------------------------------------------------------- the parity gate
+# last_taken / first_left and their relative gap decide which rows must match the
+# oracle's selection exactly; these pins hold them to values derived outside the oracle.
+
+def _gate_value(x):
+    return None if x is None else float(_ev(x))
+
+
+def test_worked_example_gate_prefill():
+    """Hand-derived cut scores of every row: t4 (gap 0.5), the exact tie at t5 (gap 0),
+    and the rows where nothing is left out (infinite gap)."""
+    ex = json.load(open(os.path.join(GOLDEN, "worked_example_s6_b2.json")))
+    sh = ex["shape"]
+    K = np.array(ex["K"], np.float32)[None, :, None, :]
+    V = np.array(ex["V"], np.float32)[None, :, None, :]
+    Q = np.array(ex["Q"], np.float32)[None]
+    for r in oracle.prefill_rows(Q, K, V, sh["block"], sh["topk"], sh["scale"]):
+        want = ex["prefill"][f"t{r.t}"]["gate"]
+        assert r.last_taken == _gate_value(want["last_taken"]), r.t
+        assert r.first_left == _gate_value(want["first_left"]), r.t
+        gap = math.inf if want["gap"] is None else float(_ev(want["gap"]))
+        assert r.gap == gap, (r.t, r.gap)
+
+
+def test_worked_example_gate_decode():
+    ex = json.load(open(os.path.join(GOLDEN, "worked_example_s6_b2.json")))
+    sh = ex["shape"]
+    K = np.array(ex["K"], np.float32)[:, None, :]
+    kbar = oracle.pool_keys(K[None], sh["block"])[0]
+    Qd = np.array(ex["decode"]["Q"], np.float32)[None]
+    (r,) = oracle.decode_rows(Qd, kbar, K, K, 6, sh["block"], sh["topk"], sh["scale"])
+    want = ex["decode"]["gate"]
+    assert (r.last_taken, r.first_left) == (float(want["last_taken"]), float(want["first_left"]))
+    assert r.gap == float(want["gap"])
+
+
+@pytest.mark.parametrize("a,b,gap", [(2.0, 1.0, 0.5), (2.0, 2.0, 0.0), (-1.0, -2.0, 0.5),
+                                     (-2.0, -2.0, 0.0), (1.0, -1.0, 2.0), (0.0, 0.0, 0.0),
+                                     (3.0, 0.0, 1.0), (0.0, -4.0, 1.0), (1e-3, -1e-3, 2.0)])
+def test_rel_gap_closed_forms(a, b, gap):
+    """(a - b) / max(|a|, |b|) by hand, including negative scores, where the larger
+    magnitude is the left-out score's (-1 vs -2 gives 1/2, not 1)."""
+    assert oracle.rel_gap(a, b) == gap
+
+
+def test_rel_gap_nothing_left_out_is_infinite():
+    assert oracle.rel_gap(None, 1.0) == math.inf
+    assert oracle.rel_gap(1.0, None) == math.inf
+    assert oracle.rel_gap(None, None) == math.inf
+
+
+def _kth_by_counting(vals, k):
+    """The k-th largest value (k >= 1) found by counting, not sorting: the v with
+    #{x > v} < k <= #{x >= v}."""
+    for v in vals:
+        if sum(x > v for x in vals) < k <= sum(x >= v for x in vals):
+            return v
+    raise AssertionError("no k-th value")
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_prefill_cut_scores_by_counting(seed):
+    """Random rows, scores rounded to a coarse grid so ties occur: last_taken is the
+    (k-1)-th best past score and first_left the k-th, found by counting.  Covers
+    negative scores, rows with fewer eligible blocks than k-1 (nothing left out) and
+    top-k 1 (nothing ranked: infinite gap)."""
+    rng = np.random.default_rng(seed)
+    for _ in range(200):
+        n_past = int(rng.integers(0, 12))
+        topk = int(rng.integers(1, 8))
+        sc = np.round(rng.standard_normal(n_past) * 2, 0 if seed % 2 else 1)
+        idx, last, first = oracle.select_prefill_row(sc, n_past, topk)
+        vals = [float(x) for x in sc]
+        n_take = min(topk - 1, n_past)
+        assert idx[:n_take + 1] == sorted(idx[:n_take + 1]) and n_past in idx
+        if n_take == 0 or n_past <= n_take:
+            assert last is None or n_past <= n_take
+            assert oracle.rel_gap(last, first) == math.inf
+        if n_take >= 1 and n_past > n_take:
+            assert last == _kth_by_counting(vals, n_take)
+            assert first == _kth_by_counting(vals, n_take + 1)
+        else:
+            assert last is None
+        # every taken past block scores >= last_taken >= first_left >= every left-out one
+        taken = [j for j in idx if 0 <= j < n_past]
+        assert len(taken) == n_take
+        if last is not None:
+            left = [j for j in range(n_past) if j not in taken]
+            assert min(vals[j] for j in taken) == last
+            assert max(vals[j] for j in left) == first
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_decode_cut_scores_by_counting(seed):
+    rng = np.random.default_rng(100 + seed)
+    for _ in range(200):
+        nb = int(rng.integers(1, 14))
+        topk = int(rng.integers(1, 9))
+        sc = np.round(rng.standard_normal(nb) * 3, 0 if seed % 2 else 1)
+        idx, last, first = oracle.select_decode_row(sc, topk)
+        vals = [float(x) for x in sc]
+        if nb > topk:
+            assert last == _kth_by_counting(vals, topk)
+            assert first == _kth_by_counting(vals, topk + 1)
+            taken = [j for j in idx if j >= 0]
+            assert min(vals[j] for j in taken) == last
+            assert max(vals[j] for j in range(nb) if j not in taken) == first
+        else:
+            assert last is None and first is None
+            assert oracle.rel_gap(last, first) == math.inf
+
+
+def test_decode_gap_closed_form():
+    """Scores (qsum . kbar_j) = j for a bank whose block j has pooled key j * e0 and a
+    query sum e0: top-3 of 10 blocks takes {7, 8, 9}, last_taken 7, first_left 6, gap
+    1/7; with the query negated the lowest blocks win and the gap is (-2 + 3) / 3."""
+    nb, block, d = 10, 4, 8
+    K = np.zeros((nb * block, 1, d), np.float32)
+    for j in range(nb):
+        K[j * block:(j + 1) * block, 0, 0] = j
+    kbar = oracle.pool_keys(K[None], block)[0]
+    q = np.zeros((1, 2, d), np.float32)
+    q[0, 0, 0] = 1.0
+    (r,) = oracle.decode_rows(q, kbar, K, K, nb * block, block, 3, 1.0)
+    assert (r.idx, r.last_taken, r.first_left) == ([7, 8, 9], 7.0, 6.0)
+    assert r.gap == 1.0 / 7.0
+    q[0, 0, 0] = -1.0
+    (r,) = oracle.decode_rows(q, kbar, K, K, nb * block, block, 3, 1.0)
+    assert (r.idx, r.last_taken, r.first_left) == ([0, 1, 2], -2.0, -3.0)
+    assert r.gap == 1.0 / 3.0
+
+
+def test_strict_rows_are_stable_under_small_perturbations():
+    """What the gate means: when the gap exceeds 1e-3, moving every score by less than
+    a quarter of the margin cannot change the selection; a row built with a smaller
+    margin flips when its two cut scores move apart the other way."""
+    rng = np.random.default_rng(7)
+    n_strict = 0
+    for _ in range(300):
+        sc = rng.standard_normal(20)
+        idx, last, first = oracle.select_prefill_row(sc, 20, 6)
+        gap = oracle.rel_gap(last, first)
+        if gap <= 1e-3:
+            continue
+        n_strict += 1
+        margin = (last - first) / 4
+        noise = rng.uniform(-margin, margin, size=20) * 0.999
+        assert oracle.select_prefill_row(sc + noise, 20, 6)[0] == idx
+    assert n_strict > 250
+    sc = np.array([5.0, 1.0, 1.0 + 5e-4, 0.0])        # blocks 1, 2 within the 1e-3 band
+    idx, last, first = oracle.select_prefill_row(sc, 4, 3)
+    assert idx == [0, 2, 4] and oracle.rel_gap(last, first) <= 1e-3
+    sc2 = sc.copy()
+    sc2[1] += 1e-3
+    assert oracle.select_prefill_row(sc2, 4, 3)[0] == [0, 1, 4]
