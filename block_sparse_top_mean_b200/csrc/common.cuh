@@ -143,6 +143,15 @@ cudaError_t launch_attn_decode(const Shape& s, int64_t n_query, const void* q, c
                                const int32_t* idx, void* o, float* lse, void* ws, int* err,
                                cudaStream_t st);
 
+// Host-side checks of a decode call's shapes and pointers (msa_api.cu), shared by the
+// decode entry points; *empty is set for a call with no work, *tc when the tensor-core
+// scan runs.  Touches no device state.
+msa_status check_decode_args(const msa_params* p, int64_t n_query, const void* q,
+                             const float* kbar, const void* kbar_hi, const void* kbar_lo,
+                             const void* k_bank, const void* v_bank, const int32_t* idx,
+                             const void* o, Shape* s, bool* tc, bool* empty);
+size_t decode_ws_bytes(const Shape& s, int64_t n_query);   // header included
+
 // Host helpers (host_util.cu): a 2-D bf16 TMA map over a row-major [rows, cols] tensor
 // with 64-column x box_rows boxes and 128-byte swizzle; the device's SM count.
 bool make_bf16_2d_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_rows);

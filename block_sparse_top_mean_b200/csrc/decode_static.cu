@@ -1,17 +1,18 @@
 // Decode against a memory bank for callers that cannot allocate device memory.
 //
 // Some callers cannot call cudaMalloc (or a caching allocator) at the point where they
-// run a decode step: a serving loop that runs inside CUDA-graph capture or a runtime
-// that forbids device allocation on its hot path.  They still own q, the bank and the
-// outputs, but have no workspace to pass.  This entry point runs the same decode
+// run a decode step: a runtime that reserves all device memory up front and forbids
+// allocation on its hot path, or a plug-in driven by a host framework that owns every
+// allocation and hands it only the tensors of the step.  They still own q, the bank and
+// the outputs, but have no workspace to pass.  This entry point runs the same decode
 // kernels as msa_decode_fwd with the workspace placed in a file-scope device array of
 // fixed size instead.
 //
 // The array is loaded with the library's device code: every GPU that loads this
 // library holds its kMsaDecodeStaticScratch bytes until the process exits.  Host code
-// cannot use the array's name as a device address, so the address is looked up once
-// per device with cudaGetSymbolAddress (on the first call made with that device
-// current) and cached.
+// cannot use the array's name as a device address (it names a host-side stand-in), so
+// the address is looked up once per device with cudaGetSymbolAddress, on the first call
+// made with that device current, and cached.
 #include <mutex>
 
 #include "common.cuh"
@@ -49,11 +50,14 @@ extern "C" msa_status msa_decode_fwd_static(const msa_params* p, int64_t n_query
                                             const void* kbar_lo, const void* k_bank,
                                             const void* v_bank, int32_t* idx, void* o,
                                             float* lse, msa_stream_t stream) {
-  if (p == nullptr || n_query < 0) return MSA_ERR_INVALID_ARG;
-  if (n_query == 0 || p->seq == 0) return MSA_OK;
-  const size_t need = msa_workspace_bytes(p, MSA_OP_DECODE, n_query);
-  if (need == 0) return MSA_ERR_INVALID_ARG;
-  if (need > kMsaDecodeStaticScratch) return MSA_ERR_WORKSPACE;   // beyond the fixed scratch
+  // every argument check runs before any CUDA call, with msa_decode_fwd's own statuses
+  msa::Shape s;
+  bool tc = false, empty = false;
+  const msa_status chk = msa::check_decode_args(p, n_query, q, kbar, kbar_hi, kbar_lo, k_bank,
+                                                v_bank, idx, o, &s, &tc, &empty);
+  if (chk != MSA_OK || empty) return chk;
+  if (msa::decode_ws_bytes(s, n_query) > kMsaDecodeStaticScratch)
+    return MSA_ERR_WORKSPACE;                                   // beyond the fixed scratch
   void* scratch = nullptr;
   const msa_status st = scratch_address(&scratch);
   if (st != MSA_OK) return st;

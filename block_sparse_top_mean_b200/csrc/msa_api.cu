@@ -130,6 +130,39 @@ cudaError_t launch_attention(const Shape& s, const void* q, const void* k, const
 
 }  // namespace
 
+namespace msa {
+
+msa_status check_decode_args(const msa_params* p, int64_t n_query, const void* q,
+                             const float* kbar, const void* kbar_hi, const void* kbar_lo,
+                             const void* k_bank, const void* v_bank, const int32_t* idx,
+                             const void* o, Shape* s, bool* tc, bool* empty) {
+  *tc = false;
+  *empty = false;
+  msa_status st = check_params(p, true, s);
+  if (st != MSA_OK) return st;
+  if (n_query < 0) return MSA_ERR_INVALID_ARG;
+  if (n_query == 0 || s->seq == 0) {
+    *empty = true;
+    return MSA_OK;
+  }
+  if (n_query > 65535 * 64) return MSA_ERR_UNSUPPORTED;
+  // the tensor-core scan reads the bf16 planes; the SIMT scan the fp32 pooled keys
+  *tc = kbar_hi != nullptr && kbar_lo != nullptr && msa::tc_decode_supported(*s);
+  if (q == nullptr || (!*tc && kbar == nullptr) || k_bank == nullptr || v_bank == nullptr ||
+      idx == nullptr || o == nullptr)
+    return MSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(kbar) || !aligned16(kbar_hi) || !aligned16(kbar_lo) ||
+      !aligned16(k_bank) || !aligned16(v_bank) || !aligned16(o))
+    return MSA_ERR_INVALID_ARG;
+  return MSA_OK;
+}
+
+size_t decode_ws_bytes(const Shape& s, int64_t n_query) {
+  return ws_bytes_for(s, MSA_OP_DECODE, n_query);
+}
+
+}  // namespace msa
+
 extern "C" {
 
 const char* msa_version(void) { return "msa-b200 0.1.0 (sm_100a)"; }
@@ -142,6 +175,7 @@ const char* msa_status_string(msa_status st) {
     case MSA_ERR_WORKSPACE: return "workspace missing, too small or misaligned";
     case MSA_ERR_CUDA: return "CUDA error";
     case MSA_ERR_DEVICE: return "device-side error flag set";
+    case MSA_ERR_TIMEOUT: return "a bounded device wait ran out";
     default: return "unknown status";
   }
 }
@@ -261,19 +295,10 @@ msa_status msa_decode_fwd(const msa_params* p, int64_t n_query, const void* q, c
                           const void* v_bank, int32_t* idx, void* o, float* lse, void* ws,
                           size_t ws_bytes, msa_stream_t stream) {
   Shape s;
-  msa_status st = check_params(p, true, &s);
-  if (st != MSA_OK) return st;
-  if (n_query < 0) return MSA_ERR_INVALID_ARG;
-  if (n_query == 0 || s.seq == 0) return MSA_OK;
-  if (n_query > 65535 * 64) return MSA_ERR_UNSUPPORTED;
-  // the tensor-core scan reads the bf16 planes; the SIMT scan the fp32 pooled keys
-  const bool tc = kbar_hi != nullptr && kbar_lo != nullptr && msa::tc_decode_supported(s);
-  if (q == nullptr || (!tc && kbar == nullptr) || k_bank == nullptr || v_bank == nullptr ||
-      idx == nullptr || o == nullptr)
-    return MSA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(kbar) || !aligned16(kbar_hi) || !aligned16(kbar_lo) ||
-      !aligned16(k_bank) || !aligned16(v_bank) || !aligned16(o))
-    return MSA_ERR_INVALID_ARG;
+  bool tc = false, empty = false;
+  msa_status st = msa::check_decode_args(p, n_query, q, kbar, kbar_hi, kbar_lo, k_bank, v_bank,
+                                         idx, o, &s, &tc, &empty);
+  if (st != MSA_OK || empty) return st;
   if ((st = check_ws(s, MSA_OP_DECODE, n_query, ws, ws_bytes)) != MSA_OK) return st;
   cudaStream_t cs = (cudaStream_t)stream;
   char* sel_ws = ws_body(ws);
@@ -383,6 +408,18 @@ msa_status msa_read_device_error(const void* ws, int32_t* bits, msa_stream_t str
   if (e != cudaSuccess) return MSA_ERR_CUDA;
   *bits = h;
   return h != 0 ? MSA_ERR_DEVICE : MSA_OK;
+}
+
+size_t msa_workspace_size(const msa_params* p, int32_t op, int64_t n_query) {
+  return msa_workspace_bytes(p, op, n_query);
+}
+
+msa_status msa_get_device_status(const void* ws, msa_stream_t stream) {
+  int32_t bits = 0;
+  const msa_status st = msa_read_device_error(ws, &bits, stream);
+  if (st != MSA_OK && st != MSA_ERR_DEVICE) return st;
+  if (bits & MSA_DEVERR_TIMEOUT) return MSA_ERR_TIMEOUT;
+  return bits != 0 ? MSA_ERR_DEVICE : MSA_OK;
 }
 
 msa_status msa_clear_device_error(void* ws, msa_stream_t stream) {

@@ -194,6 +194,21 @@ def test_static_decode_rejects_before_touching_the_device(lib):
     # more queries than the fixed 32 MiB scratch can hold
     assert st(ctypes.byref(p), 100_000, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None,
               None) == _lib.MSA_ERR_WORKSPACE
+    # null and misaligned pointers, and unsupported shapes, give msa_decode_fwd's own
+    # statuses without any CUDA call (on this host any CUDA call would return an error)
+    odd = ctypes.c_void_p(4096 + 8)
+    args = [FAKE] * 8                                 # q, kbar, hi, lo, k, v, idx, o
+    for i, bad in [(0, None), (4, None), (5, None), (6, None), (7, None), (0, odd), (4, odd),
+                   (7, odd), (2, odd)]:
+        a = list(args)
+        a[i] = bad
+        assert st(ctypes.byref(p), 4, *a, None, None) == _lib.MSA_ERR_INVALID_ARG, (i, bad)
+    # no planes and no fp32 pooled keys
+    assert st(ctypes.byref(p), 4, FAKE, None, None, None, FAKE, FAKE, FAKE, FAKE, None,
+              None) == _lib.MSA_ERR_INVALID_ARG
+    for kw in (dict(d=96), dict(hq=24)):              # G = 3 and d = 96 are unsupported
+        bad = _p(seq=10_000, block=64, topk=32, **kw)
+        assert st(ctypes.byref(bad), 4, *args, None, None) == _lib.MSA_ERR_UNSUPPORTED
 
 
 def test_empty_inputs_are_noops(lib):
@@ -208,5 +223,16 @@ def test_empty_inputs_are_noops(lib):
 
 
 def test_status_strings(lib):
-    for c in range(6):
+    for c in range(7):
         assert lib.msa_status_string(c).decode()
+
+
+def test_interface_sketch_names(lib):
+    """msa_workspace_size is msa_workspace_bytes; msa_get_device_status rejects a null
+    workspace before any CUDA call."""
+    for op in range(6):
+        p = _p()
+        assert lib.msa_workspace_size(ctypes.byref(p), op, 64) == \
+            lib.msa_workspace_bytes(ctypes.byref(p), op, 64)
+    assert lib.msa_get_device_status(None, None) == _lib.MSA_ERR_INVALID_ARG
+    assert lib.msa_status_string(_lib.MSA_ERR_TIMEOUT).decode() == "a bounded device wait ran out"

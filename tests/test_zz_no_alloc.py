@@ -1,11 +1,13 @@
 """The allocation-free decode entry point (msa_decode_fwd_static).
 
-Callers that cannot allocate device memory at decode time (graph-captured serving loops,
-runtimes that forbid device allocation on the hot path) use a fixed device scratch
-inside the library instead of a workspace.  This checks, through the C ABI, that two
-calls in a row give the same selection and outputs as msa_decode_fwd with a caller
-workspace.  It sits in its own file that pytest collects last, and it holds whether it
-runs alone in a fresh process or after the other tests.
+Some callers cannot allocate device memory at decode time: a runtime that reserves all
+device memory up front and forbids allocation on its hot path, or a plug-in whose host
+framework owns every allocation and hands it only the step's tensors.  They use a fixed
+device scratch inside the library instead of a workspace.  This checks, through the C
+ABI, that two calls in a row give exactly the selection and outputs of msa_decode_fwd
+with a caller workspace (the same kernels on the same inputs are bitwise
+deterministic).  It sits in its own file that pytest collects last, and it holds
+whether it runs alone in a fresh process or after the other tests.
 """
 import ctypes
 
@@ -46,8 +48,8 @@ def test_static_scratch_decode_matches_workspace_decode():
         assert st == _lib.MSA_OK, (call, st)
         torch.cuda.synchronize()
         assert torch.equal(idx, idx_ref), call
-        assert (o.float() - o_ref.float()).abs().max().item() <= 2e-2, call
-        assert (lse - lse_ref).abs().max().item() <= 2e-3, call
+        assert torch.equal(o, o_ref), call
+        assert torch.equal(lse, lse_ref), call
 
 
 def test_static_scratch_rejects_sizes_beyond_the_limit():
