@@ -24,7 +24,7 @@ __all__ = [
     "prefill_fwd", "decode_fwd", "decode_fwd_static", "encode_bank", "decode_fwd_tiled",
     "decode_select_tiled", "decode_attn_tiled", "attn_slab_tokens",
     "read_device_error",
-    "clear_device_error", "version",
+    "clear_device_error", "version", "exp2_poly_eval",
     "MsaError", "MsaParams",
 ]
 
@@ -291,3 +291,13 @@ def read_device_error(ws: torch.Tensor) -> int:
 def clear_device_error(ws: torch.Tensor) -> None:
     _lib.check("msa_clear_device_error", _lib.load().msa_clear_device_error(
         _ptr(ws), _stream(ws.device)))
+
+
+def exp2_poly_eval(x: torch.Tensor) -> torch.Tensor:
+    """The attention softmax's own FMA-pipe 2^x on a CUDA fp32 tensor (diagnostic)."""
+    if x.dtype != torch.float32:
+        raise ValueError("exp2_poly_eval takes fp32")
+    y = torch.empty_like(x)
+    _lib.check("msa_exp2_poly_eval", _lib.load().msa_exp2_poly_eval(
+        _ptr(x), _ptr(y), x.numel(), _stream(x.device)))
+    return y

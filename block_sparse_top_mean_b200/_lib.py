@@ -11,7 +11,7 @@ from ctypes import POINTER, c_char_p, c_float, c_int32, c_int64, c_size_t, c_voi
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmsa_b200.so")
 
 MSA_OK, MSA_ERR_INVALID_ARG, MSA_ERR_UNSUPPORTED, MSA_ERR_WORKSPACE, MSA_ERR_CUDA, \
-    MSA_ERR_DEVICE = range(6)
+    MSA_ERR_DEVICE, MSA_ERR_TIMEOUT = range(7)
 MSA_F32, MSA_BF16 = 0, 1
 OP_TOPK_SELECT, OP_SPARSE_ATTN, OP_PREFILL, OP_DECODE, OP_SPARSE_ATTN_MIN, OP_PREFILL_MIN = range(6)
 DEVERR_IDX_RANGE, DEVERR_TIMEOUT = 0x1, 0x2
@@ -49,6 +49,9 @@ SIGNATURES = {
                                        c_size_t, c_void_p]),
     "msa_read_device_error": (c_int32, [c_void_p, POINTER(c_int32), c_void_p]),
     "msa_clear_device_error": (c_int32, [c_void_p, c_void_p]),
+    "msa_workspace_size": (c_size_t, [c_void_p, c_int32, c_int64]),
+    "msa_get_device_status": (c_int32, [c_void_p, c_void_p]),
+    "msa_exp2_poly_eval": (c_int32, [c_void_p, c_void_p, c_int64, c_void_p]),
 }
 
 

@@ -23,12 +23,14 @@
 #include <math_constants.h>
 
 #include "common.cuh"
+#include "fastmath.cuh"
 #include "sm100.cuh"
 
 namespace msa {
 namespace {
 
 using namespace sm100;
+using namespace fastmath;
 
 constexpr int kD = 128;
 constexpr int kRowsT = 128;          // rows per tile
@@ -187,11 +189,6 @@ constexpr int kIssuerWarp = 8;
 constexpr int kGatherWarp = 9;
 constexpr float kRescaleLog2 = 8.f;  // chunk-1 max may exceed the reference by 2^8
 
-__device__ __forceinline__ float fast_exp2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
 
 // Decodes a tile record into (sequence, group, block, 256-key segment) with 32-bit math.
 struct TileId {
@@ -206,56 +203,6 @@ __device__ __forceinline__ TileId decode_tile(const int4& tl, const Geom& g) {
   d.b = tl.w / g.hkv;
   d.gg = tl.w - d.b * g.hkv;
   return d;
-}
-
-// Packed two-lane fp32 arithmetic (sm_100: one instruction for both lanes).
-__device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, float b0, float b1,
-                                      float c0, float c1) {
-  asm("{\n.reg .b64 a, b, c, d;\nmov.b64 a, {%2, %3};\nmov.b64 b, {%4, %5};\n"
-      "mov.b64 c, {%6, %7};\nfma.rn.f32x2 d, a, b, c;\nmov.b64 {%0, %1}, d;\n}"
-      : "=f"(d0), "=f"(d1)
-      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
-}
-__device__ __forceinline__ void fadd2(float& d0, float& d1, float a0, float a1, float b0,
-                                      float b1) {
-  asm("{\n.reg .b64 a, b, d;\nmov.b64 a, {%2, %3};\nmov.b64 b, {%4, %5};\n"
-      "add.rn.f32x2 d, a, b;\nmov.b64 {%0, %1}, d;\n}"
-      : "=f"(d0), "=f"(d1)
-      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
-}
-__device__ __forceinline__ void fmul2(float& d0, float& d1, float a0, float a1, float b0,
-                                      float b1) {
-  asm("{\n.reg .b64 a, b, d;\nmov.b64 a, {%2, %3};\nmov.b64 b, {%4, %5};\n"
-      "mul.rn.f32x2 d, a, b;\nmov.b64 {%0, %1}, d;\n}"
-      : "=f"(d0), "=f"(d1)
-      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
-}
-__device__ __forceinline__ float fmax3(float a, float b, float c) {
-  float d;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-  return d;
-}
-
-// 2^x for two lanes on the FMA pipe: adding 1.5 * 2^23 rounds x to the nearest integer n
-// and leaves n in the low mantissa bits; f = x - n lies in [-1/2, 1/2]; 2^f comes from a
-// cubic fitted here for minimal relative error on that interval (7.5e-5, below the bf16
-// rounding P goes through); n is then added to the exponent field.  x is clamped to -126.
-__device__ __forceinline__ void poly_exp2x2(float x0, float x1, float& p0, float& p1) {
-  constexpr float kShift = 12582912.f;            // 1.5 * 2^23
-  x0 = fmaxf(x0, -126.f);
-  x1 = fmaxf(x1, -126.f);
-  float t0, t1, n0, n1, f0, f1;
-  fadd2(t0, t1, x0, x1, kShift, kShift);
-  fadd2(n0, n1, t0, t1, -kShift, -kShift);        // exact: n as a float
-  ffma2(f0, f1, n0, n1, -1.f, -1.f, x0, x1);      // exact: x - n
-  float q0, q1;
-  ffma2(q0, q1, 0.0551716573536396f, 0.0551716573536396f, f0, f1, 0.2426111400127411f,
-        0.2426111400127411f);
-  ffma2(q0, q1, q0, q1, f0, f1, 0.6932609677314758f, 0.6932609677314758f);
-  ffma2(q0, q1, q0, q1, f0, f1, 0.9999280571937561f, 0.9999280571937561f);
-  // the low 9 bits of t's pattern are n's; shifted by 23 only n << 23 remains
-  p0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
-  p1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
 }
 
 #ifndef MSA_POLY_PAIRS

@@ -35,7 +35,8 @@
  *   - All tensor pointers are DEVICE pointers, row-major and contiguous, 16-byte
  *     aligned.  The caller owns every buffer; the library allocates nothing.
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
- *     stream) and never synchronise, except msa_read_device_error.
+ *     stream) and never synchronise, except msa_read_device_error and
+ *     msa_get_device_status.
  *   - Arguments are checked on the host before anything is launched; a failed check
  *     returns MSA_ERR_INVALID_ARG / MSA_ERR_UNSUPPORTED / MSA_ERR_WORKSPACE and launches
  *     nothing.  A launch failure returns MSA_ERR_CUDA.
@@ -79,7 +80,8 @@ typedef enum {
   MSA_ERR_UNSUPPORTED = 2, /* well-formed but outside what the kernels implement */
   MSA_ERR_WORKSPACE = 3,   /* workspace missing, too small or misaligned */
   MSA_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed */
-  MSA_ERR_DEVICE = 5       /* returned by msa_read_device_error when a bit is set */
+  MSA_ERR_DEVICE = 5,      /* returned by msa_read_device_error when a bit is set */
+  MSA_ERR_TIMEOUT = 6      /* msa_get_device_status: a bounded device wait ran out */
 } msa_status;
 
 typedef enum { MSA_F32 = 0, MSA_BF16 = 1 } msa_dtype;
@@ -233,19 +235,22 @@ MSA_API msa_status msa_decode_fwd_tiled(const msa_params* p, int64_t n_query, co
 #define MSA_DECODE_STATIC_SCRATCH_BYTES ((size_t)32 << 20)
 
 /* Decode without a caller workspace, for callers that cannot allocate device memory
- * where they run a decode step (for example a serving loop inside CUDA-graph capture,
- * or a runtime that forbids device allocation on its hot path).  The pages have no
- * counterpart: this is a deployment variant of msa_decode_fwd, with the same arguments
- * minus the workspace, the same kernels and the same results.
+ * where they run a decode step (for example a runtime that reserves all device memory up
+ * front and forbids allocation on its hot path, or a plug-in whose host framework owns
+ * every allocation and passes only the step's tensors).  The pages have no counterpart:
+ * this is a deployment variant of msa_decode_fwd, with the same arguments minus the
+ * workspace, the same kernels and the same results.
  *   - Scratch: a file-scope device array of MSA_DECODE_STATIC_SCRATCH_BYTES that every
  *     GPU loading this library keeps until the process exits.  The call allocates
  *     nothing (no cudaMalloc/cudaFree, no allocating library routine).
- *   - Limit: returns MSA_ERR_WORKSPACE, launching nothing, when
- *     msa_workspace_bytes(p, MSA_OP_DECODE, n_query) exceeds that size (64 queries x 32
+ *   - Checks: every argument is checked first, with msa_decode_fwd's statuses, before
+ *     any CUDA call.  Returns MSA_ERR_WORKSPACE, launching nothing, when
+ *     msa_workspace_bytes(p, MSA_OP_DECODE, n_query) exceeds the array (64 queries x 32
  *     heads against a 10M-token bank need about 21 MB).
  *   - Set-up: the first call on a device looks up the array's device address with that
- *     device current (cudaGetSymbolAddress) and caches it; make that first call before
- *     any stream capture.
+ *     device current (cudaGetSymbolAddress) and caches it for the process; make that
+ *     first call before any stream capture.  cudaDeviceReset on a device invalidates the
+ *     cached address: do not call this entry on that device again in the same process.
  *   - Sharing: every call on a device uses the same array, which keeps the last call's
  *     contents; the call clears what must start at zero.  Calls that overlap on the GPU
  *     (concurrent streams, or several host threads) race on the array: serialise them.
@@ -262,6 +267,21 @@ MSA_API msa_status msa_read_device_error(const void* ws, int32_t* bits, msa_stre
 
 /* Clears the workspace's device error word (asynchronous on `stream`). */
 MSA_API msa_status msa_clear_device_error(void* ws, msa_stream_t stream);
+
+/* The same two queries under the names of the library's original interface sketch:
+ * msa_workspace_size is msa_workspace_bytes; msa_get_device_status synchronises `stream`
+ * and returns MSA_ERR_TIMEOUT when the workspace's error word holds MSA_DEVERR_TIMEOUT,
+ * MSA_ERR_DEVICE when it holds any other bit, else MSA_OK (the word is left as it is). */
+MSA_API size_t msa_workspace_size(const msa_params* p, int32_t op, int64_t n_query);
+MSA_API msa_status msa_get_device_status(const void* ws, msa_stream_t stream);
+
+/* Diagnostic: y[i] = the attention softmax's own base-2 exponential of x[i] (device
+ * fp32 arrays of n elements), the FMA-pipe cubic that takes part of the softmax's
+ * exponentials off the MUFU unit.  [MiniMax] "How MSA Works" keeps the main branch exact;
+ * this entry lets a caller hold that helper to its bound: relative error <= 7.5e-5 for
+ * x >= -125.5, a value in [0, 2^-125] below.  The pages have no counterpart.
+ * Asynchronous on `stream`. */
+MSA_API msa_status msa_exp2_poly_eval(const float* x, float* y, int64_t n, msa_stream_t stream);
 
 #ifdef __cplusplus
 }
