@@ -1,15 +1,20 @@
 #!/usr/bin/env python
 """Benchmark of the block-sparse top-k attention hot path on B200; prints ONE JSON line.
 
-A step is one pass of the whole hot path over one synthetic sequence resident in HBM:
-pool keys -> fused block scoring + top-k -> sparse attention, each through the C ABI.
+A prefill step is one pass of the whole hot path over one synthetic sequence resident
+in HBM: pool keys -> fused block scoring + top-k -> sparse attention, each through the C
+ABI.  A decode step is the selection and the attention of 64 queries against an encoded
+10M-token bank resident in HBM.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
-Multi-GPU (torchrun, one rank per GPU): every rank runs its own independent sequence
-(weak scaling, no collective on the data path); the time is the max over ranks and
-`value` counts the work of all ranks.  `--impl reference` times the fp64 CPU oracle on
-a bounded sample of the same workload (rank 0 only).
+With no --workload the line's headline is the 1M-token prefill, and the 128K planted
+prefill and the 10M-token decode are timed the same way (K steps after W warm-ups) under
+"workloads".  Multi-GPU (torchrun, one rank per GPU): every rank runs its own independent
+problems (weak scaling, no collective on the data path); the time is the max over ranks
+and `value` counts the work of all ranks.  The CPU baseline and `--impl reference` time
+the fp64 oracle on the host's cores (worker processes forked before the first CUDA call)
+on a bounded sample of the same workload, rank 0 only.
 """
 from __future__ import annotations
 
@@ -18,11 +23,13 @@ import ctypes
 import datetime
 import json
 import math
+import multiprocessing as mp
 import os
 import statistics
 import subprocess
 import sys
 import time
+from concurrent.futures import ProcessPoolExecutor
 
 import numpy as np
 import torch
@@ -33,6 +40,7 @@ sys.path.insert(0, ROOT)
 import msa_inputs as mi  # noqa: E402
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+DEFAULT_EXTRAS = ("prefill_128k_b128_k16_planted", "decode_bank10m_b64_k32")
 
 
 # ------------------------------------------------------------------ workload arithmetic
@@ -48,14 +56,20 @@ def prefill_flops(w: mi.Workload) -> tuple[float, float]:
     return attn, score
 
 
+def prefill_entries(w: mi.Workload) -> int:
+    """Selected (token, group, block) entries of one pass (past blocks + the own block)."""
+    t = np.arange(w.seq, dtype=np.int64)
+    return int(np.minimum(w.topk, t // w.block + 1).sum()) * w.hkv * w.batch
+
+
 def decode_work(w: mi.Workload) -> dict:
     nb = w.nb
     full = min(w.topk, nb) * w.block
     return dict(
         attn_flops=float(w.n_query * w.hq * 4 * w.d * full),
         score_flops=float(w.n_query * w.hkv * 2 * w.d * nb),
-        # bytes the two phases must read at least: the pooled-key bank once (as bf16), and
-        # the selected K/V blocks once per (query, group)
+        # bytes the two phases must read at least: the pooled-key bank once as one bf16
+        # plane, and the selected K/V blocks once per (query, group)
         score_bytes=float(nb * w.hkv * w.d * 2),
         attn_bytes=float(w.n_query * w.hkv * full * w.d * 2 * 2),
     )
@@ -197,6 +211,243 @@ def max_over_ranks(x: float, world: int) -> float:
     return float(t.item())
 
 
+# ------------------------------------------------------------------ the oracle on host cores
+# Worker processes are forked before the first CUDA call of this process (a process
+# forked after CUDA is initialised can hang) and read the sampled workload's inputs from
+# host memory-mapped files; each returns the perf_counter interval of its oracle work.
+
+def _to_f32(x: np.ndarray) -> np.ndarray:
+    """fp32 values of a host array holding fp32 values or bf16 bit patterns (exact)."""
+    if x.dtype == np.uint16:
+        return (np.asarray(x).astype(np.uint32) << 16).view(np.float32)
+    return np.asarray(x, dtype=np.float32)
+
+
+class _HostRows:
+    """Read-only view of a memory-mapped [b, S, h, d] input: indexing returns fp32."""
+
+    def __init__(self, arr):
+        self.a = arr
+        self.shape = arr.shape
+
+    def __getitem__(self, key):
+        return _to_f32(self.a[key])
+
+
+class _QRows:
+    """The query rows of the sampled tokens only, indexed like Q[b, t] / Q[b, t, heads]."""
+
+    def __init__(self, rows: np.ndarray, keys, shape):
+        self.rows = rows
+        self.pos = {k: i for i, k in enumerate(keys)}
+        self.shape = shape
+
+    def __getitem__(self, key):
+        r = self.rows[self.pos[(key[0], key[1])]]
+        return r if len(key) == 2 else r[key[2]]
+
+
+def _w_init():
+    torch.set_num_threads(1)
+
+
+def _w_noop(_):
+    return os.getpid()
+
+
+def _w_pool(spec):
+    import oracle
+    from threadpoolctl import threadpool_limits
+    K = np.memmap(spec["k"], dtype=spec["k_dtype"], mode="r", shape=spec["k_shape"])
+    kbar = np.memmap(spec["kbar"], dtype=np.float64, mode="r+", shape=spec["kbar_shape"])
+    block, S = spec["block"], spec["k_shape"][1]
+    j0, j1 = spec["blocks"]
+    with threadpool_limits(limits=1):
+        t0 = time.perf_counter()
+        for b in range(spec["k_shape"][0]):
+            x = _to_f32(K[b:b + 1, j0 * block:min(S, j1 * block)])
+            kbar[b:b + 1, j0:j1] = oracle.pool_keys(x, block)
+        t1 = time.perf_counter()
+    kbar.flush()
+    return t0, t1
+
+
+def _w_prefill(spec):
+    import oracle
+    from threadpoolctl import threadpool_limits
+    K = _HostRows(np.memmap(spec["k"], dtype=spec["k_dtype"], mode="r", shape=spec["k_shape"]))
+    V = _HostRows(np.memmap(spec["v"], dtype=spec["k_dtype"], mode="r", shape=spec["k_shape"]))
+    kbar = np.memmap(spec["kbar"], dtype=np.float64, mode="r", shape=spec["kbar_shape"])
+    Q = _QRows(spec["q_rows"], spec["rows"], spec["q_shape"])
+    with threadpool_limits(limits=1):
+        t0 = time.perf_counter()
+        oracle.prefill_rows(Q, K, V, spec["block"], spec["topk"], spec["scale"],
+                            rows=spec["rows"], kbar=kbar)
+        t1 = time.perf_counter()
+    return t0, t1
+
+
+def _w_decode(spec):
+    import oracle
+    from threadpoolctl import threadpool_limits
+    w = spec["w"]
+    K, V = mi.lazy_decode_bank(w, spec["seed"])
+    kbar = np.memmap(spec["kbar"], dtype=np.float64, mode="r", shape=spec["kbar_shape"])
+    with threadpool_limits(limits=1):
+        t0 = time.perf_counter()
+        oracle.decode_rows(spec["qd"], kbar, K, V, w.seq, w.block, w.topk, w.scale,
+                           queries=spec["queries"])
+        t1 = time.perf_counter()
+    return t0, t1
+
+
+class OraclePool:
+    """Host worker processes for the oracle timings (see above)."""
+
+    def __init__(self, n: int):
+        self.n = n
+        self.ex = ProcessPoolExecutor(n, mp_context=mp.get_context("fork"), initializer=_w_init)
+        list(self.ex.map(_w_noop, range(n)))          # every worker exists from here on
+        shm = "/dev/shm"
+        self.dir = shm if os.path.isdir(shm) and os.access(shm, os.W_OK) else "/tmp"
+        self.files = []
+
+    @staticmethod
+    def cores() -> int:
+        try:
+            n = len(os.sched_getaffinity(0))
+        except AttributeError:
+            n = os.cpu_count() or 1
+        return max(1, min(n, 64))
+
+    def file(self, tag: str, shape, dtype) -> tuple[str, np.memmap]:
+        path = os.path.join(self.dir, f"msa_bench_{os.getpid()}_{tag}_{len(self.files)}.bin")
+        self.files.append(path)
+        return path, np.memmap(path, dtype=dtype, mode="w+", shape=tuple(shape))
+
+    def host_copy(self, tag: str, t: torch.Tensor) -> tuple[str, str]:
+        """A host file holding t's values (bf16 as bit patterns); returns (path, dtype)."""
+        if t.dtype == torch.bfloat16:
+            arr, dt = t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16), "uint16"
+        else:
+            arr, dt = t.float().contiguous().cpu().numpy(), "float32"
+        path, mm = self.file(tag, arr.shape, dt)
+        mm[...] = arr
+        mm.flush()
+        del mm
+        return path, dt
+
+    def run(self, fn, specs) -> float:
+        """Runs the specs on the workers; returns the wall time of their work."""
+        spans = list(self.ex.map(fn, specs))
+        return max(s[1] for s in spans) - min(s[0] for s in spans)
+
+    def clear_files(self):
+        for p in self.files:
+            try:
+                os.remove(p)
+            except OSError:
+                pass
+        self.files = []
+
+    def close(self):
+        self.clear_files()
+        self.ex.shutdown(cancel_futures=True)
+
+
+def _split(n: int, parts: int):
+    base, extra = divmod(n, parts)
+    lo = 0
+    for r in range(parts):
+        hi = lo + base + (1 if r < extra else 0)
+        if hi > lo:
+            yield lo, hi
+        lo = hi
+
+
+class PrefillOracle:
+    """The oracle's pooling (all blocks) and selection + attention (a token sample) of a
+    prefill workload, on the pool's workers."""
+
+    def __init__(self, pool: OraclePool, w: mi.Workload, q, k, v):
+        self.pool, self.w, self.q = pool, w, q
+        self.kpath, self.kdt = pool.host_copy("k", k)
+        self.vpath, _ = pool.host_copy("v", v)
+        self.kbar_shape = (w.batch, w.nb, w.hkv, w.d)
+        self.kbar_path, mm = pool.file("kbar", self.kbar_shape, np.float64)
+        del mm
+
+    def pool_keys(self) -> float:
+        w = self.w
+        specs = [dict(k=self.kpath, k_dtype=self.kdt, k_shape=(w.batch, w.seq, w.hkv, w.d),
+                      kbar=self.kbar_path, kbar_shape=self.kbar_shape, block=w.block,
+                      blocks=r) for r in _split(w.nb, self.pool.n)]
+        return self.pool.run(_w_pool, specs)
+
+    def rows(self, tokens_per_worker: int, seed: int) -> tuple[float, int]:
+        w = self.w
+        rng = np.random.default_rng(seed)
+        n = min(w.seq * w.batch, tokens_per_worker * self.pool.n)
+        flat = np.sort(rng.choice(w.seq * w.batch, size=n, replace=False))
+        rows = [(int(f // w.seq), int(f % w.seq)) for f in flat]
+        bi = torch.tensor([r[0] for r in rows], device=self.q.device)
+        ti = torch.tensor([r[1] for r in rows], device=self.q.device)
+        q_rows = self.q[bi, ti].float().cpu().numpy()
+        specs = []
+        for lo, hi in _split(len(rows), self.pool.n):
+            specs.append(dict(k=self.kpath, v=self.vpath, k_dtype=self.kdt,
+                              k_shape=(w.batch, w.seq, w.hkv, w.d), kbar=self.kbar_path,
+                              kbar_shape=self.kbar_shape, q_rows=q_rows[lo:hi],
+                              rows=rows[lo:hi], q_shape=tuple(self.q.shape), block=w.block,
+                              topk=w.topk, scale=w.scale))
+        return self.pool.run(_w_prefill, specs), len(rows)
+
+    def step_seconds(self, tokens_per_worker: int, seed: int) -> tuple[float, str]:
+        """Oracle seconds of one whole prefill step: the pooling of every block, and the
+        selection + attention of a token sample extrapolated to every token."""
+        t_pool = self.pool_keys()
+        t_rows, n = self.rows(tokens_per_worker, seed)
+        w = self.w
+        t = t_pool + t_rows * (w.seq * w.batch) / n
+        sample = (f"pooling of all {w.nb * w.batch} blocks + selection and attention of {n} "
+                  f"random tokens x {w.hkv} groups (of {w.seq * w.batch}), extrapolated to "
+                  f"every token; numpy fp64, {self.pool.n} worker processes, 1 thread each")
+        return t, sample
+
+
+class DecodeOracle:
+    """The oracle's decode of a query sample against the workload's bank (regenerated
+    block by block from the seeded generator as the oracle reads it).  The fp64 pooled
+    keys of a 10M-token bank would take minutes to build on the host, so random values of
+    the right shape stand in for them: only the time is measured."""
+
+    def __init__(self, pool: OraclePool, w: mi.Workload, q, seed: int = 0):
+        self.pool, self.w, self.seed = pool, w, seed
+        self.qd = q.float().cpu().numpy()
+        self.kbar_shape = (w.nb, w.hkv, w.d)
+        self.kbar_path, mm = pool.file("dkbar", self.kbar_shape, np.float64)
+        rng = np.random.default_rng(7)
+        for lo in range(0, w.nb, 1 << 14):
+            hi = min(w.nb, lo + (1 << 14))
+            mm[lo:hi] = rng.standard_normal((hi - lo, w.hkv, w.d)) * 0.125
+        mm.flush()
+        del mm
+
+    def step_seconds(self, queries_per_worker: int, seed: int) -> tuple[float, str]:
+        w = self.w
+        n = min(w.n_query, queries_per_worker * self.pool.n)
+        qs = [int(x) for x in np.sort(np.random.default_rng(seed).choice(w.n_query, n,
+                                                                          replace=False))]
+        specs = [dict(w=w, seed=self.seed, kbar=self.kbar_path, kbar_shape=self.kbar_shape,
+                      qd=self.qd, queries=qs[lo:hi]) for lo, hi in _split(n, self.pool.n)]
+        t = self.pool.run(_w_decode, specs) * w.n_query / n
+        sample = (f"{n} of {w.n_query} queries (all {w.hkv} groups)"
+                  + (f", extrapolated to {w.n_query}" if n < w.n_query else "")
+                  + f"; numpy fp64, {self.pool.n} worker processes, 1 thread each; random "
+                  "stand-in pooled keys")
+        return t, sample
+
+
 # ------------------------------------------------------------------ our implementation
 
 class PrefillRunner:
@@ -255,18 +506,17 @@ class PrefillRunner:
 
 class DecodeRunner:
     """Decode of n_query queries against a bank resident in HBM, through the C ABI.  The
-    bank's pooled keys are computed once up front (offline encoding, not timed)."""
+    bank's pooled keys and encoded images are built once up front (the offline encoding
+    of a bank, not timed); the step reads only the encoded images."""
 
     def __init__(self, w: mi.Workload, seed: int):
         import block_sparse_top_mean_b200 as msa
         from block_sparse_top_mean_b200 import _lib
         self.msa, self.lib, self.w = msa, _lib.load(), w
-        self.q, self.k, self.v = mi.decode_inputs(w, device="cuda", seed=seed)
-        # offline bank preparation (not timed): the routing keys as bf16 hi/lo planes, then
-        # the encoded images the decode kernels stream with one bulk copy per tile
-        _, khi, klo = (t[0] for t in msa.pool_keys(self.k[None], w.block, split=True))
-        self.kt, self.vt, self.bt = msa.encode_bank(self.k, self.v, khi, klo, w.block)
-        del khi, klo                            # the step reads only the encoded bank
+        self.q, k, v = mi.decode_inputs(w, device="cuda", seed=seed)
+        _, khi, klo = (t[0] for t in msa.pool_keys(k[None], w.block, split=True))
+        self.kt, self.vt, self.bt = msa.encode_bank(k, v, khi, klo, w.block)
+        del k, v, khi, klo                      # the natural layout is not needed any more
         dev = self.q.device
         self.p = msa.params(batch=1, seq=w.seq, hq=w.hq, hkv=w.hkv, d=w.d, block=w.block,
                             topk=w.topk, scale=w.scale, dtype=self.q.dtype)
@@ -301,20 +551,16 @@ class DecodeRunner:
             events[2].record()
 
 
-def run_decode(args, world, rank, local):
-    w = workload_of(args)
-    from block_sparse_top_mean_b200 import build
-    if rank == 0:
-        build.build()
-    barrier(world)
-    r = DecodeRunner(w, seed=rank)
-    work = decode_work(w)
+def timed_steps(r, args, world, local, n_events):
+    """W warm-ups, then exactly K steps between barriers and synchronisations, with the
+    SM clock sampled meanwhile.  Returns (ms per step max over ranks, per-step phase
+    events, clock summary)."""
     for _ in range(args.warmup):
         r.step()
     torch.cuda.synchronize()
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_events)]
+          for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    # the bank (41 GB) is far larger than L2; the pooled keys (0.6 GB) too
     with ClockSampler(local) as clk:
         barrier(world)
         torch.cuda.synchronize()
@@ -325,167 +571,20 @@ def run_decode(args, world, rank, local):
         torch.cuda.synchronize()
         barrier(world)
     ms = max_over_ranks(start.elapsed_time(end) / args.steps, world)
-    peaks, peak_src = load_peaks()
-    sel_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
-    att_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
-    # algorithmic bytes: the selection reads the pooled-key bank once at 4 bytes per element
-    # (bf16 hi + lo planes, as exact as fp32 for the selection); the attention reads the
-    # selected K/V blocks once per (query, group)
-    kbar_bytes = float(w.nb * w.hkv * w.d * 4)
-    phases = {
-        "select": {"ms": sel_ms, "bytes": kbar_bytes,
-                   "kernel": "msa_decode_select_tiled (sample scan + threshold + full "
-                             "tensor-core scan + list merge)",
-                   # DRAM bytes of its scan kernels in one ncu capture of a 1.2M-token bank
-                   # (sample 10.5 MB + scan 79.5 MB for 18,750 blocks), scaled by blocks
-                   "traffic": (10.52e6 + 79.46e6) * w.nb / 18750},
-        "attend": {"ms": att_ms, "bytes": float(work["attn_bytes"]),
-                   "kernel": "msa_decode_attn_tiled (streamed attention + split combine)",
-                   # the attention kernel's DRAM bytes in the same capture (526.3 MB read,
-                   # 16.8 MB written); they depend on the selection, not on the bank size
-                   "traffic": 543.09e6 * w.n_query * w.hkv * w.topk / (64 * 8 * 32)},
-    }
-    dom = max(phases.values(), key=lambda x: x["ms"])
-    gbs = dom["bytes"] / (dom["ms"] * 1e-3) / 1e9
-    roof = {"bound": "hbm", "kernel": dom["kernel"], "achieved": round(gbs, 1),
-            "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
-            "peak_source": f"hbm_gbs of {peak_src}", "traffic": round(dom["traffic"]),
-            "traffic_source": "ncu capture of a 1.2M-token bank, scaled (see profiles/)",
-            "algorithmic_per_launch": dom["bytes"]}
-    phase_line = {k: {"us": round(v["ms"] * 1e3, 1),
-                      "gbs": round(v["bytes"] / (v["ms"] * 1e-3) / 1e9, 1)} for k, v in phases.items()}
-    e2e = None
-    if not args.no_e2e:
-        hq_ = r.q.cpu().pin_memory()
-        ho = torch.empty(r.o.shape, dtype=r.o.dtype).pin_memory()
-
-        def one():
-            r.q.copy_(hq_, non_blocking=True)
-            r.step()
-            ho.copy_(r.o, non_blocking=True)
-        for _ in range(args.warmup):
-            one()
-        torch.cuda.synchronize()
-        s_, e_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        s_.record()
-        for _ in range(args.steps):
-            one()
-        e_.record()
-        torch.cuda.synchronize()
-        ems = max_over_ranks(s_.elapsed_time(e_) / args.steps, world)
-        e2e = {"value": round(ems * 1e3, 1), "unit": "us/step", "ms_per_step": round(ems, 4),
-               "h2d_bytes_per_step": hq_.numel() * hq_.element_size(),
-               "d2h_bytes_per_step": ho.numel() * ho.element_size()}
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline_decode(w, r.q, seed=rank)
-    line = {
-        "metric": "decode us/step", "value": round(ms * 1e3, 1), "unit": "us/step",
-        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": round(ms, 4), "higher_is_better": False, "scaling": "weak",
-        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-        "config": {"workload": w.name, "n_query": w.n_query, "bank_tokens": w.seq, "hq": w.hq,
-                   "hkv": w.hkv, "d": w.d, "block": w.block, "topk": w.topk,
-                   "l2": "bank and pooled keys larger than L2, no flush",
-                   "parallelism": f"{world} independent banks, one per GPU"},
-        "phases": phase_line, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
-        "gpu_launches": r.launches_per_step * args.steps, "clocks": clk.summary(),
-        "device_error_bits": r.msa.read_device_error(r.ws),
-    }
-    if rank == 0:
-        print(json.dumps(line), flush=True)
+    return ms, ev, clk.summary()
 
 
-def run_ours(args, world, rank, local):
-    w = workload_of(args)
-    if w.kind != "prefill":
-        return run_decode(args, world, rank, local)
-    from block_sparse_top_mean_b200 import build
-    if rank == 0:
-        build.build()
-    barrier(world)
-    r = PrefillRunner(w, seed=rank)
-    attn_flops, score_flops = prefill_flops(w)
-    for _ in range(args.warmup):
-        r.step()
-    torch.cuda.synchronize()
-
-    # device-timed region: K steps, inputs resident in HBM (Q alone is larger than L2)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local) as clk:
-        barrier(world)
-        torch.cuda.synchronize()
-        start.record()
-        for i in range(args.steps):
-            r.step(ev[i])
-        end.record()
-        torch.cuda.synchronize()
-        barrier(world)
-    ms = start.elapsed_time(end) / args.steps
-    ms_max = max_over_ranks(ms, world)
-    phase = {n: statistics.mean(e[a].elapsed_time(e[a + 1]) for e in ev)
-             for a, n in enumerate(["pool_keys", "topk_select", "sparse_attn"])}
-    err = r.msa.read_device_error(r.ws)
-
-    peaks, peak_src = load_peaks()
-    value = world * (attn_flops + score_flops) / (ms_max * 1e-3) / 1e12
-    tokens_s = world * w.seq * w.batch / (ms_max * 1e-3)
-    attn_tflops = attn_flops / (phase["sparse_attn"] * 1e-3) / 1e12
-    peak = peaks["bf16_tflops_sustained"]
-    roof = {"bound": "tensor", "kernel": "sparse_attn", "achieved": round(attn_tflops, 2),
-            "peak": peak, "unit": "TFLOP/s", "frac": round(attn_tflops / peak, 4),
-            "peak_source": f"bf16_tflops_sustained of {peak_src}", "traffic": None,
-            "algorithmic_per_launch": attn_flops}
-
-    e2e = None
-    if not args.no_e2e:
-        e2e = measure_e2e(r, args, world, attn_flops + score_flops)
-    cpu = None
-    if not args.no_cpu_baseline and world == 1 and rank == 0:
-        cpu = cpu_baseline_prefill(w, r, attn_flops + score_flops)
-
-    line = {
-        "metric": "sparse-attn prefill TFLOP/s", "value": round(value, 3), "unit": "TFLOP/s",
-        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": round(ms_max, 3), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
-        "data": "synthetic",
-        "config": {"workload": w.name, "batch_per_gpu": w.batch, "seq": w.seq, "hq": w.hq,
-                   "hkv": w.hkv, "d": w.d, "block": w.block, "topk": w.topk,
-                   "l2": f"inputs larger than L2 (Q alone {w.batch * w.seq * w.hq * w.d * 2 / 2**30:.2f} GiB), no flush",
-                   "workspace_gib": round(r.ws.numel() / 2**30, 2),
-                   "attn_token_slabs": r.n_slabs,
-                   "parallelism": f"{world} independent sequences, one per GPU"},
-        "tokens_per_s": round(tokens_s, 1),
-        "flops_per_step": {"attention": attn_flops, "scoring": score_flops},
-        "phases_ms": {k: round(v, 3) for k, v in phase.items()},
-        "attn_phase_tflops": round(attn_tflops, 2),
-        "roofline": roof,
-        "cpu_baseline": cpu,
-        "e2e": e2e,
-        "gpu_launches": r.launches_per_step * args.steps,
-        "clocks": clk.summary(),
-        "device_error_bits": err,
-    }
-    if rank == 0:
-        print(json.dumps(line), flush=True)
-
-
-def measure_e2e(r: PrefillRunner, args, world, flops):
-    """Same step through the C ABI from pinned HOST buffers: H2D of q/k/v, the three
-    calls, D2H of o, all inside the device-timed region."""
-    hq_, hk_, hv_ = (x.cpu().pin_memory() for x in (r.q, r.k, r.v))
-    ho = torch.empty(r.o.shape, dtype=r.o.dtype).pin_memory()
-    h2d = sum(x.numel() * x.element_size() for x in (hq_, hk_, hv_))
-    d2h = ho.numel() * ho.element_size()
+def e2e_steps(r, args, world, inputs, output):
+    """The same step through the C ABI from pinned HOST buffers: H2D of `inputs`, the
+    calls, D2H of `output`, all inside the device-timed region.  Returns (ms, h2d, d2h)."""
+    hosts = [x.cpu().pin_memory() for x in inputs]
+    ho = torch.empty(output.shape, dtype=output.dtype).pin_memory()
 
     def one():
-        r.q.copy_(hq_, non_blocking=True)
-        r.k.copy_(hk_, non_blocking=True)
-        r.v.copy_(hv_, non_blocking=True)
+        for d_, h_ in zip(inputs, hosts):
+            d_.copy_(h_, non_blocking=True)
         r.step()
-        ho.copy_(r.o, non_blocking=True)
+        ho.copy_(output, non_blocking=True)
 
     for _ in range(max(1, args.warmup)):
         one()
@@ -498,143 +597,221 @@ def measure_e2e(r: PrefillRunner, args, world, flops):
     e.record()
     torch.cuda.synchronize()
     ms = max_over_ranks(s.elapsed_time(e) / args.steps, world)
-    return {"value": round(world * flops / (ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
-            "ms_per_step": round(ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    return ms, sum(x.numel() * x.element_size() for x in hosts), ho.numel() * ho.element_size()
 
 
-# ------------------------------------------------------------------ the oracle on the host
-
-def _oracle_rates(w: mi.Workload, K_host, Qv, Kv, Vv, kbar, n_blocks: int, n_tokens: int,
-                  seed: int):
-    """Times the oracle on a sample: pooling of n_blocks blocks and selection+attention of
-    n_tokens tokens (all groups; they read `kbar`, the oracle's own pooled keys computed
-    once outside the timing).  Returns (s_per_block, s_per_token, sample text)."""
-    import oracle
-    from threadpoolctl import threadpool_limits
-    rng = np.random.default_rng(seed)
-    blocks = rng.choice(w.nb, size=min(n_blocks, w.nb), replace=False)
-    toks = sorted(rng.choice(w.seq, size=min(n_tokens, w.seq), replace=False).tolist())
-    with threadpool_limits(limits=1):
-        t0 = time.perf_counter()
-        for j in blocks:
-            lo, hi = int(j) * w.block, min(w.seq, (int(j) + 1) * w.block)
-            oracle.pool_keys(K_host[:, lo:hi], w.block)
-        t1 = time.perf_counter()
-        t2 = time.perf_counter()
-        oracle.prefill_rows(Qv, Kv, Vv, w.block, w.topk, w.scale,
-                            rows=[(0, t) for t in toks], kbar=kbar)
-        t3 = time.perf_counter()
-    sample = (f"pooling of {len(blocks)} random blocks + selection and attention of "
-              f"{len(toks)} random tokens x {w.hkv} groups, extrapolated to the full "
-              f"workload ({w.nb} blocks, {w.seq} tokens); numpy fp64, 1 thread")
-    return (t1 - t0) / len(blocks), (t3 - t2) / len(toks), sample
+# DRAM bytes of the prefill attention phase (index inversion, tiles, merge) per selected
+# (token, group, block) entry, from an ncu capture of the 1M workload shortened to 128K
+# tokens (inputs larger than L2): see profiles/.  None until measured.
+PREFILL_ATTN_DRAM_PER_ENTRY = None
 
 
-def cpu_baseline_prefill(w, r, flops, n_blocks=64, n_tokens=96):
-    sys.path.insert(0, os.path.join(ROOT, "tests"))
-    from parity_util import HostView
-    import oracle
-    K_host = r.k.float().cpu().numpy()
-    kbar = oracle.pool_keys(K_host, w.block)
-    spb, spt, sample = _oracle_rates(w, K_host, HostView(r.q), K_host, HostView(r.v), kbar,
-                                     n_blocks, n_tokens, 0)
-    t_full = spb * w.nb * w.batch + spt * w.seq * w.batch
-    return {"value": round(flops / t_full / 1e12, 6), "unit": "TFLOP/s", "cores": 1,
-            "kind": "oracle", "sample": sample, "extrapolated_s_per_step": round(t_full, 1)}
-
-
-def cpu_baseline_decode(w, q, seed=0, n_s=2):
-    """Oracle decode of n_s queries (all groups) on one host core, extrapolated to
-    n_query.  The fp64 pooled keys of a 10M-token bank would take minutes to build on the
-    host; random values of the right shape stand in (only the time is measured), while
-    K and V are the workload's bank, generated block by block as the oracle reads them."""
-    import oracle
-    from threadpoolctl import threadpool_limits
-    kbar = mi.normal((w.nb, w.hkv, w.d), 7, 7, "cpu", torch.float32).numpy().astype(np.float64)
-    Qd = q.float().cpu().numpy()
-    K, V = mi.lazy_decode_bank(w, seed)
-    with threadpool_limits(limits=1):
-        t0 = time.perf_counter()
-        oracle.decode_rows(Qd, kbar, K, V, w.seq, w.block, w.topk, w.scale,
-                           queries=list(range(n_s)))
-        t = (time.perf_counter() - t0) / n_s * w.n_query
-    sample = (f"{n_s} of {w.n_query} queries (all {w.hkv} groups), extrapolated to "
-              f"{w.n_query}; numpy fp64, 1 thread; random stand-in pooled keys")
-    return {"value": round(t * 1e6, 1), "unit": "us/step", "cores": 1, "kind": "oracle",
-            "sample": sample}
-
-
-def run_reference_decode(args, world, w):
-    """The oracle arm for decode: a bounded sample of the queries per step."""
-    q, _, _ = mi.decode_inputs(w, device="cpu", seed=0, bank=False)
-    times = []
-    for s_ in range(args.warmup + args.steps):
-        qs = torch.roll(q, shifts=-2 * s_, dims=0)
-        cb = cpu_baseline_decode(w, qs)
-        if s_ >= args.warmup:
-            times.append(cb["value"] * 1e-6)
-    t = statistics.mean(times)
+def bench_prefill(w, args, world, rank, local, pool):
+    r = PrefillRunner(w, seed=rank)
+    attn_flops, score_flops = prefill_flops(w)
+    ms, ev, clocks = timed_steps(r, args, world, local, 4)
+    phase = {n: statistics.mean(e[a].elapsed_time(e[a + 1]) for e in ev)
+             for a, n in enumerate(["pool_keys", "topk_select", "sparse_attn"])}
+    err = r.msa.read_device_error(r.ws)
+    peaks, peak_src = load_peaks()
+    value = world * (attn_flops + score_flops) / (ms * 1e-3) / 1e12
+    tokens_s = world * w.seq * w.batch / (ms * 1e-3)
+    attn_tflops = attn_flops / (phase["sparse_attn"] * 1e-3) / 1e12
+    peak = peaks["bf16_tflops_sustained"]
+    entries = prefill_entries(w)
+    traffic = (None if PREFILL_ATTN_DRAM_PER_ENTRY is None
+               else round(PREFILL_ATTN_DRAM_PER_ENTRY * entries))
+    roof = {"bound": "tensor",
+            "kernel": "msa_sparse_attn_fwd (index inversion, tcgen05 tiles, partial merge)",
+            "achieved": round(attn_tflops, 2), "peak": peak, "unit": "TFLOP/s",
+            "frac": round(attn_tflops / peak, 4),
+            "peak_source": f"bf16_tflops_sustained of {peak_src}", "traffic": traffic,
+            "traffic_source": "ncu dram bytes of the phase's kernels on the 1M workload "
+                              "shortened to 128K tokens, per selected (token, group, block) "
+                              "entry, times this workload's entries",
+            "algorithmic_per_launch": attn_flops, "selected_entries": entries}
+    e2e = None
+    if not args.no_e2e:
+        ems, h2d, d2h = e2e_steps(r, args, world, [r.q, r.k, r.v], r.o)
+        e2e = {"value": round(world * (attn_flops + score_flops) / (ems * 1e-3) / 1e12, 3),
+               "unit": "TFLOP/s", "ms_per_step": round(ems, 3), "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h}
+    cpu = None
+    if pool is not None:
+        orc = PrefillOracle(pool, w, r.q, r.k, r.v)
+        t, sample = orc.step_seconds(192, 0)
+        pool.clear_files()
+        cpu = {"value": round((attn_flops + score_flops) / t / 1e12, 6), "unit": "TFLOP/s",
+               "cores": pool.n, "kind": "oracle", "sample": sample,
+               "extrapolated_s_per_step": round(t, 1)}
     line = {
-        "impl": "reference", "metric": "decode us/step", "value": round(t * 1e6, 1),
-        "unit": "us/step", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": t * 1e3, "higher_is_better": False, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "n_query": w.n_query, "bank_tokens": w.seq, "hq": w.hq,
-                   "hkv": w.hkv, "d": w.d, "block": w.block, "topk": w.topk,
-                   "parallelism": "host oracle, rank 0 only"},
-        "cpu_baseline": dict(cb, value=round(t * 1e6, 1)),
-        "e2e": {"value": round(t * 1e6, 1), "unit": "us/step", "h2d_bytes_per_step": 0,
-                "d2h_bytes_per_step": 0},
-    }
-    print(json.dumps(line), flush=True)
-
-
-def run_reference(args, world, rank):
-    """The base contract's reference arm for this method: the fp64 CPU oracle, timed on the
-    host cores on a bounded sample of the same workload."""
-    if rank != 0:
-        return
-    w = workload_of(args)
-    if w.kind == "decode":
-        return run_reference_decode(args, world, w)
-    attn, score = prefill_flops(w)
-    # inputs generated on the host in the same way (bounded: only what the sample touches)
-    dev = "cuda" if torch.cuda.is_available() else "cpu"
-    q, k, v = mi.prefill_inputs(w, device=dev, seed=0)
-    sys.path.insert(0, os.path.join(ROOT, "tests"))
-    from parity_util import HostView
-    import oracle
-    K_host = k.float().cpu().numpy()
-    kbar = oracle.pool_keys(K_host, w.block)
-    times = []
-    sample = ""
-    for s in range(args.warmup + args.steps):
-        spb, spt, sample = _oracle_rates(w, K_host, HostView(q), K_host, HostView(v), kbar,
-                                         16, 24, s)
-        if s >= args.warmup:
-            times.append(spb * w.nb * w.batch + spt * w.seq * w.batch)
-    t = statistics.mean(times)
-    value = (attn + score) / t / 1e12
-    line = {
-        "impl": "reference", "metric": "sparse-attn prefill TFLOP/s", "value": value,
-        "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": t * 1e3, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "metric": "sparse-attn prefill TFLOP/s", "value": round(value, 3), "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
+        "data": "synthetic",
         "config": {"workload": w.name, "batch_per_gpu": w.batch, "seq": w.seq, "hq": w.hq,
                    "hkv": w.hkv, "d": w.d, "block": w.block, "topk": w.topk,
-                   "parallelism": "host oracle, rank 0 only"},
-        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+                   "planted_frac": w.planted_frac,
+                   "l2": f"inputs larger than L2 (Q alone {w.batch * w.seq * w.hq * w.d * 2 / 2**30:.2f} GiB), no flush",
+                   "workspace_gib": round(r.ws.numel() / 2**30, 2),
+                   "attn_token_slabs": r.n_slabs,
+                   "parallelism": f"{world} independent sequences, one per GPU"},
+        "tokens_per_s": round(tokens_s, 1),
+        "flops_per_step": {"attention": attn_flops, "scoring": score_flops},
+        "phases_ms": {k: round(v, 3) for k, v in phase.items()},
+        "attn_phase_tflops": round(attn_tflops, 2),
+        "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": r.launches_per_step * args.steps, "clocks": clocks,
+        "device_error_bits": err,
+    }
+    del r
+    torch.cuda.empty_cache()
+    return line
+
+
+def bench_decode(w, args, world, rank, local, pool):
+    r = DecodeRunner(w, seed=rank)
+    work = decode_work(w)
+    # the encoded bank (41 GB) and its pooled-key planes (0.6 GB) are larger than L2
+    ms, ev, clocks = timed_steps(r, args, world, local, 3)
+    peaks, peak_src = load_peaks()
+    sel_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    att_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    planes_read = float(w.nb * w.hkv * w.d * 4)
+    phases = {
+        "select": {"ms": sel_ms, "bytes": work["score_bytes"],
+                   "kernel": "msa_decode_select_tiled (sample scan + threshold + full "
+                             "tensor-core scan + list merge)",
+                   # DRAM bytes of its scan kernels in one ncu capture of a 1.2M-token bank
+                   # (sample 10.5 MB + scan 79.5 MB for 18,750 blocks), scaled by blocks
+                   "traffic": (10.52e6 + 79.46e6) * w.nb / 18750},
+        "attend": {"ms": att_ms, "bytes": work["attn_bytes"],
+                   "kernel": "msa_decode_attn_tiled (streamed attention + split combine)",
+                   # the attention kernel's DRAM bytes in the same capture (526.3 MB read,
+                   # 16.8 MB written); they depend on the selection, not on the bank size
+                   "traffic": 543.09e6 * w.n_query * w.hkv * w.topk / (64 * 8 * 32)},
+    }
+    dom = phases["select"]
+    gbs = dom["bytes"] / (dom["ms"] * 1e-3) / 1e9
+    roof = {"bound": "hbm", "kernel": dom["kernel"], "achieved": round(gbs, 1),
+            "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
+            "peak_source": f"hbm_gbs of {peak_src}", "traffic": round(dom["traffic"]),
+            "traffic_source": "ncu capture of a 1.2M-token bank, scaled (see profiles/)",
+            "algorithmic_per_launch": dom["bytes"],
+            "algorithmic_note": "one bf16 plane of the pooled keys; the exact selection "
+                                "streams both the hi and lo planes",
+            "planes_read_bytes": planes_read,
+            "planes_read_gbs": round(planes_read / (dom["ms"] * 1e-3) / 1e9, 1)}
+    phase_line = {k: {"us": round(v["ms"] * 1e3, 1),
+                      "gbs": round(v["bytes"] / (v["ms"] * 1e-3) / 1e9, 1)}
+                  for k, v in phases.items()}
+    e2e = None
+    if not args.no_e2e:
+        ems, h2d, d2h = e2e_steps(r, args, world, [r.q], r.o)
+        e2e = {"value": round(ems * 1e3, 1), "unit": "us/step", "ms_per_step": round(ems, 4),
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    cpu = None
+    if pool is not None:
+        t, sample = DecodeOracle(pool, w, r.q, seed=rank).step_seconds(2, 0)
+        pool.clear_files()
+        cpu = {"value": round(t * 1e6, 1), "unit": "us/step", "cores": pool.n,
+               "kind": "oracle", "sample": sample}
+    line = {
+        "metric": "decode us/step", "value": round(ms * 1e3, 1), "unit": "us/step",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms, 4), "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": {"workload": w.name, "n_query": w.n_query, "bank_tokens": w.seq, "hq": w.hq,
+                   "hkv": w.hkv, "d": w.d, "block": w.block, "topk": w.topk,
+                   "l2": "bank and pooled keys larger than L2, no flush",
+                   "parallelism": f"{world} independent banks, one per GPU"},
+        "phases": phase_line, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": r.launches_per_step * args.steps, "clocks": clocks,
+        "device_error_bits": r.msa.read_device_error(r.ws),
+    }
+    del r
+    torch.cuda.empty_cache()
+    return line
+
+
+def bench_one(name, args, world, rank, local, pool):
+    w = workload_of(name, args.seq)
+    return (bench_prefill if w.kind == "prefill" else bench_decode)(w, args, world, rank, local,
+                                                                    pool)
+
+
+def run_ours(args, world, rank, local, pool):
+    from block_sparse_top_mean_b200 import build
+    if rank == 0:
+        build.build()
+    barrier(world)
+    line = bench_one(args.workload, args, world, rank, local, pool)
+    if args.default_set:
+        line["workloads"] = {}
+        for name in DEFAULT_EXTRAS:
+            sub = bench_one(name, args, world, rank, local, pool)
+            sub.pop("n_gpus", None)
+            line["workloads"][name] = sub
+        line["gpu_launches_all_workloads"] = line["gpu_launches"] + sum(
+            s["gpu_launches"] for s in line["workloads"].values())
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ the reference arm
+
+def run_reference(args, world, rank, pool):
+    """The base contract's reference arm for this method: the fp64 CPU oracle, timed on the
+    host cores, each step a bounded sample of the same workload (rank 0 only)."""
+    if rank != 0:
+        return
+    w = workload_of(args.workload, args.seq)
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    times, sample = [], ""
+    if w.kind == "decode":
+        q, _, _ = mi.decode_inputs(w, device="cpu", seed=0, bank=False)
+        orc = DecodeOracle(pool, w, q)
+        for s_ in range(args.warmup + args.steps):
+            t, sample = orc.step_seconds(1, s_)
+            if s_ >= args.warmup:
+                times.append(t)
+        t = statistics.mean(times)
+        value, unit, hib, metric = round(t * 1e6, 1), "us/step", False, "decode us/step"
+        cfg = {"workload": w.name, "n_query": w.n_query, "bank_tokens": w.seq, "hq": w.hq,
+               "hkv": w.hkv, "d": w.d, "block": w.block, "topk": w.topk}
+    else:
+        attn, score = prefill_flops(w)
+        q, k, v = mi.prefill_inputs(w, device=dev, seed=0)
+        orc = PrefillOracle(pool, w, q, k, v)
+        del k, v
+        for s_ in range(args.warmup + args.steps):
+            t, sample = orc.step_seconds(12, s_)
+            if s_ >= args.warmup:
+                times.append(t)
+        t = statistics.mean(times)
+        value, unit, hib, metric = (attn + score) / t / 1e12, "TFLOP/s", True, \
+            "sparse-attn prefill TFLOP/s"
+        cfg = {"workload": w.name, "batch_per_gpu": w.batch, "seq": w.seq, "hq": w.hq,
+               "hkv": w.hkv, "d": w.d, "block": w.block, "topk": w.topk,
+               "planted_frac": w.planted_frac}
+    cfg["parallelism"] = "host oracle, rank 0 only"
+    line = {
+        "impl": "reference", "metric": metric, "value": value, "unit": unit, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3,
+        "higher_is_better": hib, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": cfg,
+        "cpu_baseline": {"value": value, "unit": unit, "cores": pool.n, "kind": "oracle",
                          "sample": sample},
-        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
-                "d2h_bytes_per_step": 0},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 
 
-def workload_of(args) -> mi.Workload:
-    w = mi.WORKLOADS[args.workload]
-    if args.seq is not None:
-        w = w.with_(name=f"{w.name}@seq{args.seq}", seq=args.seq)
+def workload_of(name: str, seq) -> mi.Workload:
+    w = mi.WORKLOADS[name]
+    if seq is not None:
+        w = w.with_(name=f"{w.name}@seq{seq}", seq=seq)
     return w
 
 
@@ -644,7 +821,9 @@ def main():
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="prefill_1m_b256_k16", choices=list(mi.WORKLOADS))
+    ap.add_argument("--workload", default=None, choices=list(mi.WORKLOADS),
+                    help="one workload only (default: the 1M prefill as the headline plus "
+                         "the 128K planted prefill and the 10M-token decode)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--seq", type=int, default=None,
@@ -652,13 +831,24 @@ def main():
                          "captures only; the JSON line then names the changed workload)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
+    args.default_set = args.workload is None
+    if args.default_set:
+        args.workload = "prefill_1m_b256_k16"
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    # host workers for the oracle, forked before this process makes its first CUDA call
+    pool = None
+    if rank == 0 and (args.impl == "reference" or (world == 1 and not args.no_cpu_baseline)):
+        pool = OraclePool(OraclePool.cores())
     world, rank, local = dist_setup()
     try:
         if args.impl == "reference":
-            run_reference(args, world, rank)
+            run_reference(args, world, rank, pool)
         else:
-            run_ours(args, world, rank, local)
+            run_ours(args, world, rank, local, pool)
     finally:
+        if pool is not None:
+            pool.close()
         if world > 1:
             import torch.distributed as dist
             dist.destroy_process_group()

@@ -35,7 +35,7 @@ def test_oracle_never_reaches_into_the_cuda_path():
 
 def test_bench_uses_the_oracle_only_in_its_cpu_legs():
     tree = ast.parse(open(os.path.join(ROOT, "bench.py")).read())
-    allowed = re.compile(r"^(cpu_baseline_\w+|_oracle_rates|run_reference\w*)$")
+    allowed = re.compile(r"^(_w_(pool|prefill|decode)|run_reference\w*)$")
     for node in ast.walk(tree):
         if isinstance(node, ast.FunctionDef):
             for sub in ast.walk(node):
