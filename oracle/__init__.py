@@ -18,3 +18,4 @@ from .msa_sharded import (  # noqa: F401
     decode_rows_sharded,
 )
 from .msa_backward import attend_row_backward, prefill_backward  # noqa: F401
+from .msa_docs import doc_positions, prefill_varlen_rows, rope_angles, rope_docwise  # noqa: F401

@@ -13,6 +13,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 PINS = "test_oracle_pins.py"
 SHARDED = "test_oracle_sharded.py"
 BACKWARD = "test_oracle_backward.py"
+DOCS = "test_oracle_docs.py"
 
 MUTATIONS = [
     # (file, original text, planted mistake, pins that must catch it)
@@ -46,6 +47,14 @@ MUTATIONS = [
     ("msa_backward.py", "dk = scale * (dS.T @ q)", "dk = (dS.T @ q)", BACKWARD),
     ("msa_backward.py", "dv = P.T @ g", "dv = P.T @ g[::-1]", BACKWARD),
     ("msa_backward.py", "np.add.at(dK[b, :, g], p, dk)", "dK[b, p, g] = dk", BACKWARD),
+    ("msa_docs.py", "pos[a:b] = np.arange(b - a)", "pos[a:b] = np.arange(a, b)", DOCS),  # no reset
+    ("msa_docs.py", "theta = base ** (-2.0 * i / d)", "theta = base ** (-1.0 * i / d)", DOCS),
+    ("msa_docs.py", "[a * c - b * s, b * c + a * s]", "[a * c + b * s, b * c - a * s]",
+     DOCS),                                                                          # direction
+    ("msa_docs.py", "a, b = x[..., :half], x[..., half:]", "a, b = x[..., 0::2], x[..., 1::2]",
+     DOCS),                                                                          # pairing
+    ("msa_docs.py", "res = prefill_rows(Q[None, a:b], K[None, a:b], V[None, a:b]",
+     "res = prefill_rows(Q[None, a:b], K[None, 0:b - a], V[None, a:b]", DOCS),       # wrong doc
 ]
 
 
@@ -74,7 +83,7 @@ def _copy_and_run(tmp_path, pins, fname=None, old=None, new=None):
                           cwd=tmp_path, env=env, capture_output=True, text=True, timeout=600)
 
 
-@pytest.mark.parametrize("pins", [PINS, SHARDED, BACKWARD])
+@pytest.mark.parametrize("pins", [PINS, SHARDED, BACKWARD, DOCS])
 def test_unchanged_copy_passes(tmp_path, pins):
     """Control: the copied pins pass on the unchanged oracle, so a failure below is the
     planted mistake's doing."""
