@@ -600,10 +600,14 @@ def e2e_steps(r, args, world, inputs, output):
     return ms, sum(x.numel() * x.element_size() for x in hosts), ho.numel() * ho.element_size()
 
 
-# DRAM bytes of the prefill attention phase (index inversion, tiles, merge) per selected
-# (token, group, block) entry, from an ncu capture of the 1M workload shortened to 128K
-# tokens (inputs larger than L2): see profiles/.  None until measured.
-PREFILL_ATTN_DRAM_PER_ENTRY = None
+# DRAM bytes (read + write) of the prefill attention phase per selected (token, group,
+# block) entry, from one ncu capture of the 1M workload shortened to 32K tokens (Q 256 MiB,
+# larger than L2; 3,948,544 entries): tiles kernel 2006.0, partial merge 1112.4, index
+# inversion 8.9 (profiles/prefill_32k_b256_k16_attn_dram.md).  The per-entry traffic does
+# not depend on the sequence length at this block size: every block is selected by about
+# 4096 entries per group at 32K and at 1M alike.
+PREFILL_ATTN_DRAM_PER_ENTRY = {"attn_tiles_kernel": 2006.0, "merge_partials_kernel": 1112.4,
+                               "index inversion": 8.9}
 
 
 def bench_prefill(w, args, world, rank, local, pool):
@@ -619,16 +623,19 @@ def bench_prefill(w, args, world, rank, local, pool):
     attn_tflops = attn_flops / (phase["sparse_attn"] * 1e-3) / 1e12
     peak = peaks["bf16_tflops_sustained"]
     entries = prefill_entries(w)
-    traffic = (None if PREFILL_ATTN_DRAM_PER_ENTRY is None
-               else round(PREFILL_ATTN_DRAM_PER_ENTRY * entries))
+    per_entry = sum(PREFILL_ATTN_DRAM_PER_ENTRY.values())
+    traffic = round(per_entry * entries)
     roof = {"bound": "tensor",
             "kernel": "msa_sparse_attn_fwd (index inversion, tcgen05 tiles, partial merge)",
             "achieved": round(attn_tflops, 2), "peak": peak, "unit": "TFLOP/s",
             "frac": round(attn_tflops / peak, 4),
             "peak_source": f"bf16_tflops_sustained of {peak_src}", "traffic": traffic,
             "traffic_source": "ncu dram bytes of the phase's kernels on the 1M workload "
-                              "shortened to 128K tokens, per selected (token, group, block) "
+                              "shortened to 32K tokens, per selected (token, group, block) "
                               "entry, times this workload's entries",
+            "traffic_per_entry": PREFILL_ATTN_DRAM_PER_ENTRY,
+            "traffic_floor_ms": round(traffic / (peaks["hbm_gbs"] * 1e9) * 1e3, 2),
+            "algorithmic_bytes": float(w.batch * w.seq * (2 * w.hq + 2 * w.hkv) * w.d * 2),
             "algorithmic_per_launch": attn_flops, "selected_entries": entries}
     e2e = None
     if not args.no_e2e:
