@@ -15,7 +15,7 @@ import torch
 from . import _lib
 from ._lib import (  # noqa: F401
     MsaError, MsaParams, OP_DECODE, OP_PREFILL, OP_SPARSE_ATTN, OP_TOPK_SELECT,
-    OP_SPARSE_ATTN_MIN, OP_PREFILL_MIN,
+    OP_SPARSE_ATTN_MIN, OP_PREFILL_MIN, OP_DECODE_OFFLOAD,
     DEVERR_IDX_RANGE, DEVERR_TIMEOUT, MSA_F32, MSA_BF16,
 )
 
@@ -24,7 +24,8 @@ __all__ = [
     "prefill_fwd", "decode_fwd", "decode_fwd_static", "encode_bank", "decode_fwd_tiled",
     "decode_select_tiled", "decode_attn_tiled", "attn_slab_tokens",
     "read_device_error",
-    "clear_device_error", "version", "exp2_poly_eval",
+    "clear_device_error", "version", "exp2_poly_eval", "rope_docwise", "prefill_varlen_fwd",
+    "decode_select_shard", "decode_merge_shards", "decode_combine_shards", "decode_fwd_offload",
     "MsaError", "MsaParams",
 ]
 
@@ -301,3 +302,125 @@ def exp2_poly_eval(x: torch.Tensor) -> torch.Tensor:
     _lib.check("msa_exp2_poly_eval", _lib.load().msa_exp2_poly_eval(
         _ptr(x), _ptr(y), x.numel(), _stream(x.device)))
     return y
+
+
+def rope_docwise(q: torch.Tensor, k: torch.Tensor, cu_seqlens: torch.Tensor, base: float):
+    """Rotates packed q [T, hq, d] and k [T, hkv, d] in place by each token's position in
+    its own document (cu_seqlens: int32 CUDA tensor of the n_docs + 1 boundaries)."""
+    T, hq, d = q.shape
+    hkv = k.shape[1]
+    if cu_seqlens.dtype != torch.int32:
+        raise ValueError("cu_seqlens must be int32")
+    p = params(batch=1, seq=T, hq=hq, hkv=hkv, d=d, block=1, topk=1, scale=1.0, dtype=q.dtype)
+    _lib.check("msa_rope_docwise", _lib.load().msa_rope_docwise(
+        ctypes.byref(p), _ptr(cu_seqlens), cu_seqlens.numel() - 1, _ptr(q), _ptr(k),
+        float(base), _stream(q.device)))
+    return q, k
+
+
+def varlen_workspace(q, k, cu_seqlens, block: int, topk: int, minimum: bool = False):
+    """A workspace for prefill_varlen_fwd (sized for the longest document)."""
+    T, hq, d = q.shape
+    longest = max(int(b) - int(a) for a, b in zip(cu_seqlens[:-1], cu_seqlens[1:]))
+    p = params(batch=1, seq=max(1, longest), hq=hq, hkv=k.shape[1], d=d, block=block, topk=topk,
+               scale=1.0, dtype=q.dtype)
+    return workspace(p, OP_PREFILL_MIN if minimum else OP_PREFILL, device=q.device)
+
+
+def prefill_varlen_fwd(q, k, v, cu_seqlens, block: int, topk: int, scale=None, want_lse=True,
+                       ws=None):
+    """Causal prefill of packed documents (q [T, hq, d], k/v [T, hkv, d]; cu_seqlens a host
+    sequence of the n_docs + 1 boundaries).  Returns (o [T, hq, d], lse, idx) with idx and
+    lse in the per-document layout of msa_prefill_varlen_fwd (flat tensors)."""
+    T, hq, d = q.shape
+    hkv = k.shape[1]
+    cu = [int(x) for x in cu_seqlens]
+    p = params(batch=1, seq=T, hq=hq, hkv=hkv, d=d, block=block, topk=topk,
+               scale=scale if scale is not None else d ** -0.5, dtype=q.dtype)
+    o = torch.empty_like(q)
+    lse = torch.empty(T * hq, dtype=torch.float32, device=q.device) if want_lse else None
+    idx = torch.empty(T * hkv * topk, dtype=torch.int32, device=q.device)
+    if ws is None:
+        ws = varlen_workspace(q, k, cu, block, topk)
+    cu_host = (ctypes.c_int64 * len(cu))(*cu)
+    _lib.check("msa_prefill_varlen_fwd", _lib.load().msa_prefill_varlen_fwd(
+        ctypes.byref(p), cu_host, len(cu) - 1, _ptr(q), _ptr(k), _ptr(v), _ptr(idx), _ptr(o),
+        _ptr(lse), _ptr(ws), ws.numel(), _stream(q.device)))
+    return o, lse, idx
+
+
+def decode_select_shard(q, kbar_tiles, seq: int, hkv: int, block: int, topk: int,
+                        block_offset: int, ws=None, keys=None):
+    """Memory Parallel step 1: the best topk keys per (query, group) of one bank shard of
+    `seq` tokens whose first block has bank-wide id block_offset.  Returns keys
+    [n_query, hkv, topk] as int64 bit patterns (score bits above ~block id; 0 = empty)."""
+    nq = q.shape[0]
+    p = _bank_params(q, seq, hkv, block, topk, None)
+    if keys is None:
+        keys = torch.empty(nq, hkv, topk, dtype=torch.int64, device=q.device)
+    if ws is None:
+        ws = workspace(p, OP_DECODE, nq, device=q.device)
+    _lib.check("msa_decode_select_shard", _lib.load().msa_decode_select_shard(
+        ctypes.byref(p), nq, _ptr(q), _ptr(kbar_tiles), int(block_offset), _ptr(keys),
+        _ptr(ws), ws.numel(), _stream(q.device)))
+    return keys
+
+
+def decode_merge_shards(keys_all, hq: int, d: int, block_begin: int, block_count: int,
+                        dtype=torch.bfloat16, idx=None, idx_local=None):
+    """Memory Parallel step 2: keys_all [world, n_query, hkv, topk] (all ranks' lists in
+    rank order) -> (idx [n_query, hkv, topk] bank-wide, idx_local: the ids local to the
+    shard [block_begin, block_begin + block_count) of the blocks it owns, -1 elsewhere)."""
+    world, nq, hkv, topk = keys_all.shape
+    p = params(batch=1, seq=1, hq=hq, hkv=hkv, d=d, block=1, topk=topk, scale=1.0, dtype=dtype)
+    dev = keys_all.device
+    if idx is None:
+        idx = torch.empty(nq, hkv, topk, dtype=torch.int32, device=dev)
+    if idx_local is None:
+        idx_local = torch.empty_like(idx)
+    _lib.check("msa_decode_merge_shards", _lib.load().msa_decode_merge_shards(
+        ctypes.byref(p), nq, _ptr(keys_all), world, int(block_begin), int(block_count),
+        _ptr(idx), _ptr(idx_local), _stream(dev)))
+    return idx, idx_local
+
+
+def decode_combine_shards(o_parts, lse_parts, hkv: int, o=None, lse=None):
+    """Memory Parallel step 4: partials o [world, n_query, hq, d] and lse [world, n_query,
+    hq] -> the softmax over the whole selection (o [n_query, hq, d], lse [n_query, hq])."""
+    world, nq, hq, d = o_parts.shape
+    p = params(batch=1, seq=1, hq=hq, hkv=hkv, d=d, block=1, topk=1, scale=1.0,
+               dtype=o_parts.dtype)
+    if o is None:
+        o = torch.empty(nq, hq, d, dtype=o_parts.dtype, device=o_parts.device)
+    if lse is None:
+        lse = torch.empty(nq, hq, dtype=torch.float32, device=o_parts.device)
+    _lib.check("msa_decode_combine_shards", _lib.load().msa_decode_combine_shards(
+        ctypes.byref(p), nq, _ptr(o_parts), _ptr(lse_parts), world, _ptr(o), _ptr(lse),
+        _stream(o_parts.device)))
+    return o, lse
+
+
+def decode_fwd_offload(q, kbar_tiles, k_tiles_host, v_tiles_host, seq: int, hkv: int, block: int,
+                       topk: int, scale=None, want_lse=True, ws=None, out=None):
+    """decode_fwd_tiled with the encoded K/V images in PINNED host memory (k_tiles_host,
+    v_tiles_host: pinned CPU uint8 tensors from encode_bank); the pooled-key planes
+    (kbar_tiles) in HBM.  Selected blocks are fetched over PCIe into a staging bank in the
+    workspace."""
+    nq, hq, d = q.shape
+    p = _bank_params(q, seq, hkv, block, topk, scale)
+    for t in (k_tiles_host, v_tiles_host):
+        if t.is_cuda or not t.is_pinned():
+            raise ValueError("k_tiles_host / v_tiles_host must be pinned host tensors")
+    if out is not None:
+        o, lse, idx = out
+    else:
+        o = torch.empty_like(q)
+        lse = torch.empty(nq, hq, dtype=torch.float32, device=q.device) if want_lse else None
+        idx = torch.empty(nq, hkv, topk, dtype=torch.int32, device=q.device)
+    if ws is None:
+        ws = workspace(p, OP_DECODE_OFFLOAD, nq, device=q.device)
+    _lib.check("msa_decode_fwd_offload", _lib.load().msa_decode_fwd_offload(
+        ctypes.byref(p), nq, _ptr(q), _ptr(kbar_tiles),
+        ctypes.c_void_p(k_tiles_host.data_ptr()), ctypes.c_void_p(v_tiles_host.data_ptr()),
+        _ptr(idx), _ptr(o), _ptr(lse), _ptr(ws), ws.numel(), _stream(q.device)))
+    return o, lse, idx

@@ -6,14 +6,15 @@ from __future__ import annotations
 
 import ctypes
 import os
-from ctypes import POINTER, c_char_p, c_float, c_int32, c_int64, c_size_t, c_void_p
+from ctypes import POINTER, c_char_p, c_double, c_float, c_int32, c_int64, c_size_t, c_void_p
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmsa_b200.so")
 
 MSA_OK, MSA_ERR_INVALID_ARG, MSA_ERR_UNSUPPORTED, MSA_ERR_WORKSPACE, MSA_ERR_CUDA, \
     MSA_ERR_DEVICE, MSA_ERR_TIMEOUT = range(7)
 MSA_F32, MSA_BF16 = 0, 1
-OP_TOPK_SELECT, OP_SPARSE_ATTN, OP_PREFILL, OP_DECODE, OP_SPARSE_ATTN_MIN, OP_PREFILL_MIN = range(6)
+OP_TOPK_SELECT, OP_SPARSE_ATTN, OP_PREFILL, OP_DECODE, OP_SPARSE_ATTN_MIN, OP_PREFILL_MIN, \
+    OP_DECODE_OFFLOAD = range(7)
 DEVERR_IDX_RANGE, DEVERR_TIMEOUT = 0x1, 0x2
 
 # Every symbol include/msa.h declares, with (restype, argtypes).
@@ -52,6 +53,20 @@ SIGNATURES = {
     "msa_workspace_size": (c_size_t, [c_void_p, c_int32, c_int64]),
     "msa_get_device_status": (c_int32, [c_void_p, c_void_p]),
     "msa_exp2_poly_eval": (c_int32, [c_void_p, c_void_p, c_int64, c_void_p]),
+    "msa_decode_select_shard": (c_int32, [c_void_p, c_int64, c_void_p, c_void_p, c_int64,
+                                          c_void_p, c_void_p, c_size_t, c_void_p]),
+    "msa_decode_merge_shards": (c_int32, [c_void_p, c_int64, c_void_p, c_int64, c_int64,
+                                          c_int64, c_void_p, c_void_p, c_void_p]),
+    "msa_decode_combine_shards": (c_int32, [c_void_p, c_int64, c_void_p, c_void_p, c_int64,
+                                            c_void_p, c_void_p, c_void_p]),
+    "msa_decode_fwd_offload": (c_int32, [c_void_p, c_int64, c_void_p, c_void_p, c_void_p,
+                                         c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                         c_size_t, c_void_p]),
+    "msa_rope_docwise": (c_int32, [c_void_p, c_void_p, c_int64, c_void_p, c_void_p, c_double,
+                                   c_void_p]),
+    "msa_prefill_varlen_fwd": (c_int32, [c_void_p, c_void_p, c_int64, c_void_p, c_void_p,
+                                         c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                         c_size_t, c_void_p]),
 }
 
 

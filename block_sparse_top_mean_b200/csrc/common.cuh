@@ -108,9 +108,22 @@ cudaError_t launch_topk_decode(const Shape& s, int64_t n_query, const void* q, c
 // bank's pooled keys as bf16 hi/lo planes; workspace: per-CTA candidate lists.
 bool tc_decode_supported(const Shape& s);
 size_t topk_decode_tc_ws_bytes(const Shape& s, int64_t n_query);
+// With `keys` given, writes instead of idx the best topk 64-bit keys per (query, group)
+// [n_query, hkv, topk], sorted descending, block ids raised by block_offset (a shard of a
+// bank reporting bank-wide ids).
 cudaError_t launch_topk_decode_tc(const Shape& s, int64_t n_query, const void* q,
                                   const void* kbar_hi, const void* kbar_lo,
                                   const void* kbar_tiles, int32_t* idx, void* ws, int* err,
+                                  cudaStream_t st, uint64_t* keys = nullptr,
+                                  int64_t block_offset = 0);
+
+// Memory Parallel decode (memory_parallel.cu): merge of the shards' key lists into the
+// bank-wide selection and this shard's owned local ids; log-sum-exp combine of partials.
+cudaError_t launch_merge_shard_keys(const uint64_t* keys, int64_t world, int64_t rows,
+                                    int topk, int64_t block_begin, int64_t block_count,
+                                    int32_t* idx, int32_t* idx_local, cudaStream_t st);
+cudaError_t launch_combine_shards(const void* o_parts, const float* lse_parts, int64_t world,
+                                  int64_t rows, int d, int dtype, void* o, float* lse,
                                   cudaStream_t st);
 
 // Decode attention streamed through shared memory on mma.sync (bf16, d = 128,
@@ -142,6 +155,21 @@ cudaError_t launch_attn_decode(const Shape& s, int64_t n_query, const void* q, c
                                const void* v, const void* k_tiles, const void* v_tiles,
                                const int32_t* idx, void* o, float* lse, void* ws, int* err,
                                cudaStream_t st);
+
+// Host-resident bank content (offload.cu): scratch of the staging step, and the step
+// itself (marks the selected blocks, numbers them per group, gathers their K/V tiles
+// from device-accessible host memory into an HBM staging bank and rewrites the selection
+// as staging slots).
+size_t offload_ws_bytes(const Shape& s, int64_t n_query, int tile_bytes);
+cudaError_t launch_offload_stage(const Shape& s, int64_t n_query, const int32_t* idx,
+                                 const void* k_host, const void* v_host, int tile_bytes,
+                                 char* ws, int32_t** idx_staged_out, void** k_stage_out,
+                                 void** v_stage_out, cudaStream_t st);
+
+// Document-wise rotary positions (docs.cu): rotates q [T, hq, d] and k [T, hkv, d] in
+// place, T = batch * seq packed tokens, positions from the device boundaries cu.
+cudaError_t launch_rope_docwise(const Shape& s, const int32_t* cu, int64_t n_docs, void* q,
+                                void* k, double base, cudaStream_t st);
 
 // Host-side checks of a decode call's shapes and pointers (msa_api.cu), shared by the
 // decode entry points; *empty is set for a call with no work, *tc when the tensor-core

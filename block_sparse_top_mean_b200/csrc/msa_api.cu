@@ -11,6 +11,7 @@ using msa::Shape;
 namespace {
 
 constexpr int64_t kMaxElems = (int64_t)1 << 40;   // guards every size product below
+constexpr int kTileBytesKV = 16384;                // one encoded 64-key K or V tile
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
@@ -91,6 +92,10 @@ size_t ws_bytes_for(const Shape& s, int op, int64_t n_query) {
     case MSA_OP_DECODE:
       return msa::kWsHeader + round256(decode_sel_ws(s, n_query)) +
              round256(msa::decode_attn_ws_bytes(s, n_query));
+    case MSA_OP_DECODE_OFFLOAD:
+      return msa::kWsHeader + round256(decode_sel_ws(s, n_query)) +
+             round256(msa::decode_attn_ws_bytes(s, n_query)) +
+             round256(msa::offload_ws_bytes(s, n_query, kTileBytesKV));
     default:
       return 0;
   }
@@ -182,8 +187,9 @@ const char* msa_status_string(msa_status st) {
 
 size_t msa_workspace_bytes(const msa_params* p, int32_t op, int64_t n_query) {
   Shape s;
-  if (check_params(p, op == MSA_OP_DECODE, &s) != MSA_OK) return 0;
-  if (op == MSA_OP_DECODE && n_query < 0) return 0;
+  const bool dec = op == MSA_OP_DECODE || op == MSA_OP_DECODE_OFFLOAD;
+  if (check_params(p, dec, &s) != MSA_OK) return 0;
+  if (dec && n_query < 0) return 0;
   return ws_bytes_for(s, op, n_query);
 }
 
@@ -313,6 +319,59 @@ msa_status msa_decode_fwd(const msa_params* p, int64_t n_query, const void* q, c
   return cuda_status(e);
 }
 
+msa_status msa_rope_docwise(const msa_params* p, const int32_t* cu_seqlens, int64_t n_docs,
+                            void* q, void* k, double base, msa_stream_t stream) {
+  Shape s;
+  msa_status st = check_params(p, false, &s);
+  if (st != MSA_OK) return st;
+  if (n_docs < 1 || !(base > 1.0) || !isfinite(base)) return MSA_ERR_INVALID_ARG;
+  if (empty_prefill(s)) return MSA_OK;
+  if (n_docs >= INT32_MAX || s.batch * s.seq >= INT32_MAX) return MSA_ERR_UNSUPPORTED;
+  if (cu_seqlens == nullptr || q == nullptr || k == nullptr || !aligned16(q) || !aligned16(k))
+    return MSA_ERR_INVALID_ARG;
+  return cuda_status(msa::launch_rope_docwise(s, cu_seqlens, n_docs, q, k, base,
+                                              (cudaStream_t)stream));
+}
+
+msa_status msa_prefill_varlen_fwd(const msa_params* p, const int64_t* cu_seqlens, int64_t n_docs,
+                                  const void* q, const void* k, const void* v, int32_t* idx,
+                                  void* o, float* lse, void* ws, size_t ws_bytes,
+                                  msa_stream_t stream) {
+  Shape s;
+  msa_status st = check_params(p, false, &s);
+  if (st != MSA_OK) return st;
+  if (p->batch != 1 || n_docs < 1 || cu_seqlens == nullptr) return MSA_ERR_INVALID_ARG;
+  if (cu_seqlens[0] != 0 || cu_seqlens[n_docs] != s.seq) return MSA_ERR_INVALID_ARG;
+  int64_t longest = 0;
+  for (int64_t d = 0; d < n_docs; ++d) {
+    const int64_t len = cu_seqlens[d + 1] - cu_seqlens[d];
+    if (len < 0) return MSA_ERR_INVALID_ARG;
+    if (len > longest) longest = len;
+  }
+  if (s.seq == 0) return MSA_OK;
+  if (q == nullptr || k == nullptr || v == nullptr || idx == nullptr || o == nullptr)
+    return MSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return MSA_ERR_INVALID_ARG;
+  msa_params one = *p;
+  one.seq = longest;
+  Shape sl;
+  if ((st = check_params(&one, false, &sl)) != MSA_OK) return st;
+  if ((st = check_ws(sl, MSA_OP_PREFILL, 0, ws, ws_bytes)) != MSA_OK) return st;
+  const size_t es = s.dtype == MSA_BF16 ? 2 : 4;
+  for (int64_t d = 0; d < n_docs; ++d) {
+    const int64_t a = cu_seqlens[d], len = cu_seqlens[d + 1] - a;
+    if (len == 0) continue;
+    one.seq = len;
+    st = msa_prefill_fwd(&one, (const char*)q + a * s.hq * s.d * es,
+                         (const char*)k + a * s.hkv * s.d * es,
+                         (const char*)v + a * s.hkv * s.d * es, idx + a * s.hkv * s.topk,
+                         (char*)o + a * s.hq * s.d * es, lse ? lse + a * s.hq : nullptr, ws,
+                         ws_bytes, stream);
+    if (st != MSA_OK) return st;
+  }
+  return MSA_OK;
+}
+
 size_t msa_bank_tiles_bytes(const msa_params* p, int32_t which) {
   Shape s;
   if (check_params(p, true, &s) != MSA_OK) return 0;
@@ -397,6 +456,106 @@ msa_status msa_decode_fwd_tiled(const msa_params* p, int64_t n_query, const void
   if (st != MSA_OK) return st;
   return msa_decode_attn_tiled(p, n_query, q, k_tiles, v_tiles, idx, o, lse, ws, ws_bytes,
                                stream);
+}
+
+msa_status msa_decode_select_shard(const msa_params* p, int64_t n_query, const void* q,
+                                   const void* kbar_tiles, int64_t block_offset, uint64_t* keys,
+                                   void* ws, size_t ws_bytes, msa_stream_t stream) {
+  Shape s;
+  bool empty = false;
+  const void* bufs[] = {kbar_tiles, keys};
+  msa_status st = tiled_checks(p, n_query, q, bufs, 2, ws, ws_bytes, &s, &empty);
+  if (st != MSA_OK || empty) return st;
+  if (block_offset < 0 || block_offset + s.nb > INT32_MAX / 2) return MSA_ERR_INVALID_ARG;
+  return cuda_status(msa::launch_topk_decode_tc(s, n_query, q, nullptr, nullptr, kbar_tiles,
+                                                nullptr, ws_body(ws), err_word(ws),
+                                                (cudaStream_t)stream, keys, block_offset));
+}
+
+msa_status msa_decode_merge_shards(const msa_params* p, int64_t n_query, const uint64_t* keys,
+                                   int64_t world, int64_t block_begin, int64_t block_count,
+                                   int32_t* idx, int32_t* idx_local, msa_stream_t stream) {
+  Shape s;
+  msa_status st = check_params(p, true, &s);
+  if (st != MSA_OK) return st;
+  if (n_query < 0 || world < 1 || block_begin < 0 || block_count < 0 ||
+      block_begin + block_count > INT32_MAX / 2)
+    return MSA_ERR_INVALID_ARG;
+  if (n_query == 0) return MSA_OK;
+  if (keys == nullptr || idx == nullptr) return MSA_ERR_INVALID_ARG;
+  if (world > 4096 || n_query * s.hkv > ((int64_t)1 << 31)) return MSA_ERR_UNSUPPORTED;
+  return cuda_status(msa::launch_merge_shard_keys(keys, world, n_query * s.hkv, (int)s.topk,
+                                                  block_begin, block_count, idx, idx_local,
+                                                  (cudaStream_t)stream));
+}
+
+msa_status msa_decode_combine_shards(const msa_params* p, int64_t n_query, const void* o_parts,
+                                     const float* lse_parts, int64_t world, void* o, float* lse,
+                                     msa_stream_t stream) {
+  Shape s;
+  msa_status st = check_params(p, true, &s);
+  if (st != MSA_OK) return st;
+  if (n_query < 0 || world < 1) return MSA_ERR_INVALID_ARG;
+  if (n_query == 0) return MSA_OK;
+  if (o_parts == nullptr || lse_parts == nullptr || o == nullptr) return MSA_ERR_INVALID_ARG;
+  if (world > 4096 || n_query * s.hq > ((int64_t)1 << 31)) return MSA_ERR_UNSUPPORTED;
+  return cuda_status(msa::launch_combine_shards(o_parts, lse_parts, world, n_query * s.hq,
+                                                (int)s.d, s.dtype, o, lse,
+                                                (cudaStream_t)stream));
+}
+
+// Device address under which the GPU reads a host (pinned) or device buffer; null for
+// pageable host memory the GPU cannot reach.
+static const void* gpu_address(const void* p) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();                  // clear the error the failed query recorded
+    return nullptr;
+  }
+  if (a.type != cudaMemoryTypeHost && a.type != cudaMemoryTypeDevice) return nullptr;
+  return a.devicePointer;
+}
+
+msa_status msa_decode_fwd_offload(const msa_params* p, int64_t n_query, const void* q,
+                                  const void* kbar_tiles, const void* k_tiles_host,
+                                  const void* v_tiles_host, int32_t* idx, void* o, float* lse,
+                                  void* ws, size_t ws_bytes, msa_stream_t stream) {
+  Shape s;
+  msa_status st = check_params(p, true, &s);
+  if (st != MSA_OK) return st;
+  if (n_query < 0) return MSA_ERR_INVALID_ARG;
+  if (n_query == 0 || s.seq == 0) return MSA_OK;
+  if (n_query > 65535 * 64) return MSA_ERR_UNSUPPORTED;
+  if (!tiled_decode_supported(s) || s.seq % s.block != 0) return MSA_ERR_UNSUPPORTED;
+  if (n_query * s.topk * (s.block / 64) > INT32_MAX / 64) return MSA_ERR_UNSUPPORTED;
+  if (q == nullptr || kbar_tiles == nullptr || k_tiles_host == nullptr ||
+      v_tiles_host == nullptr || idx == nullptr || o == nullptr)
+    return MSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(kbar_tiles) || !aligned16(k_tiles_host) ||
+      !aligned16(v_tiles_host) || !aligned16(o))
+    return MSA_ERR_INVALID_ARG;
+  if ((st = check_ws(s, MSA_OP_DECODE_OFFLOAD, n_query, ws, ws_bytes)) != MSA_OK) return st;
+  const void* kd = gpu_address(k_tiles_host);
+  const void* vd = gpu_address(v_tiles_host);
+  if (kd == nullptr || vd == nullptr) return MSA_ERR_INVALID_ARG;   // pageable host memory
+  cudaStream_t cs = (cudaStream_t)stream;
+  char* sel_ws = ws_body(ws);
+  char* att_ws = sel_ws + round256(decode_sel_ws(s, n_query));
+  char* off_ws = att_ws + round256(msa::decode_attn_ws_bytes(s, n_query));
+  cudaError_t e = msa::launch_topk_decode_tc(s, n_query, q, nullptr, nullptr, kbar_tiles, idx,
+                                             sel_ws, err_word(ws), cs);
+  int32_t* idx_staged = nullptr;
+  void *ks = nullptr, *vs = nullptr;
+  if (e == cudaSuccess)
+    e = msa::launch_offload_stage(s, n_query, idx, kd, vd, kTileBytesKV, off_ws, &idx_staged,
+                                  &ks, &vs, cs);
+  if (e != cudaSuccess) return MSA_ERR_CUDA;
+  // the staging bank: n_query * topk blocks per KV group, addressed by staging slot
+  Shape staged = s;
+  staged.seq = n_query * s.topk * s.block;
+  staged.nb = n_query * s.topk;
+  return cuda_status(msa::launch_attn_decode(staged, n_query, q, nullptr, nullptr, ks, vs,
+                                             idx_staged, o, lse, att_ws, err_word(ws), cs));
 }
 
 msa_status msa_read_device_error(const void* ws, int32_t* bits, msa_stream_t stream) {

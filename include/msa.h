@@ -92,7 +92,8 @@ typedef enum {
   MSA_OP_PREFILL = 2,
   MSA_OP_DECODE = 3,
   MSA_OP_SPARSE_ATTN_MIN = 4, /* smallest workspace msa_sparse_attn_fwd accepts */
-  MSA_OP_PREFILL_MIN = 5      /* smallest workspace msa_prefill_fwd accepts */
+  MSA_OP_PREFILL_MIN = 5,     /* smallest workspace msa_prefill_fwd accepts */
+  MSA_OP_DECODE_OFFLOAD = 6   /* msa_decode_fwd_offload */
 } msa_op;
 
 /* Device error bits (msa_read_device_error). */
@@ -173,6 +174,40 @@ MSA_API msa_status msa_prefill_fwd(const msa_params* p, const void* q, const voi
                            int32_t* idx, void* o, float* lse, void* ws, size_t ws_bytes,
                            msa_stream_t stream);
 
+/* Document-wise rotary positions ([MSA-DE] "Das Gehirn mit zwei Geschwindigkeiten": the
+ * position counter restarts at zero at the start of every document), applied in place:
+ * for the T = p->batch * p->seq packed tokens of q [T, hq, d] and k [T, hkv, d], dimensions
+ * i and i + d/2 of every head are rotated by pos * base^(-2i/d):
+ *   (x_i, x_{i+d/2}) -> (x_i cos a - x_{i+d/2} sin a, x_{i+d/2} cos a + x_i sin a),
+ * pos = t - cu_seqlens[doc(t)].  cu_seqlens: DEVICE int32 array of the n_docs + 1 document
+ * boundaries, 0 = cu_seqlens[0] <= ... <= cu_seqlens[n_docs] = T (other contents give
+ * meaningless positions but no out-of-range access).  base > 1.  Angles are formed in
+ * fp64, the rotation in fp32, the result rounded to the tensors' dtype.  Values are not
+ * rotated.  The rotated q and k then feed every other call unchanged. */
+MSA_API msa_status msa_rope_docwise(const msa_params* p, const int32_t* cu_seqlens,
+                                    int64_t n_docs, void* q, void* k, double base,
+                                    msa_stream_t stream);
+
+/* Causal prefill of packed documents, each its own sequence ([MSA-DE] "Das Gehirn mit
+ * zwei Geschwindigkeiten": documents are processed one by one): p->batch must be 1 and
+ * p->seq = T, the packed token count; cu_seqlens is a HOST int64 array of the n_docs + 1
+ * boundaries (0 first, T last, nondecreasing; else MSA_ERR_INVALID_ARG).  Document d =
+ * tokens [a, b) with a = cu_seqlens[d], b = cu_seqlens[d+1]: its blocks start at a, no
+ * selection or attention crosses a boundary, and the results are those of
+ * msa_prefill_fwd on that document alone, laid out as:
+ *   q, o [T, hq, d]; k, v [T, hkv, d]   (packed, natural layout);
+ *   idx: document d's [hkv, b-a, topk] at element offset a * hkv * topk, block ids
+ *        counted from the document's first block;
+ *   lse (may be NULL): document d's [hq, b-a] at element offset a * hq.
+ * ws: at least msa_workspace_bytes(p', MSA_OP_PREFILL_MIN, 0) where p' is p with seq =
+ * the longest document (MSA_OP_PREFILL recommended).  The documents run one after the
+ * other on `stream` (one msa_prefill_fwd each: about 9 launches per document, so many
+ * short documents are bound by launch cost). */
+MSA_API msa_status msa_prefill_varlen_fwd(const msa_params* p, const int64_t* cu_seqlens,
+                                          int64_t n_docs, const void* q, const void* k,
+                                          const void* v, int32_t* idx, void* o, float* lse,
+                                          void* ws, size_t ws_bytes, msa_stream_t stream);
+
 /* Decode against a memory bank ([MSA-DE] routing keys in GPU memory decide which content
  * is attended; [MiniMax] per query and GQA group top-k):  for each query n and group g,
  * idx[n,g,:] = top-`topk` of all nb bank blocks by (score desc, index asc), ascending;
@@ -230,6 +265,68 @@ MSA_API msa_status msa_decode_fwd_tiled(const msa_params* p, int64_t n_query, co
                                         const void* kbar_tiles, const void* k_tiles,
                                         const void* v_tiles, int32_t* idx, void* o, float* lse,
                                         void* ws, size_t ws_bytes, msa_stream_t stream);
+
+/* Memory Parallel decode ([MSA-DE] "Das Gehirn mit zwei Geschwindigkeiten": each GPU
+ * holds part of the routing keys, the queries are broadcast to all, the relevance scores
+ * are aggregated, and only the selected content is loaded).  The bank's blocks are split
+ * into contiguous ranges, one per rank; every shard but the last holds a whole number of
+ * blocks.  One decode step on every rank:
+ *   1. msa_decode_select_shard over the rank's shard (its own encoded planes, p->seq = the
+ *      shard's tokens): the shard's best topk 64-bit keys per (query, group),
+ *      keys [n_query, hkv, topk], sorted descending; a key holds the score's
+ *      order-preserving bits above the complement of the bank-wide block id
+ *      (block_offset = the shard's first block), 0 = empty.  Workspace as for
+ *      msa_decode_select_tiled.
+ *   2. the caller all-gathers the keys of all ranks into [world, n_query, hkv, topk]
+ *      (rank order) and calls msa_decode_merge_shards: idx [n_query, hkv, topk] gets the
+ *      bank-wide selection (ascending, -1 padded) - exactly the unsharded top-k, since each
+ *      block of the bank-wide top-k is in its own shard's top-k - and idx_local (nullable)
+ *      the ids, local to the shard [block_begin, block_begin + block_count), of the
+ *      selected blocks this rank owns, -1 elsewhere.
+ *   3. msa_decode_attn_tiled over the rank's shard with idx_local: the rank's partial o and
+ *      lse (o = 0 and lse = -inf for a row with no owned block).
+ *   4. the caller all-gathers o [world, n_query, hq, d] (dtype) and lse
+ *      [world, n_query, hq] and calls msa_decode_combine_shards: o, lse = the softmax over
+ *      the whole selection (partials weighted by exp(lse_r - max), in rank order).
+ * The three calls are asynchronous on `stream`, allocate nothing and check their arguments
+ * on the host first (p->topk, p->hkv, p->hq and p->d give the shapes; p->seq is unused by
+ * steps 2 and 4). */
+MSA_API msa_status msa_decode_select_shard(const msa_params* p, int64_t n_query, const void* q,
+                                           const void* kbar_tiles, int64_t block_offset,
+                                           uint64_t* keys, void* ws, size_t ws_bytes,
+                                           msa_stream_t stream);
+MSA_API msa_status msa_decode_merge_shards(const msa_params* p, int64_t n_query,
+                                           const uint64_t* keys, int64_t world,
+                                           int64_t block_begin, int64_t block_count,
+                                           int32_t* idx, int32_t* idx_local,
+                                           msa_stream_t stream);
+MSA_API msa_status msa_decode_combine_shards(const msa_params* p, int64_t n_query,
+                                             const void* o_parts, const float* lse_parts,
+                                             int64_t world, void* o, float* lse,
+                                             msa_stream_t stream);
+
+/* Decode against a bank whose content stays in host memory ([MSA-DE] "Das Gehirn mit
+ * zwei Geschwindigkeiten": the routing keys stay in GPU memory, the content keys and
+ * values are moved to the CPU's system RAM and brought to the GPU only once the router
+ * selects them; "100 Millionen Token auf 2xA800: Zu welchem Preis?" puts that transfer on
+ * PCIe).  Same method, arguments and results as msa_decode_fwd_tiled, except:
+ *   - k_tiles_host / v_tiles_host: the encoded K/V images (msa_encode_bank layout) in
+ *     PINNED host memory (cudaHostAlloc / cudaHostRegister, or a pinned torch tensor), which
+ *     the GPU reads directly (unified addressing); pageable memory is rejected
+ *     (MSA_ERR_INVALID_ARG).  Device memory is accepted as well.  kbar_tiles is in HBM.
+ *   - after the selection, each selected (KV group, block) is fetched once, however many
+ *     queries selected it, into an HBM staging bank in the workspace; the attention then
+ *     runs on the staged copy, so o, lse and idx are bitwise msa_decode_fwd_tiled's.
+ *   - p->seq must be a multiple of p->block (else MSA_ERR_UNSUPPORTED).
+ * ws: msa_workspace_bytes(p, MSA_OP_DECODE_OFFLOAD, n_query): the decode workspace plus the
+ * staging bank (n_query x topk x block keys of K and V per KV group: 512 MiB for 64
+ * queries, 8 groups, top-32 blocks of 64) and per-block marks (5 bytes per bank block and
+ * group). */
+MSA_API msa_status msa_decode_fwd_offload(const msa_params* p, int64_t n_query, const void* q,
+                                          const void* kbar_tiles, const void* k_tiles_host,
+                                          const void* v_tiles_host, int32_t* idx, void* o,
+                                          float* lse, void* ws, size_t ws_bytes,
+                                          msa_stream_t stream);
 
 /* Bytes of the fixed device scratch used by msa_decode_fwd_static (32 MiB). */
 #define MSA_DECODE_STATIC_SCRATCH_BYTES ((size_t)32 << 20)

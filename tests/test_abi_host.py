@@ -236,3 +236,28 @@ def test_interface_sketch_names(lib):
             lib.msa_workspace_bytes(ctypes.byref(p), op, 64)
     assert lib.msa_get_device_status(None, None) == _lib.MSA_ERR_INVALID_ARG
     assert lib.msa_status_string(_lib.MSA_ERR_TIMEOUT).decode() == "a bounded device wait ran out"
+
+
+def test_docwise_entries_reject_bad_arguments_on_the_host(lib):
+    p = _p(seq=1000, block=64, topk=4)
+    rope = lib.msa_rope_docwise
+    for n_docs, base, cu, q, k in [(0, 1e4, FAKE, FAKE, FAKE), (1, 1.0, FAKE, FAKE, FAKE),
+                                   (1, float("inf"), FAKE, FAKE, FAKE), (1, 1e4, None, FAKE, FAKE),
+                                   (1, 1e4, FAKE, None, FAKE), (1, 1e4, FAKE, FAKE,
+                                                                ctypes.c_void_p(4100))]:
+        assert rope(ctypes.byref(p), cu, n_docs, q, k, base, None) == _lib.MSA_ERR_INVALID_ARG
+    var = lib.msa_prefill_varlen_fwd
+    cu = (ctypes.c_int64 * 3)(0, 400, 1000)
+    bad_cus = [(ctypes.c_int64 * 3)(1, 400, 1000), (ctypes.c_int64 * 3)(0, 400, 999),
+               (ctypes.c_int64 * 3)(0, 1001, 1000)]
+    for c in bad_cus:
+        assert var(ctypes.byref(p), c, 2, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, 1 << 40,
+                   None) == _lib.MSA_ERR_INVALID_ARG
+    p2 = _p(batch=2, seq=1000, block=64, topk=4)
+    assert var(ctypes.byref(p2), cu, 2, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, 1 << 40,
+               None) == _lib.MSA_ERR_INVALID_ARG
+    # the workspace is sized for the longest document (600 tokens)
+    p600 = _p(seq=600, block=64, topk=4)
+    need = lib.msa_workspace_bytes(ctypes.byref(p600), _lib.OP_PREFILL_MIN, 0)
+    assert var(ctypes.byref(p), cu, 2, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, need - 1,
+               None) == _lib.MSA_ERR_WORKSPACE
