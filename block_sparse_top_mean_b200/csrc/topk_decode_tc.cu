@@ -34,12 +34,14 @@
 #include <math_constants.h>
 
 #include "common.cuh"
+#include "decode_keys.cuh"
 #include "sm100.cuh"
 
 namespace msa {
 namespace {
 
 using namespace sm100;
+using namespace keys;
 
 constexpr int kD = 128;
 constexpr int kM = 128;                   // bank blocks per chunk (MMA M, TMEM lanes)
@@ -77,39 +79,6 @@ struct DecGeom {
 constexpr size_t smem_bytes() {
   return 1024 + kQBytes + (size_t)kStages * kStageBytes + (size_t)kN * kPend * 8 +
          (size_t)kN * 8 + sizeof(DBars);
-}
-
-// Order-preserving unsigned bits of a (finite) score; 0 is below every score.
-__device__ __forceinline__ uint32_t score_ord(float s) {
-  const uint32_t b = __float_as_uint(s + 0.0f);            // -0 -> +0
-  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-}
-__device__ __forceinline__ float ord_score(uint32_t ord) {
-  if (ord == 0u) return -CUDART_INF_F;
-  return __uint_as_float((ord & 0x80000000u) ? (ord & 0x7fffffffu) : ~ord);
-}
-__device__ __forceinline__ uint64_t make_key(float s, int64_t j) {
-  return ((uint64_t)score_ord(s) << 32) | (uint32_t)(~(uint32_t)j);
-}
-__device__ __forceinline__ float key_score(uint64_t key) {   // -inf for an empty entry
-  return ord_score((uint32_t)(key >> 32));
-}
-__device__ __forceinline__ int key_block(uint64_t key) {
-  return (int)(~(uint32_t)key);
-}
-
-__device__ __forceinline__ uint64_t umax64(uint64_t a, uint64_t b) { return a > b ? a : b; }
-__device__ __forceinline__ uint64_t umin64(uint64_t a, uint64_t b) { return a < b ? a : b; }
-
-// y, x sorted descending over lanes -> the 32 largest of both, sorted descending.
-__device__ __forceinline__ uint64_t warp_merge_desc(uint64_t y, uint64_t x, int lane) {
-  uint64_t z = umax64(y, __shfl_sync(0xffffffffu, x, 31 - lane));
-#pragma unroll
-  for (int j = 16; j > 0; j >>= 1) {
-    const uint64_t p = __shfl_xor_sync(0xffffffffu, z, j);
-    z = ((lane & j) == 0) ? umax64(z, p) : umin64(z, p);
-  }
-  return z;
 }
 
 // Merges up to 32 pending keys of each of the warp's owned queries into their lists
@@ -506,9 +475,12 @@ topk_decode_tc_kernel(const __grid_constant__ CUtensorMap tmHi,
 }
 
 // One warp per (query, group): merges the sorted lists of the CTAs that covered the
-// group, then writes the best `topk` block indices ascending (-1 padded).
+// group, then writes the best `topk` block indices ascending (-1 padded) or, when `keys`
+// is given, the best `topk` keys sorted descending with their block index moved up by
+// `block_offset` (a shard's blocks renumbered to bank-wide ids; empty entries stay 0).
 __global__ void topk_decode_merge_kernel(const uint64_t* __restrict__ cand,
-                                         int32_t* __restrict__ idx, DecGeom g) {
+                                         int32_t* __restrict__ idx, uint64_t* __restrict__ keys,
+                                         int64_t block_offset, DecGeom g) {
   const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / 32;
   const int lane = threadIdx.x % 32;
   if (w >= g.n_query * g.hkv) return;
@@ -527,6 +499,13 @@ __global__ void topk_decode_merge_kernel(const uint64_t* __restrict__ cand,
     const uint64_t xn = c + 1 < nl ? __ldg(src + (c + 1) * step) : 0ull;
     y = warp_merge_desc(y, x, lane);
     x = xn;
+  }
+  if (keys != nullptr) {
+    if (lane < g.topk) {
+      const uint32_t jg = (uint32_t)((int64_t)key_block(y) + block_offset);
+      keys[w * g.topk + lane] = y == 0ull ? 0ull : ((y & 0xffffffff00000000ull) | (uint32_t)~jg);
+    }
+    return;
   }
   // the best topk, ascending by block index (empty entries sort last)
   int j = (lane < g.topk && y != 0ull) ? key_block(y) : 0x7fffffff;
@@ -669,7 +648,7 @@ size_t topk_decode_tc_ws_bytes(const Shape& s, int64_t n_query) {
 cudaError_t launch_topk_decode_tc(const Shape& s, int64_t n_query, const void* q,
                                   const void* kbar_hi, const void* kbar_lo,
                                   const void* kbar_tiles, int32_t* idx, void* ws, int* err,
-                                  cudaStream_t st) {
+                                  cudaStream_t st, uint64_t* keys, int64_t block_offset) {
   CUtensorMap mh{}, ml{};
   if (kbar_tiles == nullptr && (!make_bf16_2d_map(&mh, kbar_hi, s.nb, s.hkv * kD, kM) ||
                                 !make_bf16_2d_map(&ml, kbar_lo, s.nb, s.hkv * kD, kM)))
@@ -709,7 +688,8 @@ cudaError_t launch_topk_decode_tc(const Shape& s, int64_t n_query, const void* q
   }
   if (e != cudaSuccess) return e;
   const int64_t warps = n_query * s.hkv;
-  topk_decode_merge_kernel<<<(unsigned)((warps + 1) / 2), 64, 0, st>>>(cand, idx, g);
+  topk_decode_merge_kernel<<<(unsigned)((warps + 1) / 2), 64, 0, st>>>(cand, idx, keys,
+                                                                        block_offset, g);
   return cudaGetLastError();
 }
 

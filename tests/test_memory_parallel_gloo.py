@@ -40,13 +40,17 @@ def _worker(rank, world, port, out):
     import torch.distributed as dist
 
     import oracle
+    from block_sparse_top_mean_b200.memory_parallel import _all_gather, shard_ranges
     dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
                             world_size=world)
     try:
         Qd, K, V = _bank()
         kbar = oracle.pool_keys(K[None], BLOCK)[0]
         nb = kbar.shape[0]
+        # the package's shard ranges (the ones the GPU decode uses) are the oracle's
+        begin, count = shard_ranges(nb, world)[rank]
         lo, hi = oracle.shard_blocks(nb, world, rank)
+        assert (begin, begin + count) == (lo, hi)
         # what this rank holds: its blocks' pooled keys and the keys/values of their tokens
         kb_mine = kbar[lo:hi]
         p_lo, p_hi = lo * BLOCK, min(S, hi * BLOCK)
@@ -66,10 +70,9 @@ def _worker(rank, world, port, out):
                                                                     TOPK + 1)):
                     sc[n, g, c], ids[n, g, c] = s_, j
         # 2. all-gather and merge into the global selection (the same on every rank)
-        all_sc = [torch.empty_like(sc) for _ in range(world)]
-        all_ids = [torch.empty_like(ids) for _ in range(world)]
-        dist.all_gather(all_sc, sc)
-        dist.all_gather(all_ids, ids)
+        # through the package's gather (the GPU decode's exchange): [world, ...], rank order
+        all_sc = _all_gather(sc)
+        all_ids = _all_gather(ids)
         idx = {}
         for n in range(NQ):
             for g in range(HKV):
@@ -85,10 +88,8 @@ def _worker(rank, world, port, out):
                                          S, BLOCK, g, scale)
             O_r[n, g * G:(g + 1) * G] = torch.from_numpy(o)
             L_r[n, g * G:(g + 1) * G] = torch.from_numpy(lse)
-        all_O = [torch.empty_like(O_r) for _ in range(world)]
-        all_L = [torch.empty_like(L_r) for _ in range(world)]
-        dist.all_gather(all_O, O_r)
-        dist.all_gather(all_L, L_r)
+        all_O = _all_gather(O_r)
+        all_L = _all_gather(L_r)
         O = np.zeros((NQ, HQ, D))
         L = np.zeros((NQ, HQ))
         for n in range(NQ):
