@@ -10,9 +10,11 @@ ABI.  A decode step is the selection and the attention of 64 queries against an 
 
 With no --workload the line's headline is the 1M-token prefill, and the 128K planted
 prefill and the 10M-token decode are timed the same way (K steps after W warm-ups) under
-"workloads".  Multi-GPU (torchrun, one rank per GPU): every rank runs its own independent
-problems (weak scaling, no collective on the data path); the time is the max over ranks
-and `value` counts the work of all ranks.  The CPU baseline and `--impl reference` time
+"workloads".  Multi-GPU (torchrun, one rank per GPU): every rank
+takes a part of the same problems (strong scaling): the prefill sequence split by KV group (no
+collective on the data path), the decode bank split into block shards (Memory Parallel:
+two all-gathers per step); the time is the max over ranks and `value` counts the work of
+all ranks.  The CPU baseline and `--impl reference` time
 the fp64 oracle on the host's cores (worker processes forked before the first CUDA call)
 on a bounded sample of the same workload, rank 0 only.
 """
@@ -450,14 +452,35 @@ class DecodeOracle:
 
 # ------------------------------------------------------------------ our implementation
 
-class PrefillRunner:
-    """Holds device buffers and issues one step through the C ABI."""
+def kv_group_split(w: mi.Workload, rank: int, world: int) -> mi.Workload:
+    """Rank `rank`'s part of one sequence split by KV group: KV heads
+    [rank * hkv / world, (rank + 1) * hkv / world) and their query heads."""
+    if w.hkv % world != 0:
+        raise SystemExit(f"{w.name}: {w.hkv} KV heads do not split over {world} ranks")
+    return w.with_(hq=w.hq // world, hkv=w.hkv // world)
 
-    def __init__(self, w: mi.Workload, seed: int):
+
+class PrefillRunner:
+    """Holds device buffers and issues one step through the C ABI.  With world > 1 the
+    rank holds its KV-group slice of the one sequence (contiguous tensors of its heads, as
+    a head-sharded QKV projection produces them) and runs the same calls on it."""
+
+    def __init__(self, w: mi.Workload, seed: int, rank: int = 0, world: int = 1):
         import block_sparse_top_mean_b200 as msa
         from block_sparse_top_mean_b200 import _lib
-        self.msa, self.lib, self.w = msa, _lib.load(), w
-        self.q, self.k, self.v = mi.prefill_inputs(w, device="cuda", seed=seed)
+        self.msa, self.lib = msa, _lib.load()
+        q, k, v = mi.prefill_inputs(w, device="cuda", seed=seed)
+        if world > 1:
+            wl = kv_group_split(w, rank, world)
+            g0, g1 = rank * wl.hkv, (rank + 1) * wl.hkv
+            G = w.hq // w.hkv
+            q = q[:, :, g0 * G:g1 * G].contiguous()
+            k = k[:, :, g0:g1].contiguous()
+            v = v[:, :, g0:g1].contiguous()
+            w = wl
+            torch.cuda.empty_cache()
+        self.w = w
+        self.q, self.k, self.v = q, k, v
         dev = self.q.device
         self.p = msa.params(batch=w.batch, seq=w.seq, hq=w.hq, hkv=w.hkv, d=w.d, block=w.block,
                             topk=w.topk, scale=w.scale, dtype=self.q.dtype)
@@ -509,16 +532,33 @@ class DecodeRunner:
     bank's pooled keys and encoded images are built once up front (the offline encoding
     of a bank, not timed); the step reads only the encoded images."""
 
-    def __init__(self, w: mi.Workload, seed: int):
+    def __init__(self, w: mi.Workload, seed: int, rank: int = 0, world: int = 1):
         import block_sparse_top_mean_b200 as msa
         from block_sparse_top_mean_b200 import _lib
         self.msa, self.lib, self.w = msa, _lib.load(), w
-        self.q, k, v = mi.decode_inputs(w, device="cuda", seed=seed)
-        _, khi, klo = (t[0] for t in msa.pool_keys(k[None], w.block, split=True))
-        self.kt, self.vt, self.bt = msa.encode_bank(k, v, khi, klo, w.block)
-        del k, v, khi, klo                      # the natural layout is not needed any more
+        self.rank, self.world = rank, world
+        self.q, _, _ = mi.decode_inputs(w, device="cuda", seed=seed, bank=False)
         dev = self.q.device
-        self.p = msa.params(batch=1, seq=w.seq, hq=w.hq, hkv=w.hkv, d=w.d, block=w.block,
+        if world > 1:
+            # Memory Parallel: this rank holds only its contiguous shard of the bank
+            from block_sparse_top_mean_b200.memory_parallel import BankShard, shard_ranges
+            begin, count = shard_ranges(w.nb, world)[rank]
+            t0, t1 = begin * w.block, min(w.seq, (begin + count) * w.block)
+            k, v = mi.decode_bank_rows(w, t0, t1, device="cuda", seed=seed)
+            self.shard = BankShard(k, v, w.block, begin)
+            del k, v
+            self.kt, self.vt, self.bt = (self.shard.k_tiles, self.shard.v_tiles,
+                                         self.shard.kbar_tiles)
+            seq_local = t1 - t0
+        else:
+            self.shard = None
+            _, k, v = mi.decode_inputs(w, device="cuda", seed=seed)
+            _, khi, klo = (t[0] for t in msa.pool_keys(k[None], w.block, split=True))
+            self.kt, self.vt, self.bt = msa.encode_bank(k, v, khi, klo, w.block)
+            del k, v, khi, klo                  # the natural layout is not needed any more
+            seq_local = w.seq
+        torch.cuda.empty_cache()
+        self.p = msa.params(batch=1, seq=seq_local, hq=w.hq, hkv=w.hkv, d=w.d, block=w.block,
                             topk=w.topk, scale=w.scale, dtype=self.q.dtype)
         self.o = torch.empty_like(self.q)
         self.lse = torch.empty(w.n_query, w.hq, dtype=torch.float32, device=dev)
@@ -535,6 +575,8 @@ class DecodeRunner:
         self.launches_per_step = 6
 
     def step(self, events=None):
+        if self.shard is not None:
+            return self.step_sharded(events)
         # msa_decode_fwd_tiled as its two calls, so the phases can be timed apart
         s = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
         P, w = self.ptr, self.w
@@ -548,6 +590,20 @@ class DecodeRunner:
             self.pp, w.n_query, P["q"], P["kt"], P["vt"], P["idx"], P["o"], P["lse"], P["ws"],
             self.ws.numel(), s))
         if events:
+            events[2].record()
+
+
+    def step_sharded(self, events=None):
+        """Memory Parallel decode step: shard scan, all-gather of the keys, merge, owned-block
+        attention, all-gather of the partials, combine (block_sparse_top_mean_b200.
+        memory_parallel.decode_step)."""
+        from block_sparse_top_mean_b200.memory_parallel import decode_step
+        if events:
+            events[0].record()
+        self.o, self.lse, self.idx = decode_step(self.q, self.shard, self.w.topk, self.w.scale,
+                                                 ws=self.ws)
+        if events:
+            events[1].record()
             events[2].record()
 
 
@@ -611,15 +667,17 @@ PREFILL_ATTN_DRAM_PER_ENTRY = {"attn_tiles_kernel": 2006.0, "merge_partials_kern
 
 
 def bench_prefill(w, args, world, rank, local, pool):
-    r = PrefillRunner(w, seed=rank)
+    r = PrefillRunner(w, seed=0, rank=rank, world=world)
+    w_full, w = w, r.w
     attn_flops, score_flops = prefill_flops(w)
     ms, ev, clocks = timed_steps(r, args, world, local, 4)
     phase = {n: statistics.mean(e[a].elapsed_time(e[a + 1]) for e in ev)
              for a, n in enumerate(["pool_keys", "topk_select", "sparse_attn"])}
     err = r.msa.read_device_error(r.ws)
     peaks, peak_src = load_peaks()
+    # every rank holds 1/world of the sequence's KV groups: world x its work = the sequence
     value = world * (attn_flops + score_flops) / (ms * 1e-3) / 1e12
-    tokens_s = world * w.seq * w.batch / (ms * 1e-3)
+    tokens_s = w_full.seq * w_full.batch / (ms * 1e-3)
     attn_tflops = attn_flops / (phase["sparse_attn"] * 1e-3) / 1e12
     peak = peaks["bf16_tflops_sustained"]
     entries = prefill_entries(w)
@@ -654,16 +712,19 @@ def bench_prefill(w, args, world, rank, local, pool):
     line = {
         "metric": "sparse-attn prefill TFLOP/s", "value": round(value, 3), "unit": "TFLOP/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
+        "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "strong",
         "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
         "data": "synthetic",
-        "config": {"workload": w.name, "batch_per_gpu": w.batch, "seq": w.seq, "hq": w.hq,
-                   "hkv": w.hkv, "d": w.d, "block": w.block, "topk": w.topk,
+        "config": {"workload": w_full.name, "batch": w.batch, "seq": w.seq, "hq": w_full.hq,
+                   "hkv": w_full.hkv, "d": w.d, "block": w.block, "topk": w.topk,
+                   "kv_heads_per_gpu": w.hkv,
                    "planted_frac": w.planted_frac,
                    "l2": f"inputs larger than L2 (Q alone {w.batch * w.seq * w.hq * w.d * 2 / 2**30:.2f} GiB), no flush",
                    "workspace_gib": round(r.ws.numel() / 2**30, 2),
                    "attn_token_slabs": r.n_slabs,
-                   "parallelism": f"{world} independent sequences, one per GPU"},
+                   "parallelism": ("one GPU" if world == 1 else
+                                   f"one sequence split by KV group over {world} GPUs "
+                                   f"({w.hkv} KV heads each), no collective on the data path")},
         "tokens_per_s": round(tokens_s, 1),
         "flops_per_step": {"attention": attn_flops, "scoring": score_flops},
         "phases_ms": {k: round(v, 3) for k, v in phase.items()},
@@ -678,7 +739,7 @@ def bench_prefill(w, args, world, rank, local, pool):
 
 
 def bench_decode(w, args, world, rank, local, pool):
-    r = DecodeRunner(w, seed=rank)
+    r = DecodeRunner(w, seed=0, rank=rank, world=world)
     work = decode_work(w)
     # the encoded bank (41 GB) and its pooled-key planes (0.6 GB) are larger than L2
     ms, ev, clocks = timed_steps(r, args, world, local, 3)
@@ -686,6 +747,8 @@ def bench_decode(w, args, world, rank, local, pool):
     sel_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
     att_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
     planes_read = float(w.nb * w.hkv * w.d * 4)
+    if world > 1:
+        return bench_decode_sharded(w, r, args, world, ms, clocks, peaks, peak_src, work)
     phases = {
         "select": {"ms": sel_ms, "bytes": work["score_bytes"],
                    "kernel": "msa_decode_select_tiled (sample scan + threshold + full "
@@ -727,14 +790,44 @@ def bench_decode(w, args, world, rank, local, pool):
     line = {
         "metric": "decode us/step", "value": round(ms * 1e3, 1), "unit": "us/step",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": round(ms, 4), "higher_is_better": False, "scaling": "weak",
+        "ms_per_step": round(ms, 4), "higher_is_better": False, "scaling": "strong",
         "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
         "config": {"workload": w.name, "n_query": w.n_query, "bank_tokens": w.seq, "hq": w.hq,
                    "hkv": w.hkv, "d": w.d, "block": w.block, "topk": w.topk,
                    "l2": "bank and pooled keys larger than L2, no flush",
-                   "parallelism": f"{world} independent banks, one per GPU"},
+                   "parallelism": "one GPU"},
         "phases": phase_line, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": r.launches_per_step * args.steps, "clocks": clocks,
+        "device_error_bits": r.msa.read_device_error(r.ws),
+    }
+    del r
+    torch.cuda.empty_cache()
+    return line
+
+
+def bench_decode_sharded(w, r, args, world, ms, clocks, peaks, peak_src, work):
+    """The Memory Parallel decode line: the bank split over the ranks, one step = shard
+    scan + key all-gather + merge + owned-block attention + partial all-gather + combine."""
+    per_rank = (work["score_bytes"] + work["attn_bytes"]) / world
+    gbs = per_rank / (ms * 1e-3) / 1e9
+    roof = {"bound": "hbm", "kernel": "Memory Parallel decode step (one rank)",
+            "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": round(gbs / peaks["hbm_gbs"], 4), "peak_source": f"hbm_gbs of {peak_src}",
+            "traffic": None, "algorithmic_per_launch": per_rank,
+            "algorithmic_note": "one bf16 plane of the rank's pooled keys and, on average, "
+                                "1/world of the selected K/V blocks"}
+    line = {
+        "metric": "decode us/step", "value": round(ms * 1e3, 1), "unit": "us/step",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms, 4), "higher_is_better": False, "scaling": "strong",
+        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": {"workload": w.name, "n_query": w.n_query, "bank_tokens": w.seq, "hq": w.hq,
+                   "hkv": w.hkv, "d": w.d, "block": w.block, "topk": w.topk,
+                   "l2": "bank and pooled keys larger than L2, no flush",
+                   "parallelism": f"Memory Parallel: the bank in {world} contiguous block "
+                                  f"shards, two NCCL all-gathers per step"},
+        "roofline": roof, "cpu_baseline": None, "e2e": None,
+        "gpu_launches": 9 * args.steps, "clocks": clocks,
         "device_error_bits": r.msa.read_device_error(r.ws),
     }
     del r

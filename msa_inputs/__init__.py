@@ -31,7 +31,7 @@ import torch
 __all__ = [
     "LazyBank", "lazy_decode_bank",
     "Workload", "WORKLOADS", "normal", "planted_blocks", "planted_directions",
-    "prefill_inputs", "decode_inputs", "STREAM_Q", "STREAM_K", "STREAM_V",
+    "prefill_inputs", "decode_inputs", "normal_rows", "decode_bank_rows", "STREAM_Q", "STREAM_K", "STREAM_V",
     "STREAM_U", "STREAM_PLANT", "STREAM_DECODE_Q",
 ]
 
@@ -113,6 +113,32 @@ def normal(shape, seed: int, stream: int, device="cpu", dtype=torch.float32,
             x = shift(x, start)
         out[start:start + cnt] = x.to(torch.float32).to(dtype)
     return out.view(shape)
+
+
+def normal_rows(shape, row_lo: int, row_hi: int, seed: int, stream: int, device="cpu",
+                dtype=torch.float32) -> torch.Tensor:
+    """Rows [row_lo, row_hi) along the first axis of normal(shape, seed, stream, ...),
+    generated alone (the same values: element i depends only on its flat index)."""
+    shape = tuple(int(s) for s in shape)
+    row = 1
+    for s in shape[1:]:
+        row *= s
+    n = (row_hi - row_lo) * row
+    out = torch.empty(n, dtype=dtype, device=device)
+    base = stream_base(seed, stream)
+    for start in range(0, n, _CHUNK):
+        cnt = min(_CHUNK, n - start)
+        out[start:start + cnt] = _normal_chunk(base, row_lo * row + start, cnt,
+                                               device).to(torch.float32).to(dtype)
+    return out.view((row_hi - row_lo,) + shape[1:])
+
+
+def decode_bank_rows(w: "Workload", lo: int, hi: int, device="cpu", seed: int = 0):
+    """Tokens [lo, hi) of the bank K and V of decode_inputs(w, seed=seed)."""
+    dt = w.torch_dtype
+    shape = (w.seq, w.hkv, w.d)
+    return (normal_rows(shape, lo, hi, seed, STREAM_K, device, dt),
+            normal_rows(shape, lo, hi, seed, STREAM_V, device, dt))
 
 
 class LazyBank:

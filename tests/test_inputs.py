@@ -48,3 +48,15 @@ def test_bf16_tensor_is_one_rounding_of_the_fp32_tensor():
     x32 = mi.normal((4096,), seed=3, stream=1, dtype=torch.float32)
     x16 = mi.normal((4096,), seed=3, stream=1, dtype=torch.bfloat16)
     assert torch.equal(x32.to(torch.bfloat16), x16)
+
+
+def test_rows_of_a_tensor_generate_alone():
+    """A shard's rows of a bank, generated on their own, are the full tensor's rows."""
+    full = mi.normal((300, 3, 8), 5, mi.STREAM_K, "cpu", torch.bfloat16)
+    for lo, hi in [(0, 300), (17, 18), (100, 299), (0, 1)]:
+        part = mi.normal_rows((300, 3, 8), lo, hi, 5, mi.STREAM_K, "cpu", torch.bfloat16)
+        assert torch.equal(part, full[lo:hi])
+    w = mi.Workload("b", "decode", 1, 500, 8, 2, 16, 16, 4, "bf16", n_query=2)
+    _, k, v = mi.decode_inputs(w, seed=1)
+    k2, v2 = mi.decode_bank_rows(w, 123, 456, seed=1)
+    assert torch.equal(k2, k[123:456]) and torch.equal(v2, v[123:456])

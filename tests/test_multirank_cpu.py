@@ -59,3 +59,52 @@ def test_reference_arm_under_torchrun_prints_one_line(workload):
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
     assert d["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def _split_worker(rank, world, port, out):
+    """One rank of the KV-group split: the oracle on this rank's head slice of one
+    sequence, gathered over gloo in rank order."""
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import bench
+    import msa_inputs as mi
+    import oracle
+    from block_sparse_top_mean_b200.memory_parallel import _all_gather
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world)
+    try:
+        w = mi.Workload("split", "prefill", 1, 192, 8, 4, 16, 16, 4, "f32")
+        q, k, v = mi.prefill_inputs(w)
+        wl = bench.kv_group_split(w, rank, world)
+        G = w.hq // w.hkv
+        g0, g1 = rank * wl.hkv, (rank + 1) * wl.hkv
+        ql, kl, vl = (x.numpy() for x in (q[:, :, g0 * G:g1 * G], k[:, :, g0:g1], v[:, :, g0:g1]))
+        rows = oracle.prefill_rows(ql, kl, vl, w.block, w.topk, w.scale)
+        O = np.zeros((w.seq, wl.hq, w.d))
+        for r in rows:
+            O[r.t, r.g * G:(r.g + 1) * G] = r.O
+        allO = _all_gather(torch.from_numpy(O))           # [world, S, hq/world, d]
+        full = torch.cat(list(allO), dim=1).numpy()       # heads in rank order
+        ref = oracle.prefill_rows(q.numpy(), k.numpy(), v.numpy(), w.block, w.topk, w.scale)
+        Ofull = np.zeros((w.seq, w.hq, w.d))
+        for r in ref:
+            Ofull[r.t, r.g * G:(r.g + 1) * G] = r.O
+        af, sf = bench.prefill_flops(w)
+        al, sl = bench.prefill_flops(wl)
+        out[rank] = (float(np.abs(full - Ofull).max()), (al + sl) * world == af + sf)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_kv_group_split_reassembles_the_sequence():
+    """bench.py --gpus N splits one sequence by KV group: the ranks' outputs, gathered in
+    rank order, are the whole sequence's, and world x a rank's FLOPs is the sequence's."""
+    port = _free_port()
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.spawn(_split_worker, args=(2, port, out), nprocs=2, join=True)
+    for rank in range(2):
+        err, flops_ok = out[rank]
+        assert err == 0.0 and flops_ok
