@@ -31,7 +31,8 @@ import torch
 __all__ = [
     "LazyBank", "lazy_decode_bank",
     "Workload", "WORKLOADS", "normal", "planted_blocks", "planted_directions",
-    "prefill_inputs", "decode_inputs", "normal_rows", "decode_bank_rows", "STREAM_Q", "STREAM_K", "STREAM_V",
+    "prefill_inputs", "decode_inputs", "normal_rows", "decode_bank_rows", "doc_lengths",
+    "cu_seqlens", "STREAM_Q", "STREAM_K", "STREAM_V",
     "STREAM_U", "STREAM_PLANT", "STREAM_DECODE_Q",
 ]
 
@@ -187,6 +188,9 @@ class Workload:
     n_query: int = 0
     planted_frac: float = 0.0
     planted_shift: float = 0.0
+    n_docs: int = 0            # packed documents (kind "prefill_docs")
+    rope_base: float = 0.0     # document-wise RoPE base (kind "prefill_docs")
+    host_bank: bool = False    # decode bank content in pinned host memory
     note: str = field(default="", compare=False)
 
     @property
@@ -221,8 +225,34 @@ WORKLOADS = {
         Workload("decode_bank10m_b64_k32", "decode", 1, 10_000_000, 32, 8, 128, 64, 32, "bf16",
                  n_query=64,
                  note="64 decode queries against a 10M-token bank, 156250 blocks of 64, top-32"),
+        Workload("decode_bank10m_b64_k32_hostbank", "decode", 1, 10_000_000, 32, 8, 128, 64, 32,
+                 "bf16", n_query=64, host_bank=True,
+                 note="the 10M-token decode with the bank's K/V in pinned host memory"),
+        Workload("prefill_docs_1m_b256_k16_rope", "prefill_docs", 1, 1048576, 32, 8, 128, 256,
+                 16, "bf16", n_docs=64, rope_base=1_000_000.0,
+                 note="1M packed tokens in 64 documents (log-uniform lengths 2K-64K), "
+                      "document-wise RoPE, each document its own causal prefill"),
     ]
 }
+
+
+def doc_lengths(total: int, n_docs: int, seed: int = 0, lo: int = 2048, hi: int = 65536):
+    """n_docs document lengths summing to `total`: log-uniform draws in [lo, hi] from a
+    seeded numpy generator, scaled to the total (the last one takes the rounding)."""
+    rng = np.random.default_rng(seed + 1000)
+    x = np.exp(rng.uniform(math.log(lo), math.log(hi), n_docs))
+    n = np.floor(x / x.sum() * total).astype(np.int64)
+    n = np.maximum(n, 1)
+    n[-1] = total - n[:-1].sum()
+    assert n[-1] >= 1
+    return [int(v) for v in n]
+
+
+def cu_seqlens(lengths) -> list[int]:
+    out = [0]
+    for n in lengths:
+        out.append(out[-1] + int(n))
+    return out
 
 
 def planted_blocks(nb: int, frac: float, seed: int) -> list[int]:
@@ -241,8 +271,9 @@ def planted_directions(hkv: int, d: int, seed: int, device="cpu") -> torch.Tenso
 
 
 def prefill_inputs(w: Workload, device="cpu", seed: int = 0):
-    """Q, K, V for a prefill workload, in the workload's dtype, on `device`."""
-    assert w.kind == "prefill"
+    """Q, K, V for a prefill workload, in the workload's dtype, on `device` (packed
+    documents: the batch-1 tensors of all their tokens)."""
+    assert w.kind in ("prefill", "prefill_docs")
     b, s, hq, hkv, d = w.batch, w.seq, w.hq, w.hkv, w.d
     dt = w.torch_dtype
     qshift = kshift = None
