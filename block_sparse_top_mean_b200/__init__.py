@@ -15,7 +15,8 @@ import torch
 from . import _lib
 from ._lib import (  # noqa: F401
     MsaError, MsaParams, OP_DECODE, OP_PREFILL, OP_SPARSE_ATTN, OP_TOPK_SELECT,
-    OP_SPARSE_ATTN_MIN, OP_PREFILL_MIN, OP_DECODE_OFFLOAD,
+    OP_SPARSE_ATTN_MIN, OP_PREFILL_MIN, OP_DECODE_OFFLOAD, OP_SPARSE_ATTN_BWD,
+    OP_SPARSE_ATTN_BWD_MIN,
     DEVERR_IDX_RANGE, DEVERR_TIMEOUT, MSA_F32, MSA_BF16,
 )
 
@@ -26,6 +27,7 @@ __all__ = [
     "read_device_error",
     "clear_device_error", "version", "exp2_poly_eval", "rope_docwise", "prefill_varlen_fwd",
     "decode_select_shard", "decode_merge_shards", "decode_combine_shards", "decode_fwd_offload",
+    "sparse_attn_bwd",
     "MsaError", "MsaParams",
 ]
 
@@ -424,3 +426,23 @@ def decode_fwd_offload(q, kbar_tiles, k_tiles_host, v_tiles_host, seq: int, hkv:
         ctypes.c_void_p(k_tiles_host.data_ptr()), ctypes.c_void_p(v_tiles_host.data_ptr()),
         _ptr(idx), _ptr(o), _ptr(lse), _ptr(ws), ws.numel(), _stream(q.device)))
     return o, lse, idx
+
+
+def sparse_attn_bwd(q, k, v, o, lse, dout, idx, block: int, scale=None, ws=None, out=None):
+    """Gradients of the causal sparse attention for a fixed selection idx: (dq, dk, dv),
+    fp32, shapes of q, k, v.  o and lse are the forward's outputs, dout the upstream
+    gradient of o."""
+    topk = idx.shape[-1]
+    p = _prefill_params(q, k, block, topk, scale)
+    if out is not None:
+        dq, dk, dv = out
+    else:
+        dq = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+        dk = torch.empty(k.shape, dtype=torch.float32, device=q.device)
+        dv = torch.empty(v.shape, dtype=torch.float32, device=q.device)
+    if ws is None:
+        ws = workspace(p, OP_SPARSE_ATTN_BWD, device=q.device)
+    _lib.check("msa_sparse_attn_bwd", _lib.load().msa_sparse_attn_bwd(
+        ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(idx),
+        _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws), ws.numel(), _stream(q.device)))
+    return dq, dk, dv

@@ -14,7 +14,7 @@ MSA_OK, MSA_ERR_INVALID_ARG, MSA_ERR_UNSUPPORTED, MSA_ERR_WORKSPACE, MSA_ERR_CUD
     MSA_ERR_DEVICE, MSA_ERR_TIMEOUT = range(7)
 MSA_F32, MSA_BF16 = 0, 1
 OP_TOPK_SELECT, OP_SPARSE_ATTN, OP_PREFILL, OP_DECODE, OP_SPARSE_ATTN_MIN, OP_PREFILL_MIN, \
-    OP_DECODE_OFFLOAD = range(7)
+    OP_DECODE_OFFLOAD, OP_SPARSE_ATTN_BWD, OP_SPARSE_ATTN_BWD_MIN = range(9)
 DEVERR_IDX_RANGE, DEVERR_TIMEOUT = 0x1, 0x2
 
 # Every symbol include/msa.h declares, with (restype, argtypes).
@@ -59,6 +59,9 @@ SIGNATURES = {
                                           c_int64, c_void_p, c_void_p, c_void_p]),
     "msa_decode_combine_shards": (c_int32, [c_void_p, c_int64, c_void_p, c_void_p, c_int64,
                                             c_void_p, c_void_p, c_void_p]),
+    "msa_sparse_attn_bwd": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                      c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                      c_void_p, c_void_p, c_size_t, c_void_p]),
     "msa_decode_fwd_offload": (c_int32, [c_void_p, c_int64, c_void_p, c_void_p, c_void_p,
                                          c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                          c_size_t, c_void_p]),

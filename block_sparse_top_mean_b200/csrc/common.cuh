@@ -156,6 +156,15 @@ cudaError_t launch_attn_decode(const Shape& s, int64_t n_query, const void* q, c
                                const int32_t* idx, void* o, float* lse, void* ws, int* err,
                                cudaStream_t st);
 
+// Backward of the key-centric tensor-core attention (attn_bwd_tc.cu): dq, dk, dv fp32.
+bool tc_attn_bwd_supported(const Shape& s);
+size_t tc_attn_bwd_ws_bytes(const Shape& s);       // recommended (one pass or 32 GiB slabs)
+size_t tc_attn_bwd_ws_min_bytes(const Shape& s);   // one 2048-token slab
+cudaError_t launch_attn_bwd_tc(const Shape& s, const void* q, const void* k, const void* v,
+                               const void* o, const float* lse, const void* dout,
+                               const int32_t* idx, float* dq, float* dk, float* dv, void* ws_body,
+                               size_t ws_body_bytes, int* err, cudaStream_t st);
+
 // Host-resident bank content (offload.cu): scratch of the staging step, and the step
 // itself (marks the selected blocks, numbers them per group, gathers their K/V tiles
 // from device-accessible host memory into an HBM staging bank and rewrites the selection

@@ -92,6 +92,12 @@ size_t ws_bytes_for(const Shape& s, int op, int64_t n_query) {
     case MSA_OP_DECODE:
       return msa::kWsHeader + round256(decode_sel_ws(s, n_query)) +
              round256(msa::decode_attn_ws_bytes(s, n_query));
+    case MSA_OP_SPARSE_ATTN_BWD:
+    case MSA_OP_SPARSE_ATTN_BWD_MIN:
+      if (!msa::tc_attn_bwd_supported(s)) return 0;
+      return msa::kWsHeader + round256(op == MSA_OP_SPARSE_ATTN_BWD_MIN
+                                           ? msa::tc_attn_bwd_ws_min_bytes(s)
+                                           : msa::tc_attn_bwd_ws_bytes(s));
     case MSA_OP_DECODE_OFFLOAD:
       return msa::kWsHeader + round256(decode_sel_ws(s, n_query)) +
              round256(msa::decode_attn_ws_bytes(s, n_query)) +
@@ -105,6 +111,7 @@ size_t ws_bytes_for(const Shape& s, int op, int64_t n_query) {
 msa_status check_ws(const Shape& s, int op, int64_t n_query, const void* ws, size_t ws_bytes) {
   if (op == MSA_OP_SPARSE_ATTN) op = MSA_OP_SPARSE_ATTN_MIN;
   if (op == MSA_OP_PREFILL) op = MSA_OP_PREFILL_MIN;
+  if (op == MSA_OP_SPARSE_ATTN_BWD) op = MSA_OP_SPARSE_ATTN_BWD_MIN;
   const size_t need = ws_bytes_for(s, op, n_query);
   if (ws == nullptr || ws_bytes < need || !aligned256(ws)) return MSA_ERR_WORKSPACE;
   return MSA_OK;
@@ -262,6 +269,27 @@ msa_status msa_sparse_attn_fwd(const msa_params* p, const void* q, const void* k
   return cuda_status(launch_attention(s, q, k, v, idx, o, lse, ws_body(ws),
                                       ws_bytes - msa::kWsHeader, err_word(ws),
                                       (cudaStream_t)stream));
+}
+
+msa_status msa_sparse_attn_bwd(const msa_params* p, const void* q, const void* k, const void* v,
+                               const void* o, const float* lse, const void* dout,
+                               const int32_t* idx, float* dq, float* dk, float* dv, void* ws,
+                               size_t ws_bytes, msa_stream_t stream) {
+  Shape s;
+  msa_status st = check_params(p, false, &s);
+  if (st != MSA_OK) return st;
+  if (empty_prefill(s)) return MSA_OK;
+  if (!msa::tc_attn_bwd_supported(s)) return MSA_ERR_UNSUPPORTED;
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || lse == nullptr ||
+      dout == nullptr || idx == nullptr || dq == nullptr || dk == nullptr || dv == nullptr)
+    return MSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return MSA_ERR_INVALID_ARG;
+  if ((st = check_ws(s, MSA_OP_SPARSE_ATTN_BWD, 0, ws, ws_bytes)) != MSA_OK) return st;
+  return cuda_status(msa::launch_attn_bwd_tc(s, q, k, v, o, lse, dout, idx, dq, dk, dv,
+                                             ws_body(ws), ws_bytes - msa::kWsHeader,
+                                             err_word(ws), (cudaStream_t)stream));
 }
 
 msa_status msa_prefill_fwd(const msa_params* p, const void* q, const void* k, const void* v,

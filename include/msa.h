@@ -93,7 +93,9 @@ typedef enum {
   MSA_OP_DECODE = 3,
   MSA_OP_SPARSE_ATTN_MIN = 4, /* smallest workspace msa_sparse_attn_fwd accepts */
   MSA_OP_PREFILL_MIN = 5,     /* smallest workspace msa_prefill_fwd accepts */
-  MSA_OP_DECODE_OFFLOAD = 6   /* msa_decode_fwd_offload */
+  MSA_OP_DECODE_OFFLOAD = 6,  /* msa_decode_fwd_offload */
+  MSA_OP_SPARSE_ATTN_BWD = 7, /* msa_sparse_attn_bwd, recommended */
+  MSA_OP_SPARSE_ATTN_BWD_MIN = 8  /* smallest workspace msa_sparse_attn_bwd accepts */
 } msa_op;
 
 /* Device error bits (msa_read_device_error). */
@@ -165,6 +167,25 @@ MSA_API msa_status msa_topk_select(const msa_params* p, const void* q, const flo
 MSA_API msa_status msa_sparse_attn_fwd(const msa_params* p, const void* q, const void* k, const void* v,
                                const int32_t* idx, void* o, float* lse, void* ws,
                                size_t ws_bytes, msa_stream_t stream);
+
+/* Backward of step 4 ([MSA-DE] "Eleganter Proof-of-Concept oder fertiges System?": the
+ * router and the sparse attention are trained end to end).  The selection idx is held
+ * fixed (top-k passes no gradient, so the pooled keys get none through it); the rest is
+ * the exact gradient of the attention over each row's selected keys:
+ *   P_p = exp(scale q.k_p - lse), D = dO . o (per row and head),
+ *   dv_p += P_p dO,  dk_p += scale P_p (dO.v_p - D) q,  dq = scale sum_p P_p (dO.v_p - D) k_p,
+ * summed over every (row, head) that attends key p.  Inputs as for msa_sparse_attn_fwd plus
+ * its outputs o [b,S,hq,d] and lse [b,hq,S] (required) and the upstream gradient dout
+ * [b,S,hq,d]; outputs dq [b,S,hq,d], dk, dv [b,S,hkv,d], all fp32, overwritten.
+ * Supported: bf16, d = 128, block a multiple of 128, G in {1,2,4,8}, topk * block/128 <= 64
+ * (else MSA_ERR_UNSUPPORTED).  ws: msa_workspace_bytes(p, MSA_OP_SPARSE_ATTN_BWD, 0)
+ * recommended, at least MSA_OP_SPARSE_ATTN_BWD_MIN (token slabs of 2048 multiples).
+ * Bitwise deterministic: every sum runs in a fixed order. */
+MSA_API msa_status msa_sparse_attn_bwd(const msa_params* p, const void* q, const void* k,
+                                       const void* v, const void* o, const float* lse,
+                                       const void* dout, const int32_t* idx, float* dq,
+                                       float* dk, float* dv, void* ws, size_t ws_bytes,
+                                       msa_stream_t stream);
 
 /* Whole causal prefill: msa_pool_keys -> msa_topk_select -> msa_sparse_attn_fwd, with the
  * pooled keys kept in the workspace.  idx is written (caller-owned, [b,hkv,S,topk]);
