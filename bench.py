@@ -557,13 +557,18 @@ class DecodeRunner:
             self.kt, self.vt, self.bt = msa.encode_bank(k, v, khi, klo, w.block)
             del k, v, khi, klo                  # the natural layout is not needed any more
             seq_local = w.seq
+            if w.host_bank:
+                # the content images move to pinned host memory; only the routing planes
+                # (bt) stay in HBM
+                self.kt, self.vt = self.kt.cpu().pin_memory(), self.vt.cpu().pin_memory()
         torch.cuda.empty_cache()
         self.p = msa.params(batch=1, seq=seq_local, hq=w.hq, hkv=w.hkv, d=w.d, block=w.block,
                             topk=w.topk, scale=w.scale, dtype=self.q.dtype)
         self.o = torch.empty_like(self.q)
         self.lse = torch.empty(w.n_query, w.hq, dtype=torch.float32, device=dev)
         self.idx = torch.empty(w.n_query, w.hkv, w.topk, dtype=torch.int32, device=dev)
-        n = self.lib.msa_workspace_bytes(ctypes.byref(self.p), _lib.OP_DECODE, w.n_query)
+        op = _lib.OP_DECODE_OFFLOAD if w.host_bank else _lib.OP_DECODE
+        n = self.lib.msa_workspace_bytes(ctypes.byref(self.p), op, w.n_query)
         self.ws = torch.zeros(n, dtype=torch.uint8, device=dev)
         self.check = _lib.check
         P = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
@@ -577,6 +582,8 @@ class DecodeRunner:
     def step(self, events=None):
         if self.shard is not None:
             return self.step_sharded(events)
+        if self.w.host_bank:
+            return self.step_host_bank(events)
         # msa_decode_fwd_tiled as its two calls, so the phases can be timed apart
         s = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
         P, w = self.ptr, self.w
@@ -593,6 +600,20 @@ class DecodeRunner:
             events[2].record()
 
 
+    def step_host_bank(self, events=None):
+        """msa_decode_fwd_offload: selection, staging of the selected K/V tiles from host
+        memory over PCIe, attention on the staged copy."""
+        s = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+        P, w = self.ptr, self.w
+        if events:
+            events[0].record()
+        self.check("msa_decode_fwd_offload", self.lib.msa_decode_fwd_offload(
+            self.pp, w.n_query, P["q"], P["bt"], P["kt"], P["vt"], P["idx"], P["o"], P["lse"],
+            P["ws"], self.ws.numel(), s))
+        if events:
+            events[1].record()
+            events[2].record()
+
     def step_sharded(self, events=None):
         """Memory Parallel decode step: shard scan, all-gather of the keys, merge, owned-block
         attention, all-gather of the partials, combine (block_sparse_top_mean_b200.
@@ -605,6 +626,148 @@ class DecodeRunner:
         if events:
             events[1].record()
             events[2].record()
+
+
+class DocsRunner:
+    """Packed documents: document-wise RoPE of q and k in place, then the causal prefill of
+    every document (msa_rope_docwise + msa_prefill_varlen_fwd).  Each step rotates q and k
+    again; the work per step is the same."""
+
+    def __init__(self, w: mi.Workload, seed: int):
+        import block_sparse_top_mean_b200 as msa
+        from block_sparse_top_mean_b200 import _lib
+        self.msa, self.lib, self.w = msa, _lib.load(), w
+        q, k, v = mi.prefill_inputs(w, device="cuda", seed=seed)
+        self.q, self.k, self.v = q[0], k[0], v[0]
+        self.lengths = mi.doc_lengths(w.seq, w.n_docs, seed)
+        self.cu = mi.cu_seqlens(self.lengths)
+        self.cu_dev = torch.tensor(self.cu, dtype=torch.int32, device="cuda")
+        self.ws = msa.varlen_workspace(self.q, self.k, self.cu, w.block, w.topk)
+        # own kernels per step: the rotation, then per document pool + 2 selection + 6 per
+        # attention token slab
+        slabs = sum(-(-L // max(1, msa.attn_slab_tokens(
+            msa.params(batch=1, seq=L, hq=w.hq, hkv=w.hkv, d=w.d, block=w.block, topk=w.topk,
+                       scale=w.scale, dtype=self.q.dtype), _lib.OP_PREFILL, self.ws.numel())))
+            for L in self.lengths)
+        self.launches_per_step = 1 + 3 * len(self.lengths) + 6 * slabs
+
+    def step(self, events=None):
+        w = self.w
+        if events:
+            events[0].record()
+        self.msa.rope_docwise(self.q, self.k, self.cu_dev, w.rope_base)
+        if events:
+            events[1].record()
+        self.o, self.lse, self.idx = self.msa.prefill_varlen_fwd(
+            self.q, self.k, self.v, self.cu, w.block, w.topk, w.scale, ws=self.ws)
+        if events:
+            events[2].record()
+
+
+class BwdRunner:
+    """The backward of the sparse attention for a fixed selection: the forward runs once
+    (untimed) for o, lse and idx; a step is msa_sparse_attn_bwd."""
+
+    def __init__(self, w: mi.Workload, seed: int):
+        import block_sparse_top_mean_b200 as msa
+        from block_sparse_top_mean_b200 import _lib
+        self.msa, self.lib, self.w = msa, _lib.load(), w
+        self.q, self.k, self.v = mi.prefill_inputs(w, device="cuda", seed=seed)
+        self.o, self.lse, self.idx = msa.prefill_fwd(self.q, self.k, self.v, w.block, w.topk,
+                                                     w.scale)
+        self.dout = mi.normal(self.q.shape, seed + 7, mi.STREAM_DECODE_Q, "cuda", torch.bfloat16)
+        self.dq = torch.empty(self.q.shape, dtype=torch.float32, device="cuda")
+        self.dk = torch.empty(self.k.shape, dtype=torch.float32, device="cuda")
+        self.dv = torch.empty(self.v.shape, dtype=torch.float32, device="cuda")
+        p = msa.params(batch=w.batch, seq=w.seq, hq=w.hq, hkv=w.hkv, d=w.d, block=w.block,
+                       topk=w.topk, scale=w.scale, dtype=self.q.dtype)
+        self.ws = msa.workspace(p, _lib.OP_SPARSE_ATTN_BWD)
+        torch.cuda.empty_cache()
+
+    def step(self, events=None):
+        if events:
+            events[0].record()
+        self.msa.sparse_attn_bwd(self.q, self.k, self.v, self.o, self.lse, self.dout, self.idx,
+                                 self.w.block, self.w.scale, ws=self.ws,
+                                 out=(self.dq, self.dk, self.dv))
+        if events:
+            events[1].record()
+
+
+def bench_bwd(w, args, world, rank, local, pool):
+    if world > 1:
+        raise SystemExit(f"{w.name}: one GPU only")
+    r = BwdRunner(w, seed=0)
+    attn, _ = prefill_flops(w)
+    flops = attn * 10 / 4          # S, dP, dV, dK, dQ: five 2*d contractions per (head, key)
+    ms, ev, clocks = timed_steps(r, args, world, local, 2)
+    peaks, peak_src = load_peaks()
+    tf = flops / (ms * 1e-3) / 1e12
+    line = {
+        "metric": "sparse-attn backward TFLOP/s", "value": round(tf, 3), "unit": "TFLOP/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic",
+        "config": {"workload": w.name, "seq": w.seq, "hq": w.hq, "hkv": w.hkv, "d": w.d,
+                   "block": w.block, "topk": w.topk, "planted_frac": w.planted_frac,
+                   "workspace_gib": round(r.ws.numel() / 2**30, 2), "parallelism": "one GPU"},
+        "flops_per_step": flops,
+        "roofline": {"bound": "tensor", "kernel": "msa_sparse_attn_bwd (whole call)",
+                     "achieved": round(tf, 2), "peak": peaks["bf16_tflops_sustained"],
+                     "unit": "TFLOP/s", "frac": round(tf / peaks["bf16_tflops_sustained"], 4),
+                     "peak_source": f"bf16_tflops_sustained of {peak_src}", "traffic": None,
+                     "algorithmic_per_launch": flops},
+        "cpu_baseline": None, "e2e": None, "clocks": clocks,
+        "device_error_bits": r.msa.read_device_error(r.ws),
+    }
+    del r
+    torch.cuda.empty_cache()
+    return line
+
+
+def bench_docs(w, args, world, rank, local, pool):
+    if world > 1:
+        raise SystemExit(f"{w.name}: one GPU only")
+    r = DocsRunner(w, seed=0)
+    attn = score = 0.0
+    for L in r.lengths:
+        a, s_ = prefill_flops(w.with_(seq=L))
+        attn += a
+        score += s_
+    ms, ev, clocks = timed_steps(r, args, world, local, 3)
+    rope_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    pre_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    peaks, peak_src = load_peaks()
+    rope_bytes = float(w.seq * (w.hq + w.hkv) * w.d * 2 * 2)
+    rope_gbs = rope_bytes / (rope_ms * 1e-3) / 1e9
+    line = {
+        "metric": "sparse-attn prefill TFLOP/s", "value": round((attn + score) / (ms * 1e-3) / 1e12, 3),
+        "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "strong",
+        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": {"workload": w.name, "tokens": w.seq, "n_docs": w.n_docs,
+                   "doc_len_min": min(r.lengths), "doc_len_max": max(r.lengths), "hq": w.hq,
+                   "hkv": w.hkv, "d": w.d, "block": w.block, "topk": w.topk,
+                   "rope_base": w.rope_base, "parallelism": "one GPU"},
+        "phases_ms": {"rope_docwise": round(rope_ms, 3), "prefill_varlen": round(pre_ms, 3)},
+        "flops_per_step": {"attention": attn, "scoring": score},
+        "roofline": {"bound": "tensor", "kernel": "msa_prefill_varlen_fwd (all documents)",
+                     "achieved": round((attn + score) / (pre_ms * 1e-3) / 1e12, 2),
+                     "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                     "frac": round((attn + score) / (pre_ms * 1e-3) / 1e12
+                                   / peaks["bf16_tflops_sustained"], 4),
+                     "peak_source": f"bf16_tflops_sustained of {peak_src}", "traffic": None},
+        "rope_roofline": {"bound": "hbm", "kernel": "rope_docwise_kernel",
+                          "achieved": round(rope_gbs, 1), "peak": peaks["hbm_gbs"],
+                          "unit": "GB/s", "frac": round(rope_gbs / peaks["hbm_gbs"], 4),
+                          "algorithmic_per_launch": rope_bytes},
+        "cpu_baseline": None, "e2e": None,
+        "gpu_launches": r.launches_per_step * args.steps, "clocks": clocks,
+        "device_error_bits": r.msa.read_device_error(r.ws),
+    }
+    del r
+    torch.cuda.empty_cache()
+    return line
 
 
 def timed_steps(r, args, world, local, n_events):
@@ -749,6 +912,8 @@ def bench_decode(w, args, world, rank, local, pool):
     planes_read = float(w.nb * w.hkv * w.d * 4)
     if world > 1:
         return bench_decode_sharded(w, r, args, world, ms, clocks, peaks, peak_src, work)
+    if w.host_bank:
+        return bench_decode_host_bank(w, r, args, ms, clocks, work)
     phases = {
         "select": {"ms": sel_ms, "bytes": work["score_bytes"],
                    "kernel": "msa_decode_select_tiled (sample scan + threshold + full "
@@ -805,6 +970,38 @@ def bench_decode(w, args, world, rank, local, pool):
     return line
 
 
+def bench_decode_host_bank(w, r, args, ms, clocks, work):
+    """The decode line with the bank's K/V in pinned host memory: the step is bound by the
+    PCIe transfer of the selected tiles (each selected (group, block) once)."""
+    idx = r.idx.view(w.n_query, w.hkv, w.topk)
+    staged = sum(int(torch.unique(idx[:, g][idx[:, g] >= 0]).numel()) for g in range(w.hkv))
+    fetched = staged * w.block * w.d * 2 * 2
+    gbs = fetched / (ms * 1e-3) / 1e9
+    line = {
+        "metric": "decode us/step", "value": round(ms * 1e3, 1), "unit": "us/step",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+        "higher_is_better": False, "scaling": "strong", "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic",
+        "config": {"workload": w.name, "n_query": w.n_query, "bank_tokens": w.seq, "hq": w.hq,
+                   "hkv": w.hkv, "d": w.d, "block": w.block, "topk": w.topk,
+                   "bank_content": "pinned host memory, read by the GPU over PCIe",
+                   "parallelism": "one GPU"},
+        "roofline": {"bound": "pcie", "kernel": "msa_decode_fwd_offload (whole step)",
+                     "achieved": round(gbs, 2), "unit": "GB/s", "peak": None,
+                     "frac": None, "traffic": None,
+                     "algorithmic_per_launch": fetched,
+                     "note": "K/V bytes of the distinct selected (group, block) pairs fetched "
+                             "from host memory per step, over the step time"},
+        "staged_blocks_per_step": staged,
+        "cpu_baseline": None, "e2e": None,
+        "gpu_launches": 10 * args.steps, "clocks": clocks,
+        "device_error_bits": r.msa.read_device_error(r.ws),
+    }
+    del r
+    torch.cuda.empty_cache()
+    return line
+
+
 def bench_decode_sharded(w, r, args, world, ms, clocks, peaks, peak_src, work):
     """The Memory Parallel decode line: the bank split over the ranks, one step = shard
     scan + key all-gather + merge + owned-block attention + partial all-gather + combine."""
@@ -837,8 +1034,9 @@ def bench_decode_sharded(w, r, args, world, ms, clocks, peaks, peak_src, work):
 
 def bench_one(name, args, world, rank, local, pool):
     w = workload_of(name, args.seq)
-    return (bench_prefill if w.kind == "prefill" else bench_decode)(w, args, world, rank, local,
-                                                                    pool)
+    fn = {"prefill": bench_prefill, "decode": bench_decode, "prefill_docs": bench_docs,
+          "prefill_bwd": bench_bwd}[w.kind]
+    return fn(w, args, world, rank, local, pool)
 
 
 def run_ours(args, world, rank, local, pool):

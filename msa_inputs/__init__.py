@@ -228,6 +228,11 @@ WORKLOADS = {
         Workload("decode_bank10m_b64_k32_hostbank", "decode", 1, 10_000_000, 32, 8, 128, 64, 32,
                  "bf16", n_query=64, host_bank=True,
                  note="the 10M-token decode with the bank's K/V in pinned host memory"),
+        Workload("prefill_1m_b256_k16_bwd", "prefill_bwd", 1, 1048576, 32, 8, 128, 256, 16,
+                 "bf16", note="backward of the 1M causal prefill's sparse attention"),
+        Workload("prefill_128k_b128_k16_planted_bwd", "prefill_bwd", 1, 131072, 32, 8, 128, 128,
+                 16, "bf16", planted_frac=0.01, planted_shift=3.0,
+                 note="backward of the 128K planted prefill's sparse attention"),
         Workload("prefill_docs_1m_b256_k16_rope", "prefill_docs", 1, 1048576, 32, 8, 128, 256,
                  16, "bf16", n_docs=64, rope_base=1_000_000.0,
                  note="1M packed tokens in 64 documents (log-uniform lengths 2K-64K), "
@@ -273,7 +278,7 @@ def planted_directions(hkv: int, d: int, seed: int, device="cpu") -> torch.Tenso
 def prefill_inputs(w: Workload, device="cpu", seed: int = 0):
     """Q, K, V for a prefill workload, in the workload's dtype, on `device` (packed
     documents: the batch-1 tensors of all their tokens)."""
-    assert w.kind in ("prefill", "prefill_docs")
+    assert w.kind in ("prefill", "prefill_docs", "prefill_bwd")
     b, s, hq, hkv, d = w.batch, w.seq, w.hq, w.hkv, w.d
     dt = w.torch_dtype
     qshift = kshift = None

@@ -20,9 +20,12 @@ def msa():
 
 
 def _tol(ref):
-    """Gradient tolerance: 2e-2 absolute on tensors of unit scale, relative to the
-    tensor's largest magnitude beyond that (bf16 P and dS, bf16 dQ partials)."""
-    return 2e-2 * max(1.0, float(np.abs(ref).max()))
+    """Gradient tolerance: the forward's 2e-2 absolute bar for bf16 inputs, plus one bf16
+    rounding (2^-9 relative) of the tensor's largest magnitude.  The gradients are sums
+    over up to thousands of (row, key) terms whose P and dS factors are rounded to bf16
+    before the tensor-core products, so their error grows with their magnitude; on these
+    cases the observed errors are <= 1.8e-2 for magnitudes up to 12."""
+    return 2e-2 + 2.0 ** -9 * float(np.abs(ref).max())
 
 
 CASES = [
@@ -54,6 +57,7 @@ def test_backward_vs_oracle(msa, w):
     ref = oracle.prefill_backward(Q, K, V, dO, w.block, w.topk, w.scale, idx_override=fixed)
     for name, got, want in zip(("dq", "dk", "dv"), grads, ref):
         err = float(np.abs(got.double().cpu().numpy() - want).max())
+        print(f"{w.name} {name}: max |err| {err:.3e}, max |ref| {float(np.abs(want).max()):.3e}")
         assert err <= _tol(want), (name, err, float(np.abs(want).max()))
 
 
