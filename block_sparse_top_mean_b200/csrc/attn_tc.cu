@@ -651,7 +651,9 @@ attn_tiles_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
 
 // ------------------------------------------------------------------ merge partials
 // One row = (sequence, group, token); G*8 threads per row, 16 output elements (32 bytes)
-// each.  One pass over the row's partials with a running max, four loads in flight.
+// each.  One pass over the row's partials with a running max, kMergeBatch loads in flight
+// per thread.
+constexpr int kMergeBatch = 4;   // 8 measured 2% slower at 1M
 __device__ __forceinline__ void ld_global_nc_v8(const void* p, uint32_t* r) {
   asm volatile("ld.global.nc.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
@@ -683,19 +685,19 @@ merge_partials_kernel(const int32_t* __restrict__ idx, const __nv_bfloat16* __re
   float acc[16];
 #pragma unroll
   for (int e = 0; e < 16; ++e) acc[e] = 0.f;
-  int ps_list[4];
+  int ps_list[kMergeBatch];
   int np = 0;
   auto flush = [&]() {
-    float lv[4];
-    uint32_t raw[4][8];
+    float lv[kMergeBatch];
+    uint32_t raw[kMergeBatch][8];
 #pragma unroll
-    for (int u = 0; u < 4; ++u)
+    for (int u = 0; u < kMergeBatch; ++u)
       if (u < np) {
         lv[u] = lrow[ps_list[u] * G + h];
         ld_global_nc_v8(prow + (int64_t)ps_list[u] * G * kD, raw[u]);
       }
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < kMergeBatch; ++u) {
       if (u >= np || !(lv[u] > -CUDART_INF_F)) continue;
       const float mn = fmaxf(mx, lv[u]);
       const float sc = exp2f((mx - mn) * kLog2e);
@@ -716,7 +718,7 @@ merge_partials_kernel(const int32_t* __restrict__ idx, const __nv_bfloat16* __re
     for (int sub = 0; sub < g.nsub; ++sub) {
       if (!sub_has_keys32(j, own, t, sub, g)) continue;
       ps_list[np++] = sl * g.nsub + sub;
-      if (np == 4) flush();
+      if (np == kMergeBatch) flush();
     }
   }
   if (np > 0) flush();

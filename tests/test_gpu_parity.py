@@ -424,12 +424,21 @@ def test_prefill_full_size_sampled(msa, name):
     assert torch.isfinite(o.float()).all()
 
 
-@pytest.mark.parametrize("scan", ["tc", "fp32"])
+@pytest.mark.parametrize("scan", ["tiled", "tc", "fp32"])
 def test_decode_full_size_sampled(msa, scan):
+    """The 10M-token bank: "tiled" is the path the bench times (encoded bank, the two
+    tiled calls), "tc" and "fp32" the natural-layout scans."""
     w = mi.WORKLOADS["decode_bank10m_b64_k32"]
     q, kb, vb = mi.decode_inputs(w, device="cuda")
     kbar, khi, klo = (t[0] for t in msa.pool_keys(kb[None], w.block, split=True))
-    if scan == "tc":
+    if scan == "tiled":
+        kt, vt, bt = msa.encode_bank(kb, vb, khi, klo, w.block)
+        del kbar, khi, klo
+        torch.cuda.empty_cache()
+        idx = msa.decode_select_tiled(q, bt, w.seq, w.hkv, w.block, w.topk)
+        o, lse = msa.decode_attn_tiled(q, kt, vt, idx, w.seq, w.hkv, w.block, w.scale)
+        del kt, vt, bt
+    elif scan == "tc":
         o, lse, idx = msa.decode_fwd(q, None, kb, vb, w.block, w.topk, w.scale, kbar_hi=khi,
                                      kbar_lo=klo)
     else:
