@@ -28,6 +28,7 @@
 #include <math_constants.h>
 
 #include "common.cuh"
+#include "fastmath.cuh"
 #include "sm100.cuh"
 
 namespace msa {
@@ -218,7 +219,7 @@ constexpr int kIssuer = 4;
 constexpr int kGather = 5;
 
 struct __align__(8) BBars {
-  uint64_t kv_full, q_full, q_empty, sdp, pds, dq, s_free, acc_empty;
+  uint64_t kv_full, q_full[2], q_empty[2], sdp, pds, dq, s_free, acc_empty, meta_full, meta_free;
   uint32_t tmem_base;
   int abort;
 };
@@ -257,28 +258,34 @@ attn_bwd_tiles_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* base = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  unsigned char* Ks = base;
-  unsigned char* Vs = Ks + kTile;
-  unsigned char* Qs = Vs + kTile;
-  unsigned char* DOs = Qs + kTile;
-  unsigned char* Ps = DOs + kTile;
-  unsigned char* DSs = Ps + kTile;
-  BBars* bars = reinterpret_cast<BBars*>(DSs + kTile);
+  unsigned char* Ks = base;                      // the segment's 128 keys   [key][d]
+  unsigned char* Vs = Ks + kTile;                // and values               [key][d]
+  unsigned char* Qs = Vs + kTile;                // 2 stages of query rows   [row][d]
+  unsigned char* DOs = Qs + 2 * kTile;           // 2 stages of dO rows      [row][d]
+  unsigned char* DSs = DOs + 2 * kTile;          // dS of the tile           [key][row]
+  float* m_lse = reinterpret_cast<float*>(DSs + kTile);   // per row: lse * log2(e)
+  float* m_dd = m_lse + kRowsT;                            // per row: D = dO . O
+  uint8_t* m_lim = reinterpret_cast<uint8_t*>(m_dd + kRowsT);   // per row: keys it reads
+  BBars* bars = reinterpret_cast<BBars*>(m_lim + kRowsT);
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
 
   // rows of a tile past its entries are never loaded: start from zeros, so the products
   // with their zero P and dS stay zero
-  for (int i = tid; i < (int)(2 * kTile / 16); i += kBwdThreads)
+  for (int i = tid; i < (int)(4 * kTile / 16); i += kBwdThreads)
     reinterpret_cast<uint4*>(Qs)[i] = make_uint4(0, 0, 0, 0);
   if (tid == 0) {
     mbar_init(&bars->kv_full, 1);
-    mbar_init(&bars->q_full, 1);
-    mbar_init(&bars->q_empty, 1);
+    for (int st = 0; st < 2; ++st) {
+      mbar_init(&bars->q_full[st], 1);
+      mbar_init(&bars->q_empty[st], 1);
+    }
     mbar_init(&bars->sdp, 1);
     mbar_init(&bars->pds, 128);
     mbar_init(&bars->dq, 1);
     mbar_init(&bars->s_free, 128);
     mbar_init(&bars->acc_empty, 128);
+    mbar_init(&bars->meta_full, 128);
+    mbar_init(&bars->meta_free, 128);
     bars->abort = 0;
     fence_mbar_init();
   }
@@ -301,13 +308,23 @@ attn_bwd_tiles_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
     if (lane == 0) { prefetch_tmap(&tmK); prefetch_tmap(&tmV); prefetch_tmap(&tmQ); prefetch_tmap(&tmDO); }
     int n = 0;
     bool stop = false;
+    int ent_next[kPerLane];
     for (int64_t s = blockIdx.x; s < g.nseg && !stop; s += gridDim.x) {
       const int ta = tile_off[s], tb = tile_off[s + 1];
       if (ta == tb) continue;
       const SegId id = seg_id(s, g);
       for (int tile = ta; tile < tb; ++tile, ++n) {
         if (__any_sync(0xffffffffu, *abort_flag != 0)) { stop = true; break; }
-        if (n > 0 && !mbar_wait_warp(&bars->q_empty, (uint32_t)(n - 1) & 1)) {
+        const int st = n & 1;
+        // this stage's previous tile (n - 2) and, at a segment's start, the tile before
+        // (the last reader of K and V) must have finished their MMAs
+        if (n >= 2 && !mbar_wait_warp(&bars->q_empty[st], (uint32_t)((n - 2) >> 1) & 1)) {
+          if (lane == 0) fail();
+          stop = true;
+          break;
+        }
+        if (tile == ta && n >= 1 &&
+            !mbar_wait_warp(&bars->q_empty[st ^ 1], (uint32_t)((n - 1) >> 1) & 1)) {
           if (lane == 0) fail();
           stop = true;
           break;
@@ -321,43 +338,69 @@ attn_bwd_tiles_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
             tma_load_2d(Vs + hf * kHalf, &tmV, &bars->kv_full, x, y0);
           }
         }
-        const int4 tl = tiles[tile];
+        if (tile == ta) {                              // a segment's first tile: load it
+          const int4 t0 = tiles[tile];
+#pragma unroll
+          for (int u = 0; u < kPerLane; ++u) {
+            const int i = lane + u * 32;
+            ent_next[u] = (i < kTok && i < t0.z) ? entries[t0.y + i] : -1;
+          }
+        }
         int ent[kPerLane];
         int n_valid = 0;
 #pragma unroll
         for (int u = 0; u < kPerLane; ++u) {
-          const int i = lane + u * 32;
-          ent[u] = (i < kTok && i < tl.z) ? entries[tl.y + i] : -1;
+          ent[u] = ent_next[u];
           n_valid += __popc(__ballot_sync(0xffffffffu, ent[u] >= 0));
         }
-        if (lane == 0) mbar_arrive_expect_tx(&bars->q_full, (uint32_t)(n_valid * G * kD * 2 * 2));
+        if (lane == 0)
+          mbar_arrive_expect_tx(&bars->q_full[st], (uint32_t)(n_valid * G * kD * 2 * 2));
         __syncwarp();
+        unsigned char* qd = Qs + st * kTile;
+        unsigned char* od = DOs + st * kTile;
 #pragma unroll
         for (int u = 0; u < kPerLane; ++u) {
           if (ent[u] < 0) continue;
           const int i = lane + u * 32;
           const int y = (int)(((int64_t)id.b * g.S + (ent[u] >> 6)) * g.hq + id.gg * G);
-          tma_load_2d(Qs + i * G * 128, &tmQ, &bars->q_full, 0, y);
-          tma_load_2d(Qs + kHalf + i * G * 128, &tmQ, &bars->q_full, 64, y);
-          tma_load_2d(DOs + i * G * 128, &tmDO, &bars->q_full, 0, y);
-          tma_load_2d(DOs + kHalf + i * G * 128, &tmDO, &bars->q_full, 64, y);
+          tma_load_2d(qd + i * G * 128, &tmQ, &bars->q_full[st], 0, y);
+          tma_load_2d(qd + kHalf + i * G * 128, &tmQ, &bars->q_full[st], 64, y);
+          tma_load_2d(od + i * G * 128, &tmDO, &bars->q_full[st], 0, y);
+          tma_load_2d(od + kHalf + i * G * 128, &tmDO, &bars->q_full[st], 64, y);
+        }
+        // the next tile of the segment: its rows into L2 now, its entries kept for the
+        // next iteration's copies
+        if (tile + 1 < tb) {
+          const int4 tn = tiles[tile + 1];
+#pragma unroll
+          for (int u = 0; u < kPerLane; ++u) {
+            const int i = lane + u * 32;
+            const int e = (i < kTok && i < tn.z) ? entries[tn.y + i] : -1;
+            ent_next[u] = e;
+            if (e < 0) continue;
+            const int y = (int)(((int64_t)id.b * g.S + (e >> 6)) * g.hq + id.gg * G);
+            tma_prefetch_2d(&tmQ, 0, y);
+            tma_prefetch_2d(&tmQ, 64, y);
+            tma_prefetch_2d(&tmDO, 0, y);
+            tma_prefetch_2d(&tmDO, 64, y);
+          }
         }
       }
     }
     // nothing may still be landing when the CTA exits
-    if (n > 0) mbar_wait_warp(&bars->q_empty, (uint32_t)(n - 1) & 1);
+    for (int m = n >= 2 ? n - 2 : 0; m < n; ++m)
+      if (!mbar_wait_warp(&bars->q_empty[m & 1], (uint32_t)(m >> 1) & 1)) break;
   } else if (warp == kIssuer) {
     // ---------------------------------------------------------------- MMA issue
     if (lane == 0) {
-      const uint32_t idKK = idesc_bf16(128, 128, 0, 0);   // S, dP
-      const uint32_t idMM = idesc_bf16(128, 128, 1, 1);   // dV, dK (A = P^T / dS^T)
-      const uint32_t idKM = idesc_bf16(128, 128, 0, 1);   // dQ
-      const uint64_t kq = sdesc_sw128(smem_u32(Qs), 16, 1024), kdo = sdesc_sw128(smem_u32(DOs), 16, 1024);
+      const uint32_t idKK = idesc_bf16(128, 128, 0, 0);   // S^T, dP^T: both operands K-major
+      const uint32_t idTM = idesc_bf16(128, 128, 0, 1);   // dV, dK: A = P^T / dS^T in TMEM
+      const uint32_t idMM = idesc_bf16(128, 128, 1, 1);   // dQ: A = dS MN-major
       const uint64_t kk = sdesc_sw128(smem_u32(Ks), 16, 1024), kv = sdesc_sw128(smem_u32(Vs), 16, 1024);
-      const uint64_t kds = sdesc_sw128(smem_u32(DSs), 16, 1024);
-      const uint64_t mp = sdesc_sw128(smem_u32(Ps), kHalf, 1024), mds = sdesc_sw128(smem_u32(DSs), kHalf, 1024);
-      const uint64_t mdo = sdesc_sw128(smem_u32(DOs), kHalf, 1024), mq = sdesc_sw128(smem_u32(Qs), kHalf, 1024);
-      const uint64_t mk = sdesc_sw128(smem_u32(Ks), kHalf, 1024);
+      const uint64_t kq0 = sdesc_sw128(smem_u32(Qs), 16, 1024), kdo0 = sdesc_sw128(smem_u32(DOs), 16, 1024);
+      const uint64_t mq0 = sdesc_sw128(smem_u32(Qs), kHalf, 1024), mdo0 = sdesc_sw128(smem_u32(DOs), kHalf, 1024);
+      const uint64_t mk = sdesc_sw128(smem_u32(Ks), kHalf, 1024), mds = sdesc_sw128(smem_u32(DSs), kHalf, 1024);
+      constexpr uint64_t kStage = kTile >> 4;            // descriptor units between stages
       auto koff = [](int ks) -> uint64_t {             // K-major: 16 elements of the d axis
         return (uint64_t)((ks >> 2) * (kHalf >> 4) + (ks & 3) * 2);
       };
@@ -370,13 +413,16 @@ attn_bwd_tiles_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
         if (!mbar_wait(&bars->kv_full, (uint32_t)sc & 1)) { ok = false; break; }
         for (int tile = ta; tile < tb; ++tile, ++n) {
           if (*abort_flag) { ok = false; break; }
-          if (!mbar_wait(&bars->q_full, (uint32_t)n & 1)) { ok = false; break; }
+          const int st = n & 1;
+          if (!mbar_wait(&bars->q_full[st], (uint32_t)(n >> 1) & 1)) { ok = false; break; }
           if (n > 0 && !mbar_wait(&bars->s_free, (uint32_t)(n - 1) & 1)) { ok = false; break; }
           tc_fence_after();
+          const uint64_t kq = kq0 + st * kStage, kdo = kdo0 + st * kStage;
+          const uint64_t mq = mq0 + st * kStage, mdo = mdo0 + st * kStage;
 #pragma unroll
-          for (int ks = 0; ks < kD / 16; ++ks) umma_ss(tmem + 0, kq + koff(ks), kk + koff(ks), idKK, ks > 0);
+          for (int ks = 0; ks < kD / 16; ++ks) umma_ss(tmem + 0, kk + koff(ks), kq + koff(ks), idKK, ks > 0);
 #pragma unroll
-          for (int ks = 0; ks < kD / 16; ++ks) umma_ss(tmem + 128, kdo + koff(ks), kv + koff(ks), idKK, ks > 0);
+          for (int ks = 0; ks < kD / 16; ++ks) umma_ss(tmem + 128, kv + koff(ks), kdo + koff(ks), idKK, ks > 0);
           umma_commit(&bars->sdp);
           if (!mbar_wait(&bars->pds, (uint32_t)n & 1)) { ok = false; break; }
           if (tile == ta && sc > 0 && !mbar_wait(&bars->acc_empty, (uint32_t)(sc - 1) & 1)) {
@@ -387,14 +433,16 @@ attn_bwd_tiles_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
           const uint32_t first = tile == ta ? 1u : 0u;
 #pragma unroll
           for (int ks = 0; ks < kRowsT / 16; ++ks)
-            umma_ss(tmem + 256, mp + moff(ks), mdo + moff(ks), idMM, (first && ks == 0) ? 0u : 1u);
+            umma_ts(tmem + 256, tmem + 0 + ks * 8, mdo + moff(ks), idTM, (first && ks == 0) ? 0u : 1u);
 #pragma unroll
           for (int ks = 0; ks < kRowsT / 16; ++ks)
-            umma_ss(tmem + 384, mds + moff(ks), mq + moff(ks), idMM, (first && ks == 0) ? 0u : 1u);
+            umma_ts(tmem + 384, tmem + 128 + ks * 8, mq + moff(ks), idTM, (first && ks == 0) ? 0u : 1u);
+          // dQ over S^T's columns: the MMAs of this thread run in issue order, so the dV
+          // products above have read P^T from them before these write
 #pragma unroll
-          for (int ks = 0; ks < kSeg / 16; ++ks) umma_ss(tmem + 0, kds + koff(ks), mk + moff(ks), idKM, ks > 0);
+          for (int ks = 0; ks < kSeg / 16; ++ks) umma_ss(tmem + 0, mds + moff(ks), mk + moff(ks), idMM, ks > 0);
           umma_commit(&bars->dq);
-          umma_commit(&bars->q_empty);
+          umma_commit(&bars->q_empty[st]);
         }
         ++sc;
       }
@@ -402,11 +450,13 @@ attn_bwd_tiles_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
     }
   } else {
     // ---------------------------------------------------------------- rows (warps 0-3)
-    const int r = tid;                                   // tile row = TMEM lane
+    // Thread r is tile row r for the per-row data and the dQ epilogue, and key r (TMEM
+    // lane r of S^T, dP^T, dV, dK) for the softmax and the dV / dK epilogue.
+    const int r = tid;
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
     const int i_tok = r / G, h = r % G;
     const float c2 = g.scale_log2;
-    const uint32_t sP = smem_u32(Ps), sDS = smem_u32(DSs);
+    const uint32_t sDS = smem_u32(DSs);
     int n = 0;
     bool ok = true;
     for (int64_t s = blockIdx.x; s < g.nseg && ok; s += gridDim.x) {
@@ -415,10 +465,12 @@ attn_bwd_tiles_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
       const SegId id = seg_id(s, g);
       const int64_t kbase = (int64_t)id.j * g.block + (int64_t)id.sub * kSeg;
       const int64_t seg_end = min(min((int64_t)id.j * g.block + g.block, kbase + kSeg), g.S);
+      int4 tl_next = tiles[ta];
+      int ent_next = i_tok < tl_next.z ? entries[tl_next.y + i_tok] : -1;
       for (int tile = ta; tile < tb; ++tile, ++n) {
         if (__any_sync(0xffffffffu, *abort_flag != 0)) { ok = false; break; }
-        const int4 tl = tiles[tile];
-        const int ent = i_tok < tl.z ? entries[tl.y + i_tok] : -1;
+        const int ent = ent_next;
+        if (tile + 1 < tb) tl_next = tiles[tile + 1];
         const bool valid = ent >= 0;
         const int64_t t = valid ? (ent >> 6) : 0;
         const int pslot = valid ? (ent & 63) : 0;
@@ -426,42 +478,59 @@ attn_bwd_tiles_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
         if (valid && t / g.block == id.j) end = min(end, t + 1);     // causal, own block
         const int lim = valid ? (int)max((int64_t)0, end - kbase) : 0;
         const int64_t hrow = ((int64_t)id.b * g.hq + id.gg * G + h) * g.S + t;
-        const float lse2 = valid ? lse[hrow] * kLog2e : 0.f;
-        const float dd = valid ? Dd[hrow] : 0.f;
+        // row r's data for every key thread, once the previous tile's readers are done
+        // with it (bounded mbarrier waits: a warp that gives up cannot strand the others)
+        const float lse_r = valid ? lse[hrow] * kLog2e : 0.f;
+        const float dd_r = valid ? Dd[hrow] : 0.f;
+        if (n > 0 && !mbar_wait_warp(&bars->meta_free, (uint32_t)(n - 1) & 1)) { ok = false; break; }
+        m_lse[r] = lse_r;
+        m_dd[r] = dd_r;
+        m_lim[r] = (uint8_t)lim;
+        mbar_arrive(&bars->meta_full);
+        if (!mbar_wait_warp(&bars->meta_full, (uint32_t)n & 1)) { ok = false; break; }
         if (!mbar_wait_warp(&bars->sdp, (uint32_t)n & 1)) { ok = false; break; }
         tc_fence_after();
+        if (tile + 1 < tb) ent_next = i_tok < tl_next.z ? entries[tl_next.y + i_tok] : -1;
+        // key r: P^T and dS^T over the 128 rows, back into TMEM as bf16 (A operands of dV
+        // and dK) and dS into shared memory ([key][row], A operand of dQ)
 #pragma unroll 1
-        for (int kc = 0; kc < 4; ++kc) {
+        for (int c = 0; c < 4; ++c) {
           uint32_t sv[32], pv[32];
-          tmem_ld32(lane_base + kc * 32, sv);
-          tmem_ld32(lane_base + 128 + kc * 32, pv);
+          tmem_ld32(lane_base + c * 32, sv);
+          tmem_ld32(lane_base + 128 + c * 32, pv);
           tmem_ld_wait();
           uint32_t pp[16], pd[16];
 #pragma unroll
           for (int k = 0; k < 32; k += 2) {
-            const int key = kc * 32 + k;
-            const float p0 = key < lim ? exp2f(__uint_as_float(sv[k]) * c2 - lse2) : 0.f;
-            const float p1 = key + 1 < lim ? exp2f(__uint_as_float(sv[k + 1]) * c2 - lse2) : 0.f;
-            const float d0 = p0 * (__uint_as_float(pv[k]) - dd) * g.scale;
-            const float d1 = p1 * (__uint_as_float(pv[k + 1]) - dd) * g.scale;
+            const int rr = c * 32 + k;
+            const float p0 = r < m_lim[rr]
+                                 ? fastmath::fast_exp2(__uint_as_float(sv[k]) * c2 - m_lse[rr]) : 0.f;
+            const float p1 = r < m_lim[rr + 1]
+                                 ? fastmath::fast_exp2(__uint_as_float(sv[k + 1]) * c2 - m_lse[rr + 1])
+                                 : 0.f;
+            const float d0 = p0 * (__uint_as_float(pv[k]) - m_dd[rr]) * g.scale;
+            const float d1 = p1 * (__uint_as_float(pv[k + 1]) - m_dd[rr + 1]) * g.scale;
             pp[k / 2] = pack_bf16x2(p0, p1);
             pd[k / 2] = pack_bf16x2(d0, d1);
           }
-          const uint32_t half = (uint32_t)(kc >> 1) * kHalf + (uint32_t)r * 128;
+          tmem_st16(lane_base + c * 16, pp);           // over S^T columns already read
+          tmem_st16(lane_base + 128 + c * 16, pd);     // over dP^T columns already read
+          const uint32_t half = (uint32_t)(c >> 1) * kHalf + (uint32_t)r * 128;
 #pragma unroll
           for (int c4 = 0; c4 < 4; ++c4) {
-            const uint32_t chunk = (uint32_t)((kc & 1) * 4 + c4);
+            const uint32_t chunk = (uint32_t)((c & 1) * 4 + c4);
             const uint32_t off = half + ((chunk ^ (uint32_t)(r & 7)) << 4);
-            st_shared_v4(sP + off, pp[c4 * 4], pp[c4 * 4 + 1], pp[c4 * 4 + 2], pp[c4 * 4 + 3]);
             st_shared_v4(sDS + off, pd[c4 * 4], pd[c4 * 4 + 1], pd[c4 * 4 + 2], pd[c4 * 4 + 3]);
           }
         }
+        tmem_st_wait();
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(&bars->pds);
+        mbar_arrive(&bars->meta_free);                 // this thread is done with the row data
         if (!mbar_wait_warp(&bars->dq, (uint32_t)n & 1)) { ok = false; break; }
         tc_fence_after();
-        // this row's dQ partial (bf16), 32-byte stores
+        // row r's dQ partial (lane r of the dQ accumulator), bf16, 32-byte stores
         const int64_t prow = ((int64_t)(id.b * g.hkv + id.gg)) * g.slab + (t - g.t_base);
         __nv_bfloat16* dst = dq_part + ((prow * g.kslots + pslot) * G + h) * kD;
 #pragma unroll 1
@@ -627,7 +696,9 @@ cudaError_t run_bwd(const Shape& s, const BGeom& g, const CUtensorMap& mk, const
                     const CUtensorMap& mq, const CUtensorMap& mdo, const int32_t* idx,
                     const float* lse, float* dq, float* dk, float* dv, char* ws, const BLayout& L,
                     int* err, cudaStream_t st) {
-  const size_t smem = 1024 + 6 * (size_t)kTile + sizeof(BBars);
+  const size_t smem = 1024 + 7 * (size_t)kTile + kRowsT * (4 + 4 + 1) + sizeof(BBars);
+  static_assert(1024 + 7 * (size_t)kTile + kRowsT * (4 + 4 + 1) + sizeof(BBars) <= 232448,
+                "backward tile kernel exceeds 227 KB of shared memory");
   cudaError_t e = cudaFuncSetAttribute(attn_bwd_tiles_kernel<G>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
