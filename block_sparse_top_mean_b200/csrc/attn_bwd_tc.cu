@@ -214,9 +214,9 @@ __global__ void bwd_dot_kernel(const __nv_bfloat16* __restrict__ dO,
 }
 
 // ------------------------------------------------------------------ the tile kernel
-constexpr int kBwdThreads = 192;      // warps 0-3 rows (softmax, epilogues), 4 MMA, 5 copies
-constexpr int kIssuer = 4;
-constexpr int kGather = 5;
+constexpr int kBwdThreads = 320;      // warps 0-7 rows (softmax, epilogues), 8 MMA, 9 copies
+constexpr int kIssuer = 8;
+constexpr int kGather = 9;
 
 struct __align__(8) BBars {
   uint64_t kv_full, q_full[2], q_empty[2], sdp, pds, dq, s_free, acc_empty, meta_full, meta_free;
@@ -280,12 +280,12 @@ attn_bwd_tiles_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
       mbar_init(&bars->q_empty[st], 1);
     }
     mbar_init(&bars->sdp, 1);
-    mbar_init(&bars->pds, 128);
+    mbar_init(&bars->pds, 256);
     mbar_init(&bars->dq, 1);
-    mbar_init(&bars->s_free, 128);
-    mbar_init(&bars->acc_empty, 128);
-    mbar_init(&bars->meta_full, 128);
-    mbar_init(&bars->meta_free, 128);
+    mbar_init(&bars->s_free, 256);
+    mbar_init(&bars->acc_empty, 256);
+    mbar_init(&bars->meta_full, 128);                 // threads 0-127 publish the row data
+    mbar_init(&bars->meta_free, 256);
     bars->abort = 0;
     fence_mbar_init();
   }
@@ -368,21 +368,15 @@ attn_bwd_tiles_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
           tma_load_2d(od + i * G * 128, &tmDO, &bars->q_full[st], 0, y);
           tma_load_2d(od + kHalf + i * G * 128, &tmDO, &bars->q_full[st], 64, y);
         }
-        // the next tile of the segment: its rows into L2 now, its entries kept for the
-        // next iteration's copies
+        // the next tile of the segment: its entries kept for the next iteration's copies
+        // (an L2 prefetch of its rows was measured 31% slower: the tile kernel is bound by
+        // the rate of small tensor-map operations)
         if (tile + 1 < tb) {
           const int4 tn = tiles[tile + 1];
 #pragma unroll
           for (int u = 0; u < kPerLane; ++u) {
             const int i = lane + u * 32;
-            const int e = (i < kTok && i < tn.z) ? entries[tn.y + i] : -1;
-            ent_next[u] = e;
-            if (e < 0) continue;
-            const int y = (int)(((int64_t)id.b * g.S + (e >> 6)) * g.hq + id.gg * G);
-            tma_prefetch_2d(&tmQ, 0, y);
-            tma_prefetch_2d(&tmQ, 64, y);
-            tma_prefetch_2d(&tmDO, 0, y);
-            tma_prefetch_2d(&tmDO, 64, y);
+            ent_next[u] = (i < kTok && i < tn.z) ? entries[tn.y + i] : -1;
           }
         }
       }
@@ -431,12 +425,16 @@ attn_bwd_tiles_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
           }
           tc_fence_after();
           const uint32_t first = tile == ta ? 1u : 0u;
+          // P^T / dS^T as packed bf16: rows 16 ks.. at column 8 ks, plus 32 for rows 64..127
+          // (each half of the rows is packed into the columns its threads read)
 #pragma unroll
           for (int ks = 0; ks < kRowsT / 16; ++ks)
-            umma_ts(tmem + 256, tmem + 0 + ks * 8, mdo + moff(ks), idTM, (first && ks == 0) ? 0u : 1u);
+            umma_ts(tmem + 256, tmem + 0 + ks * 8 + (ks >= 4 ? 32 : 0), mdo + moff(ks), idTM,
+                    (first && ks == 0) ? 0u : 1u);
 #pragma unroll
           for (int ks = 0; ks < kRowsT / 16; ++ks)
-            umma_ts(tmem + 384, tmem + 128 + ks * 8, mq + moff(ks), idTM, (first && ks == 0) ? 0u : 1u);
+            umma_ts(tmem + 384, tmem + 128 + ks * 8 + (ks >= 4 ? 32 : 0), mq + moff(ks), idTM,
+                    (first && ks == 0) ? 0u : 1u);
           // dQ over S^T's columns: the MMAs of this thread run in issue order, so the dV
           // products above have read P^T from them before these write
 #pragma unroll
@@ -449,11 +447,13 @@ attn_bwd_tiles_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
       if (!ok) fail();
     }
   } else {
-    // ---------------------------------------------------------------- rows (warps 0-3)
-    // Thread r is tile row r for the per-row data and the dQ epilogue, and key r (TMEM
-    // lane r of S^T, dP^T, dV, dK) for the softmax and the dV / dK epilogue.
-    const int r = tid;
-    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    // ---------------------------------------------------------------- rows (warps 0-7)
+    // Thread tid covers tile row r = tid % 128 for the per-row data (threads 0-127 publish
+    // it) and the dQ epilogue (d half hf = tid / 128), and key r (TMEM lane r of S^T, dP^T,
+    // dV, dK) for the softmax over rows [64 hf, 64 hf + 64) and the dV / dK epilogue of
+    // d half hf.  Two threads per lane keep eight warps on the elementwise work.
+    const int r = tid & (kRowsT - 1), hf = tid >> 7;
+    const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const int i_tok = r / G, h = r % G;
     const float c2 = g.scale_log2;
     const uint32_t sDS = smem_u32(DSs);
@@ -465,11 +465,21 @@ attn_bwd_tiles_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
       const SegId id = seg_id(s, g);
       const int64_t kbase = (int64_t)id.j * g.block + (int64_t)id.sub * kSeg;
       const int64_t seg_end = min(min((int64_t)id.j * g.block + g.block, kbase + kSeg), g.S);
+      // row r of a tile: its entry, and its lse and D (loaded one tile ahead)
+      auto row_of = [&](int e, float& lse_o, float& dd_o) {
+        if (e < 0) { lse_o = 0.f; dd_o = 0.f; return; }
+        const int64_t hr = ((int64_t)id.b * g.hq + id.gg * G + h) * g.S + (e >> 6);
+        lse_o = lse[hr] * kLog2e;
+        dd_o = Dd[hr];
+      };
       int4 tl_next = tiles[ta];
       int ent_next = i_tok < tl_next.z ? entries[tl_next.y + i_tok] : -1;
+      float lse_next, dd_next;
+      row_of(hf == 0 ? ent_next : -1, lse_next, dd_next);
       for (int tile = ta; tile < tb; ++tile, ++n) {
         if (__any_sync(0xffffffffu, *abort_flag != 0)) { ok = false; break; }
         const int ent = ent_next;
+        const float lse_r = lse_next, dd_r = dd_next;
         if (tile + 1 < tb) tl_next = tiles[tile + 1];
         const bool valid = ent >= 0;
         const int64_t t = valid ? (ent >> 6) : 0;
@@ -477,44 +487,55 @@ attn_bwd_tiles_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
         int64_t end = seg_end;
         if (valid && t / g.block == id.j) end = min(end, t + 1);     // causal, own block
         const int lim = valid ? (int)max((int64_t)0, end - kbase) : 0;
-        const int64_t hrow = ((int64_t)id.b * g.hq + id.gg * G + h) * g.S + t;
         // row r's data for every key thread, once the previous tile's readers are done
         // with it (bounded mbarrier waits: a warp that gives up cannot strand the others)
-        const float lse_r = valid ? lse[hrow] * kLog2e : 0.f;
-        const float dd_r = valid ? Dd[hrow] : 0.f;
         if (n > 0 && !mbar_wait_warp(&bars->meta_free, (uint32_t)(n - 1) & 1)) { ok = false; break; }
-        m_lse[r] = lse_r;
-        m_dd[r] = dd_r;
-        m_lim[r] = (uint8_t)lim;
-        mbar_arrive(&bars->meta_full);
+        if (hf == 0) {
+          m_lse[r] = lse_r;
+          m_dd[r] = dd_r;
+          m_lim[r] = (uint8_t)lim;
+          mbar_arrive(&bars->meta_full);
+        }
         if (!mbar_wait_warp(&bars->meta_full, (uint32_t)n & 1)) { ok = false; break; }
         if (!mbar_wait_warp(&bars->sdp, (uint32_t)n & 1)) { ok = false; break; }
         tc_fence_after();
-        if (tile + 1 < tb) ent_next = i_tok < tl_next.z ? entries[tl_next.y + i_tok] : -1;
-        // key r: P^T and dS^T over the 128 rows, back into TMEM as bf16 (A operands of dV
-        // and dK) and dS into shared memory ([key][row], A operand of dQ)
+        if (tile + 1 < tb) {
+          ent_next = i_tok < tl_next.z ? entries[tl_next.y + i_tok] : -1;
+          row_of(hf == 0 ? ent_next : -1, lse_next, dd_next);
+        }
+        // key r: P^T and dS^T over rows [64 hf, 64 hf + 64), back into TMEM as bf16 (A
+        // operands of dV and dK), and dS into shared memory ([key][row], A of dQ)
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 2 * hf; c < 2 * hf + 2; ++c) {
           uint32_t sv[32], pv[32];
           tmem_ld32(lane_base + c * 32, sv);
           tmem_ld32(lane_base + 128 + c * 32, pv);
           tmem_ld_wait();
           uint32_t pp[16], pd[16];
 #pragma unroll
-          for (int k = 0; k < 32; k += 2) {
+          for (int k = 0; k < 32; k += 4) {
             const int rr = c * 32 + k;
-            const float p0 = r < m_lim[rr]
-                                 ? fastmath::fast_exp2(__uint_as_float(sv[k]) * c2 - m_lse[rr]) : 0.f;
-            const float p1 = r < m_lim[rr + 1]
-                                 ? fastmath::fast_exp2(__uint_as_float(sv[k + 1]) * c2 - m_lse[rr + 1])
-                                 : 0.f;
-            const float d0 = p0 * (__uint_as_float(pv[k]) - m_dd[rr]) * g.scale;
-            const float d1 = p1 * (__uint_as_float(pv[k + 1]) - m_dd[rr + 1]) * g.scale;
-            pp[k / 2] = pack_bf16x2(p0, p1);
-            pd[k / 2] = pack_bf16x2(d0, d1);
+            const float4 l4 = *reinterpret_cast<const float4*>(m_lse + rr);
+            const float4 d4 = *reinterpret_cast<const float4*>(m_dd + rr);
+            const uint32_t lim4 = *reinterpret_cast<const uint32_t*>(m_lim + rr);
+            const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dvv[4] = {d4.x, d4.y, d4.z, d4.w};
+            float p[4], ds[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int lim_e = (int)((lim4 >> (8 * e)) & 0xffu);
+              p[e] = r < lim_e ? fastmath::fast_exp2(__uint_as_float(sv[k + e]) * c2 - lv[e]) : 0.f;
+              ds[e] = p[e] * (__uint_as_float(pv[k + e]) - dvv[e]) * g.scale;
+            }
+            pp[k / 2] = pack_bf16x2(p[0], p[1]);
+            pp[k / 2 + 1] = pack_bf16x2(p[2], p[3]);
+            pd[k / 2] = pack_bf16x2(ds[0], ds[1]);
+            pd[k / 2 + 1] = pack_bf16x2(ds[2], ds[3]);
           }
-          tmem_st16(lane_base + c * 16, pp);           // over S^T columns already read
-          tmem_st16(lane_base + 128 + c * 16, pd);     // over dP^T columns already read
+          // packed bf16 pairs over S^T / dP^T columns this thread has already read: rows
+          // 32c.. of half 0 at column 16c, of half 1 at 64 + 16(c - 2)
+          const uint32_t colp = (uint32_t)(c * 16 + (c >= 2 ? 32 : 0));
+          tmem_st16(lane_base + colp, pp);
+          tmem_st16(lane_base + 128 + colp, pd);
           const uint32_t half = (uint32_t)(c >> 1) * kHalf + (uint32_t)r * 128;
 #pragma unroll
           for (int c4 = 0; c4 < 4; ++c4) {
@@ -530,11 +551,11 @@ attn_bwd_tiles_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
         mbar_arrive(&bars->meta_free);                 // this thread is done with the row data
         if (!mbar_wait_warp(&bars->dq, (uint32_t)n & 1)) { ok = false; break; }
         tc_fence_after();
-        // row r's dQ partial (lane r of the dQ accumulator), bf16, 32-byte stores
+        // row r's dQ partial, d half hf (lane r of the dQ accumulator), bf16, 32-byte stores
         const int64_t prow = ((int64_t)(id.b * g.hkv + id.gg)) * g.slab + (t - g.t_base);
         __nv_bfloat16* dst = dq_part + ((prow * g.kslots + pslot) * G + h) * kD;
 #pragma unroll 1
-        for (int kc = 0; kc < 4; ++kc) {
+        for (int kc = 2 * hf; kc < 2 * hf + 2; ++kc) {
           uint32_t qv[32];
           tmem_ld32(lane_base + kc * 32, qv);
           tmem_ld_wait();
@@ -551,14 +572,14 @@ attn_bwd_tiles_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
         mbar_arrive(&bars->s_free);
         if (tile == tb - 1) {
           // the segment's dV and dK are complete (the commit covered every earlier MMA):
-          // lane r = key kbase + r, added to the fp32 gradients
+          // lane r = key kbase + r, d half hf, added to the fp32 gradients
           const int64_t key = kbase + r;
           const bool kvalid = key < seg_end;
 #pragma unroll 1
           for (int which = 0; which < 2; ++which) {
             float* outp = (which == 0 ? dv : dk) + (((int64_t)id.b * g.S + key) * g.hkv + id.gg) * kD;
 #pragma unroll 1
-            for (int kc = 0; kc < 4; ++kc) {
+            for (int kc = 2 * hf; kc < 2 * hf + 2; ++kc) {
               uint32_t av[32];
               tmem_ld32(lane_base + 256 + which * 128 + kc * 32, av);
               tmem_ld_wait();
