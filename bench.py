@@ -770,6 +770,21 @@ def bench_docs(w, args, world, rank, local, pool):
     return line
 
 
+E2E_OVERLAP = ("double-buffered: per step H2D of the inputs, the calls and D2H of the "
+               "output on their own streams; step i's D2H overlaps step i+1's H2D and compute")
+
+
+def set_io_of(self, **tensors):
+    """Points a runner's step at other device tensors of the same shapes."""
+    for name, t in tensors.items():
+        setattr(self, name, t)
+        self.ptr[name] = ctypes.c_void_p(t.data_ptr())
+
+
+PrefillRunner.set_io = set_io_of
+DecodeRunner.set_io = set_io_of
+
+
 def timed_steps(r, args, world, local, n_events):
     """W warm-ups, then exactly K steps between barriers and synchronisations, with the
     SM clock sampled meanwhile.  Returns (ms per step max over ranks, per-step phase
@@ -793,30 +808,59 @@ def timed_steps(r, args, world, local, n_events):
     return ms, ev, clk.summary()
 
 
-def e2e_steps(r, args, world, inputs, output):
-    """The same step through the C ABI from pinned HOST buffers: H2D of `inputs`, the
-    calls, D2H of `output`, all inside the device-timed region.  Returns (ms, h2d, d2h)."""
-    hosts = [x.cpu().pin_memory() for x in inputs]
-    ho = torch.empty(output.shape, dtype=output.dtype).pin_memory()
+def e2e_steps(r, args, world, in_names, out_name):
+    """The same step through the C ABI from pinned HOST buffers: every step copies its
+    inputs host -> device, runs the calls and copies its output device -> host, all inside
+    the device-timed region.  Double-buffered over three streams (copies in, compute,
+    copies out) with two device buffer sets, so step i's device -> host copy overlaps
+    step i+1's host -> device copy and compute.  Returns (ms per step, h2d, d2h bytes)."""
+    ins = [getattr(r, n) for n in in_names]
+    out = getattr(r, out_name)
+    hosts = [x.cpu().pin_memory() for x in ins]
+    ho = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
+    sets = [ins + [out], [torch.empty_like(x) for x in ins] + [torch.empty_like(out)]]
+    names = list(in_names) + [out_name]
+    s_cmp = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_cmp = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+    used = [False, False]
 
-    def one():
-        for d_, h_ in zip(inputs, hosts):
-            d_.copy_(h_, non_blocking=True)
+    def one(i):
+        b = i & 1
+        bufs = sets[b]
+        with torch.cuda.stream(s_in):
+            if used[b]:
+                s_in.wait_event(ev_cmp[b])         # step i-2's compute is done with set b
+            for d_, h_ in zip(bufs[:-1], hosts):
+                d_.copy_(h_, non_blocking=True)
+            ev_in[b].record(s_in)
+        s_cmp.wait_event(ev_in[b])
+        if used[b]:
+            s_cmp.wait_event(ev_out[b])            # step i-2's output has left set b
+        r.set_io(**dict(zip(names, bufs)))
         r.step()
-        ho.copy_(output, non_blocking=True)
+        ev_cmp[b].record(s_cmp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_cmp[b])
+            ho[b].copy_(bufs[-1], non_blocking=True)
+            ev_out[b].record(s_out)
+        used[b] = True
 
-    for _ in range(max(1, args.warmup)):
-        one()
+    for i in range(max(1, args.warmup)):
+        one(i)
     torch.cuda.synchronize()
     barrier(world)
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s.record()
-    for _ in range(args.steps):
-        one()
-    e.record()
+    s.record(s_in)
+    for i in range(args.steps):
+        one(i)
+    e.record(s_out)
     torch.cuda.synchronize()
+    r.set_io(**dict(zip(names, sets[0])))
     ms = max_over_ranks(s.elapsed_time(e) / args.steps, world)
-    return ms, sum(x.numel() * x.element_size() for x in hosts), ho.numel() * ho.element_size()
+    return ms, sum(x.numel() * x.element_size() for x in hosts), ho[0].numel() * ho[0].element_size()
 
 
 # DRAM bytes (read + write) of the prefill attention phase per selected (token, group,
@@ -860,10 +904,10 @@ def bench_prefill(w, args, world, rank, local, pool):
             "algorithmic_per_launch": attn_flops, "selected_entries": entries}
     e2e = None
     if not args.no_e2e:
-        ems, h2d, d2h = e2e_steps(r, args, world, [r.q, r.k, r.v], r.o)
+        ems, h2d, d2h = e2e_steps(r, args, world, ["q", "k", "v"], "o")
         e2e = {"value": round(world * (attn_flops + score_flops) / (ems * 1e-3) / 1e12, 3),
                "unit": "TFLOP/s", "ms_per_step": round(ems, 3), "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": d2h}
+               "d2h_bytes_per_step": d2h, "overlap": E2E_OVERLAP}
     cpu = None
     if pool is not None:
         orc = PrefillOracle(pool, w, r.q, r.k, r.v)
@@ -943,9 +987,9 @@ def bench_decode(w, args, world, rank, local, pool):
                   for k, v in phases.items()}
     e2e = None
     if not args.no_e2e:
-        ems, h2d, d2h = e2e_steps(r, args, world, [r.q], r.o)
+        ems, h2d, d2h = e2e_steps(r, args, world, ["q"], "o")
         e2e = {"value": round(ems * 1e3, 1), "unit": "us/step", "ms_per_step": round(ems, 4),
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "overlap": E2E_OVERLAP}
     cpu = None
     if pool is not None:
         t, sample = DecodeOracle(pool, w, r.q, seed=rank).step_seconds(2, 0)
