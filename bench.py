@@ -527,6 +527,14 @@ class PrefillRunner:
             events[3].record()
 
 
+def select_launches(nb: int) -> int:
+    """Own kernels of one selection over an encoded bank of nb blocks: [sample scan,
+    threshold,] hi-plane scan, candidate select or merge, exact rescoring, and the two
+    launches of the exact rescan (which exit at once when every row is certified).  The
+    sample pass runs from 128 chunks of 128 blocks per group."""
+    return 7 if -(-nb // 128) >= 128 else 5
+
+
 class DecodeRunner:
     """Decode of n_query queries against a bank resident in HBM, through the C ABI.  The
     bank's pooled keys and encoded images are built once up front (the offline encoding
@@ -575,9 +583,9 @@ class DecodeRunner:
         self.ptr = {k: P(getattr(self, k)) for k in ("q", "kt", "vt", "bt", "idx", "o", "lse",
                                                      "ws")}
         self.pp = ctypes.byref(self.p)
-        # own kernels per step: sample scan, sample threshold, bank scan, list merge,
-        # attention, combine
-        self.launches_per_step = 6
+        # own kernels per step: the selection's, then attention and split combine
+        self.nb_local = -(-seq_local // w.block)
+        self.launches_per_step = select_launches(self.nb_local) + 2
 
     def step(self, events=None):
         if self.shard is not None:
@@ -953,18 +961,26 @@ def bench_decode(w, args, world, rank, local, pool):
     peaks, peak_src = load_peaks()
     sel_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
     att_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
-    planes_read = float(w.nb * w.hkv * w.d * 4)
+    # what the selection streams: the hi plane, every 8th chunk of it again for the sample
+    # bounds, and the hi + lo rows of 64 candidates per (query, group) for the rescoring
+    nch = -(-w.nb // 128)
+    planes_read = float(w.nb * w.hkv * w.d * 2 + -(-nch // 8) * 128 * w.hkv * w.d * 2 +
+                        w.n_query * w.hkv * 64 * w.d * 2 * 2)
     if world > 1:
         return bench_decode_sharded(w, r, args, world, ms, clocks, peaks, peak_src, work)
     if w.host_bank:
         return bench_decode_host_bank(w, r, args, ms, clocks, work)
     phases = {
         "select": {"ms": sel_ms, "bytes": work["score_bytes"],
-                   "kernel": "msa_decode_select_tiled (sample scan + threshold + full "
-                             "tensor-core scan + list merge)",
-                   # DRAM bytes of its scan kernels in one ncu capture of a 1.2M-token bank
-                   # (sample 10.5 MB + scan 79.5 MB for 18,750 blocks), scaled by blocks
-                   "traffic": (10.52e6 + 79.46e6) * w.nb / 18750},
+                   "kernel": "msa_decode_select_tiled (hi-plane sample scan + threshold + "
+                             "hi-plane filter scan + candidate select + exact rescoring "
+                             "with certificate; the exact rescan launches exit at once)",
+                   # DRAM bytes of its kernels in one ncu capture of this 10M-token bank's
+                   # planes (profiles/decode_bank10m_b64_k32_select_dram.md): the two scans
+                   # (40.69 + 321.94 MB) scale with the bank's blocks, the threshold, select
+                   # and rescoring (1.26 + 2.86 + 17.10 MB) with the 512 (query, group) rows
+                   "traffic": (40.69e6 + 321.94e6) * w.nb / 156250 +
+                              (1.26e6 + 2.86e6 + 17.10e6) * w.n_query * w.hkv / 512},
         "attend": {"ms": att_ms, "bytes": work["attn_bytes"],
                    "kernel": "msa_decode_attn_tiled (streamed attention + split combine)",
                    # the attention kernel's DRAM bytes in the same capture (526.3 MB read,
@@ -976,10 +992,12 @@ def bench_decode(w, args, world, rank, local, pool):
     roof = {"bound": "hbm", "kernel": dom["kernel"], "achieved": round(gbs, 1),
             "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
             "peak_source": f"hbm_gbs of {peak_src}", "traffic": round(dom["traffic"]),
-            "traffic_source": "ncu capture of a 1.2M-token bank, scaled (see profiles/)",
+            "traffic_source": "ncu dram bytes of the selection's kernels on the 10M-token "
+                              "bank's planes (see profiles/)",
             "algorithmic_per_launch": dom["bytes"],
-            "algorithmic_note": "one bf16 plane of the pooled keys; the exact selection "
-                                "streams both the hi and lo planes",
+            "algorithmic_note": "one bf16 plane of the pooled keys: the scan streams the hi "
+                                "plane; the lo plane is read only for each row's 64 "
+                                "candidates",
             "planes_read_bytes": planes_read,
             "planes_read_gbs": round(planes_read / (dom["ms"] * 1e-3) / 1e9, 1)}
     phase_line = {k: {"us": round(v["ms"] * 1e3, 1),
@@ -1038,7 +1056,8 @@ def bench_decode_host_bank(w, r, args, ms, clocks, work):
                              "from host memory per step, over the step time"},
         "staged_blocks_per_step": staged,
         "cpu_baseline": None, "e2e": None,
-        "gpu_launches": 10 * args.steps, "clocks": clocks,
+        # selection, the four staging kernels, attention and split combine
+        "gpu_launches": (select_launches(w.nb) + 6) * args.steps, "clocks": clocks,
         "device_error_bits": r.msa.read_device_error(r.ws),
     }
     del r
@@ -1068,7 +1087,8 @@ def bench_decode_sharded(w, r, args, world, ms, clocks, peaks, peak_src, work):
                    "parallelism": f"Memory Parallel: the bank in {world} contiguous block "
                                   f"shards, two NCCL all-gathers per step"},
         "roofline": roof, "cpu_baseline": None, "e2e": None,
-        "gpu_launches": 9 * args.steps, "clocks": clocks,
+        # the shard's selection, key merge, attention, split combine, shard combine
+        "gpu_launches": (select_launches(r.nb_local) + 5) * args.steps, "clocks": clocks,
         "device_error_bits": r.msa.read_device_error(r.ws),
     }
     del r

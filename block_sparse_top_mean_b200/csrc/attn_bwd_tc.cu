@@ -623,7 +623,6 @@ bwd_merge_dq_kernel(const int32_t* __restrict__ idx, const __nv_bfloat16* __rest
   const int64_t row = (int64_t)blockIdx.x * RPC + threadIdx.x / TPR;
   if (row >= n_rows) return;
   const int lt = threadIdx.x % TPR;
-  const int h = lt / 8;
   const int64_t bg = row / g.slab;
   const int t = (int)(g.t_base + row % g.slab);
   if (t >= g.t_end) return;

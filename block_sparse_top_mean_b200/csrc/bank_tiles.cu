@@ -10,6 +10,8 @@
 // single 1-D bulk copy lands it ready for ldmatrix / tcgen05:
 //   K, V tiles   [hkv][ceil(S/64)][2 halves of 64 dims][64 rows][128 B]   16 KB a tile
 //   kbar tiles   [2 planes: hi, lo][hkv][ceil(nb/128)][2 halves][128 rows][128 B]
+//                then bounds [2][hkv] fp32: max_j ||lo_j||_2 and max_j ||hi_j||_2 per KV
+//                head, which bound how far a hi-plane-only score can be from the full one
 // Rows past the end of the bank (keys >= S, blocks >= nb) are zero.
 #include "common.cuh"
 
@@ -50,14 +52,47 @@ cudaError_t launch_image(const void* src, void* dst, int64_t n_rows, int hkv, cu
   return cudaGetLastError();
 }
 
+// One warp per (block, KV head): the Euclidean norms of the block's hi and lo rows,
+// folded into the per-head maxima with an unsigned atomic max (non-negative floats order
+// like their bit patterns; the bounds start at zero).
+__global__ void plane_bounds_kernel(const __nv_bfloat16* __restrict__ hi,
+                                    const __nv_bfloat16* __restrict__ lo, int64_t n_rows,
+                                    int hkv, unsigned* __restrict__ bounds) {
+  const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / 32;
+  const int lane = threadIdx.x % 32;
+  if (w >= n_rows) return;                     // n_rows = nb * hkv, row w = (j, head)
+  const int g = (int)(w % hkv);
+  const uint2 h = *reinterpret_cast<const uint2*>(hi + w * 128 + lane * 4);
+  const uint2 l = *reinterpret_cast<const uint2*>(lo + w * 128 + lane * 4);
+  float sh = 0.f, sl = 0.f;
+  const uint32_t hw[2] = {h.x, h.y}, lw[2] = {l.x, l.y};
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const float a = __uint_as_float(hw[k] << 16), b = __uint_as_float(hw[k] & 0xffff0000u);
+    const float c = __uint_as_float(lw[k] << 16), d = __uint_as_float(lw[k] & 0xffff0000u);
+    sh += a * a + b * b;
+    sl += c * c + d * d;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    sh += __shfl_xor_sync(0xffffffffu, sh, o);
+    sl += __shfl_xor_sync(0xffffffffu, sl, o);
+  }
+  if (lane == 0) {
+    atomicMax(bounds + g, __float_as_uint(sqrtf(sl)));
+    atomicMax(bounds + hkv + g, __float_as_uint(sqrtf(sh)));
+  }
+}
+
 }  // namespace
 
 size_t bank_kv_tiles_bytes(const Shape& s) {
   return (size_t)s.hkv * ((s.seq + 63) / 64) * 16384;
 }
-size_t bank_kbar_tiles_bytes(const Shape& s) {
-  return 2 * (size_t)s.hkv * ((s.nb + 127) / 128) * 32768;
+size_t bank_kbar_planes_bytes(const Shape& s) {
+  return (size_t)s.hkv * ((s.nb + 127) / 128) * 32768;
 }
+size_t bank_kbar_tiles_bytes(const Shape& s) { return 2 * bank_kbar_planes_bytes(s) + 256; }
 
 cudaError_t launch_encode_bank(const Shape& s, const void* k, const void* v, const void* kbar_hi,
                                const void* kbar_lo, void* k_tiles, void* v_tiles,
@@ -69,9 +104,18 @@ cudaError_t launch_encode_bank(const Shape& s, const void* k, const void* v, con
     return e;
   if (kbar_tiles != nullptr) {
     char* hi_img = reinterpret_cast<char*>(kbar_tiles);
-    char* lo_img = hi_img + bank_kbar_tiles_bytes(s) / 2;
+    char* lo_img = hi_img + bank_kbar_planes_bytes(s);
+    char* bounds = lo_img + bank_kbar_planes_bytes(s);
     if ((e = launch_image<128>(kbar_hi, hi_img, s.nb, (int)s.hkv, st)) != cudaSuccess) return e;
     if ((e = launch_image<128>(kbar_lo, lo_img, s.nb, (int)s.hkv, st)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(bounds, 0, 256, st)) != cudaSuccess) return e;
+    const int64_t rows = s.nb * s.hkv;
+    if (rows > 0) {
+      plane_bounds_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(
+          (const __nv_bfloat16*)kbar_hi, (const __nv_bfloat16*)kbar_lo, rows, (int)s.hkv,
+          (unsigned*)bounds);
+    }
+    e = cudaGetLastError();
   }
   return e;
 }

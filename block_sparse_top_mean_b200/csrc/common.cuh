@@ -142,6 +142,11 @@ cudaError_t launch_attn_decode_tc(const Shape& s, int64_t n_query, const void* q
 // 128-byte-swizzled shared-memory layout the decode kernels consume.
 size_t bank_kv_tiles_bytes(const Shape& s);
 size_t bank_kbar_tiles_bytes(const Shape& s);
+// One plane (hi or lo) of the encoded pooled keys; the image is the hi plane, the lo
+// plane, then the selection bounds [2][hkv] fp32 (max ||lo_j||_2, max ||hi_j||_2 over the
+// bank's blocks), padded to 256 bytes.
+size_t bank_kbar_planes_bytes(const Shape& s);
+constexpr int kMaxBoundGroups = 32;      // KV heads the bounds' 256 bytes hold
 cudaError_t launch_encode_bank(const Shape& s, const void* k, const void* v, const void* kbar_hi,
                                const void* kbar_lo, void* k_tiles, void* v_tiles,
                                void* kbar_tiles, cudaStream_t st);

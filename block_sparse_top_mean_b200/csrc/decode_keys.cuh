@@ -42,5 +42,21 @@ __device__ __forceinline__ uint64_t warp_merge_desc(uint64_t y, uint64_t x, int 
   return z;
 }
 
+// Descending bitonic merge of a 64-key list held as (z0, z1): lane l holds ranks l and
+// 32 + l of a bitonic sequence; afterwards they hold ranks l and 32 + l sorted.
+__device__ __forceinline__ void warp_sort_bitonic64(uint64_t& z0, uint64_t& z1, int lane) {
+  const uint64_t a = umax64(z0, z1), b = umin64(z0, z1);
+  z0 = a;
+  z1 = b;
+#pragma unroll
+  for (int j = 16; j > 0; j >>= 1) {
+    const uint64_t p0 = __shfl_xor_sync(0xffffffffu, z0, j);
+    const uint64_t p1 = __shfl_xor_sync(0xffffffffu, z1, j);
+    const bool lower = (lane & j) == 0;
+    z0 = lower ? umax64(z0, p0) : umin64(z0, p0);
+    z1 = lower ? umax64(z1, p1) : umin64(z1, p1);
+  }
+}
+
 }  // namespace keys
 }  // namespace msa

@@ -404,7 +404,7 @@ size_t msa_bank_tiles_bytes(const msa_params* p, int32_t which) {
   Shape s;
   if (check_params(p, true, &s) != MSA_OK) return 0;
   if (which == 0) return msa::bank_kv_tiles_bytes(s);
-  if (which == 1) return msa::bank_kbar_tiles_bytes(s);
+  if (which == 1) return s.hkv <= msa::kMaxBoundGroups ? msa::bank_kbar_tiles_bytes(s) : 0;
   return 0;
 }
 

@@ -253,10 +253,20 @@ MSA_API msa_status msa_decode_fwd(const msa_params* p, int64_t n_query, const vo
  *                     rows past S are zero.  msa_bank_tiles_bytes(p, 0) bytes each.
  *   kbar_tiles        [2][hkv][ceil(nb/128)][2][128][64] bf16: the hi planes, then the lo
  *                     planes of the pooled keys, per KV head in 128-block chunks, the
- *                     same half/row/chunk order and swizzle; rows past nb are zero.
+ *                     same half/row/chunk order and swizzle; rows past nb are zero.  Then
+ *                     256 bytes: fp32 [2][hkv] = max over blocks of ||lo_j||_2, then of
+ *                     ||hi_j||_2, per KV head (the selection's error bound, below).
  *                     msa_bank_tiles_bytes(p, 1) bytes.
- * Supported: bf16, d = 128, block a multiple of 64, G in {1, 2, 4, 8} (else
- * MSA_ERR_UNSUPPORTED).  msa_bank_tiles_bytes returns 0 for invalid shapes or `which`. */
+ * Supported: bf16, d = 128, block a multiple of 64, G in {1, 2, 4, 8}, hkv <= 32 (else
+ * MSA_ERR_UNSUPPORTED).  msa_bank_tiles_bytes returns 0 for invalid shapes or `which`,
+ * and for which = 1 when hkv > 32.
+ * On large encoded banks (at least 1017 chunks of 128 blocks per KV head, about 8.3M
+ * tokens at block 64) the selection reads the lo plane only where it matters: a scan of
+ * the hi plane proposes each row's 64 best blocks, these are scored exactly, and a row is
+ * accepted when the bound max||lo|| * ||q|| on the dropped term proves that no other
+ * block can reach its top k; if any row is not proven (near-equal scores across many
+ * blocks, such as exact ties), the whole bank is scanned exactly as well.  Smaller banks
+ * scan both planes.  The selection is the natural-layout one in every case. */
 MSA_API size_t msa_bank_tiles_bytes(const msa_params* p, int32_t which);
 
 /* Writes the encoded images of a bank in the natural layout (k_bank, v_bank [S, hkv, d];

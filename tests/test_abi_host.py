@@ -138,9 +138,13 @@ def test_encoded_bank_sizes_closed_form(lib):
     p = _p(seq=10_000_000, block=64, topk=32)
     nb = -(-10_000_000 // 64)
     assert lib.msa_bank_tiles_bytes(ctypes.byref(p), 0) == 8 * (-(-10_000_000 // 64)) * 16384
-    assert lib.msa_bank_tiles_bytes(ctypes.byref(p), 1) == 2 * 8 * (-(-nb // 128)) * 32768
+    # hi plane, lo plane, then 256 bytes of per-head bounds (max ||lo_j||, max ||hi_j||)
+    assert lib.msa_bank_tiles_bytes(ctypes.byref(p), 1) == 2 * 8 * (-(-nb // 128)) * 32768 + 256
     assert lib.msa_bank_tiles_bytes(ctypes.byref(p), 2) == 0
     assert lib.msa_bank_tiles_bytes(ctypes.byref(_p(seq=1000, hq=30)), 0) == 0
+    # the bounds hold at most 32 KV heads
+    assert lib.msa_bank_tiles_bytes(ctypes.byref(_p(seq=1000, hq=64, hkv=64)), 1) == 0
+    assert lib.msa_bank_tiles_bytes(ctypes.byref(_p(seq=1000, hq=32, hkv=32)), 1) > 0
 
 
 def test_encoded_bank_entries_check_arguments_before_launch(lib):

@@ -274,11 +274,12 @@ def test_decode_tc_scan(msa, w):
     check_decode(q, kbar_np, kb, vb, w.block, w.topk, w.scale, idx, o, lse, queries=qs)
 
 
-@pytest.mark.parametrize("w", [DECODE_TC[0], DECODE_TC[2], DECODE_TC[3], DECODE_TC[6]],
-                         ids=lambda w: w.name)
+@pytest.mark.parametrize("w", DECODE_TC, ids=lambda w: w.name)
 def test_decode_tiled_bank_matches_natural_layout(msa, w):
-    # the encoded bank changes only where the bytes live: selection and outputs are
-    # bitwise those of the natural layout, which the oracle checks
+    # the encoded bank changes where the bytes live and how the selection gets there (a
+    # certified hi-plane pre-selection, then the three-term scores of the candidates):
+    # selection and outputs are bitwise those of the natural layout, which the oracle
+    # checks
     q, kb, vb = mi.decode_inputs(w, device="cuda")
     _, khi, klo = (t[0] for t in msa.pool_keys(kb[None], w.block, split=True))
     o, lse, idx = msa.decode_fwd(q, None, kb, vb, w.block, w.topk, w.scale, kbar_hi=khi,
@@ -347,7 +348,13 @@ def test_encode_bank_layout(msa):
         assert img[g, t, h, r, c ^ (r % 8), e].item() == kb[tok, g, dim].item()
     assert int(img[0, ntile - 1, 0, (w.seq % 64):].abs().sum().float().item()) == 0   # rows past S
     nch = -(-w.nb // 128)
-    bimg = bt.view(torch.bfloat16).view(2, w.hkv, nch, 2, 128, 8, 8)
+    plane = w.hkv * nch * 2 * 128 * 64 * 2
+    assert bt.numel() == 2 * plane + 256
+    bimg = bt[:2 * plane].view(torch.bfloat16).view(2, w.hkv, nch, 2, 128, 8, 8)
+    # the bounds after the planes: max over blocks of ||lo_j||_2 and ||hi_j||_2 per head
+    bounds = bt[2 * plane:2 * plane + 8 * w.hkv].view(torch.float32).view(2, w.hkv)
+    want = torch.stack([klo.float().norm(dim=-1).amax(dim=0), khi.float().norm(dim=-1).amax(dim=0)])
+    torch.testing.assert_close(bounds, want, rtol=1e-6, atol=0)
     for g, j, dim in [(0, 0, 0), (1, 15, 100)]:
         h, c, e, r = dim // 64, (dim % 64) // 8, dim % 8, j % 128
         assert bimg[0, g, j // 128, h, r, c ^ (r % 8), e].item() == khi[j, g, dim].item()
