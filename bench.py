@@ -1032,6 +1032,76 @@ def bench_decode(w, args, world, rank, local, pool):
     return line
 
 
+class SelectOnlyRunner:
+    """The decode selection alone over a bank's encoded pooled-key image: the bank's keys
+    are generated and pooled in slices, only the routing image is kept (no K/V images)."""
+
+    def __init__(self, w: mi.Workload, seed: int):
+        import block_sparse_top_mean_b200 as msa
+        from block_sparse_top_mean_b200 import _lib
+        self.msa, self.lib, self.w = msa, _lib.load(), w
+        self.q, _, _ = mi.decode_inputs(w, device="cuda", seed=seed, bank=False)
+        khi = torch.empty(w.nb, w.hkv, w.d, dtype=torch.bfloat16, device="cuda")
+        klo = torch.empty_like(khi)
+        step = 1 << 20                                   # tokens per slice (whole blocks)
+        for t0 in range(0, w.seq, step):
+            t1 = min(w.seq, t0 + step)
+            k, _ = mi.decode_bank_rows(w, t0, t1, device="cuda", seed=seed)
+            _, h, l = (t[0] for t in msa.pool_keys(k[None], w.block, split=True))
+            b0 = t0 // w.block
+            khi[b0:b0 + h.shape[0]], klo[b0:b0 + h.shape[0]] = h, l
+            del k, h, l
+        P = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
+        pe = msa.params(batch=1, seq=w.seq, hq=w.hkv, hkv=w.hkv, d=w.d, block=w.block, topk=1,
+                        scale=1.0, dtype=torch.bfloat16)
+        self.bt = torch.empty(self.lib.msa_bank_tiles_bytes(ctypes.byref(pe), 1),
+                              dtype=torch.uint8, device="cuda")
+        _lib.check("msa_encode_bank", self.lib.msa_encode_bank(
+            ctypes.byref(pe), None, None, P(khi), P(klo), None, None, P(self.bt), None))
+        del khi, klo
+        torch.cuda.empty_cache()
+        self.p = msa.params(batch=1, seq=w.seq, hq=w.hq, hkv=w.hkv, d=w.d, block=w.block,
+                            topk=w.topk, scale=w.scale, dtype=self.q.dtype)
+        self.idx = torch.empty(w.n_query, w.hkv, w.topk, dtype=torch.int32, device="cuda")
+        n = self.lib.msa_workspace_bytes(ctypes.byref(self.p), _lib.OP_DECODE, w.n_query)
+        self.ws = torch.zeros(n, dtype=torch.uint8, device="cuda")
+        self.check = _lib.check
+        self.ptr = {k: P(getattr(self, k)) for k in ("q", "bt", "idx", "ws")}
+        self.launches_per_step = select_launches(w.nb)
+
+    def step(self, events=None):
+        s = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+        P, w = self.ptr, self.w
+        if events:
+            events[0].record()
+        self.check("msa_decode_select_tiled", self.lib.msa_decode_select_tiled(
+            ctypes.byref(self.p), w.n_query, P["q"], P["bt"], P["idx"], P["ws"],
+            self.ws.numel(), s))
+        if events:
+            events[1].record()
+
+
+def bench_decode_select_only(w, args, local):
+    r = SelectOnlyRunner(w, seed=0)
+    ms, _, clocks = timed_steps(r, args, 1, local, 2)
+    work = decode_work(w)
+    line = {
+        "metric": "decode selection us/step", "value": round(ms * 1e3, 1), "unit": "us/step",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+        "higher_is_better": False, "scaling": "strong", "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic",
+        "config": {"workload": w.name, "n_query": w.n_query, "bank_tokens": w.seq, "hq": w.hq,
+                   "hkv": w.hkv, "d": w.d, "block": w.block, "topk": w.topk,
+                   "scope": "msa_decode_select_tiled alone (no K/V images)"},
+        "gbs_one_plane": round(work["score_bytes"] / (ms * 1e-3) / 1e9, 1),
+        "gpu_launches": r.launches_per_step * args.steps, "clocks": clocks,
+        "device_error_bits": r.msa.read_device_error(r.ws),
+    }
+    del r
+    torch.cuda.empty_cache()
+    return line
+
+
 def bench_decode_host_bank(w, r, args, ms, clocks, work):
     """The decode line with the bank's K/V in pinned host memory: the step is bound by the
     PCIe transfer of the selected tiles (each selected (group, block) once)."""
@@ -1098,6 +1168,9 @@ def bench_decode_sharded(w, r, args, world, ms, clocks, peaks, peak_src, work):
 
 def bench_one(name, args, world, rank, local, pool):
     w = workload_of(name, args.seq)
+    if getattr(args, "select_only", False):
+        assert w.kind == "decode" and world == 1, "--select-only: one GPU, a decode workload"
+        return bench_decode_select_only(w, args, local)
     fn = {"prefill": bench_prefill, "decode": bench_decode, "prefill_docs": bench_docs,
           "prefill_bwd": bench_bwd}[w.kind]
     return fn(w, args, world, rank, local, pool)
@@ -1191,6 +1264,10 @@ def main():
     ap.add_argument("--seq", type=int, default=None,
                     help="override the workload's sequence / bank length (small profiling "
                          "captures only; the JSON line then names the changed workload)")
+    ap.add_argument("--select-only", action="store_true",
+                    help="decode workloads: build only the bank's pooled-key image and time "
+                         "the selection alone (a small footprint for profiling captures; "
+                         "the JSON line names it)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     args.default_set = args.workload is None
