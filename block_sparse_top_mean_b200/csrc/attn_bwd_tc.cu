@@ -11,10 +11,10 @@
 // Key-centric, like the forward: the selection is inverted into per-(sequence, group,
 // block, 128-key segment) lists of (token, slot) entries, and one tile = the G heads of
 // 128/G such tokens (128 rows) against the segment's 128 keys.  A CTA owns whole segments
-// (a static round-robin over segments), so dK and dV of a key accumulate in TMEM over all
-// tiles that read it, in the order of the segment's entries, and are written once.  That
-// order is fixed: the fill places entries in a sequence that depends only on idx (one
-// warp per 2048-token range walks its tokens in order), so results are bitwise
+// (dealt out by tile count, bwd_balance_kernel), so dK and dV of a key accumulate in TMEM
+// over all tiles that read it, in the order of the segment's entries, and are written
+// once.  That order is fixed: the fill places entries in a sequence that depends only on
+// idx (one warp per 2048-token range walks its tokens in order), so results are bitwise
 // reproducible.  Per tile:
 //   S = Q K^T, dP = dO V^T        tcgen05, both operands K-major in shared memory
 //   P, dS (bf16, scale folded into dS) written to shared memory by the 128 row threads
@@ -189,6 +189,97 @@ __global__ void bwd_tile_table_kernel(const int* __restrict__ totals, const int*
   tiles[tile] = make_int4((int)lo, seg_off[lo] + k * tpt, cnt, (int)(lo / nseg_per_bg));
 }
 
+// The CTAs' segment lists: every non-empty segment goes to exactly one CTA, which runs
+// all of its tiles (dK and dV of its keys accumulate in that CTA's TMEM).  Segments of at
+// least a quarter of a CTA's fair share of tiles are dealt out first, round-robin; the
+// others fill each CTA up to the fair share in segment order.  Without such segments the
+// plain round-robin over all segments is kept (seg_beg[kMaxBwdCtas] = 1), which measured
+// faster when every segment is small.  The assignment changes neither any result nor its
+// bits: a segment's tiles run in entry order wherever it runs.
+constexpr int kBalThreads = 1024;
+constexpr int kMaxBwdCtas = 1024;
+__global__ void __launch_bounds__(kBalThreads)
+bwd_balance_kernel(const int* __restrict__ tile_off, int64_t nseg, int ncta,
+                   int* __restrict__ seg_list, int* __restrict__ seg_beg) {
+  __shared__ long long s_a[kBalThreads], s_b[kBalThreads];
+  __shared__ long long cap_off[kMaxBwdCtas + 1];
+  __shared__ int load[kMaxBwdCtas], cnt[kMaxBwdCtas], fill[kMaxBwdCtas];
+  const int tid = threadIdx.x;
+  const long long total = tile_off[nseg];
+  const long long fair = (total + ncta - 1) / ncta;
+  const long long big = fair / 4 > 1 ? fair / 4 : 1;
+  for (int c = tid; c < ncta; c += kBalThreads) { load[c] = 0; cnt[c] = 0; fill[c] = 0; }
+  // per-thread contiguous ranges of segments: ranks of big segments, small-tile prefixes
+  const int64_t per = (nseg + kBalThreads - 1) / kBalThreads;
+  const int64_t lo = tid * per, hi = lo + per < nseg ? lo + per : nseg;
+  long long nbig = 0, small = 0;
+  for (int64_t i = lo; i < hi; ++i) {
+    const long long t = tile_off[i + 1] - tile_off[i];
+    if (t >= big) ++nbig; else small += t;
+  }
+  s_a[tid] = nbig;
+  s_b[tid] = small;
+  __syncthreads();
+  for (int off = 1; off < kBalThreads; off <<= 1) {     // inclusive Hillis-Steele scans
+    const long long a = tid >= off ? s_a[tid - off] : 0, b = tid >= off ? s_b[tid - off] : 0;
+    __syncthreads();
+    s_a[tid] += a;
+    s_b[tid] += b;
+    __syncthreads();
+  }
+  const long long big0 = s_a[tid] - nbig, small0 = s_b[tid] - small;
+  const bool round_robin = s_a[kBalThreads - 1] == 0;
+  if (tid == 0) seg_beg[kMaxBwdCtas] = round_robin ? 1 : 0;
+  if (round_robin) return;                             // uniform for the block
+  // big segments round-robin, and the load they put on each CTA
+  long long r = big0;
+  for (int64_t i = lo; i < hi; ++i) {
+    const long long t = tile_off[i + 1] - tile_off[i];
+    if (t >= big) atomicAdd(&load[(int)(r++ % ncta)], (int)t);
+  }
+  __syncthreads();
+  if (tid == 0) {                                      // room left per CTA, as a prefix
+    cap_off[0] = 0;
+    for (int c = 0; c < ncta; ++c) {
+      const long long room = fair - load[c];
+      cap_off[c + 1] = cap_off[c] + (room > 0 ? room : 0);
+    }
+  }
+  __syncthreads();
+  // each segment's CTA (big: its round-robin CTA; small: the CTA whose room covers the
+  // segment's first tile among the small ones)
+  auto owner = [&](int64_t i, long long& rb, long long& ps) -> int {
+    const long long t = tile_off[i + 1] - tile_off[i];
+    if (t >= big) return (int)(rb++ % ncta);
+    int a = 0, b = ncta - 1;                         // last c with cap_off[c] <= ps
+    while (a < b) {
+      const int m = (a + b + 1) / 2;
+      if (cap_off[m] <= ps) a = m; else b = m - 1;
+    }
+    ps += t;
+    return a;
+  };
+  r = big0;
+  long long ps = small0;
+  for (int64_t i = lo; i < hi; ++i)
+    if (tile_off[i + 1] > tile_off[i]) atomicAdd(&cnt[owner(i, r, ps)], 1);
+    else owner(i, r, ps);
+  __syncthreads();
+  if (tid == 0) {
+    int acc = 0;
+    for (int c = 0; c < ncta; ++c) { seg_beg[c] = acc; acc += cnt[c]; }
+    seg_beg[ncta] = acc;
+  }
+  __syncthreads();
+  r = big0;
+  ps = small0;
+  for (int64_t i = lo; i < hi; ++i) {
+    const bool nonempty = tile_off[i + 1] > tile_off[i];
+    const int c = owner(i, r, ps);
+    if (nonempty) seg_list[seg_beg[c] + atomicAdd(&fill[c], 1)] = (int)i;
+  }
+}
+
 // D[b, h, t] = dO[b, t, h, :] . O[b, t, h, :] in fp32; 16 threads per row.
 __global__ void bwd_dot_kernel(const __nv_bfloat16* __restrict__ dO,
                                const __nv_bfloat16* __restrict__ O, float* __restrict__ Dd,
@@ -252,9 +343,15 @@ attn_bwd_tiles_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
                       const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmDO, const int4* __restrict__ tiles,
                       const int* __restrict__ tile_off, const int* __restrict__ entries,
+                      const int* __restrict__ seg_list, const int* __restrict__ seg_beg,
                       const float* __restrict__ lse, const float* __restrict__ Dd,
                       __nv_bfloat16* __restrict__ dq_part, float* __restrict__ dk,
                       float* __restrict__ dv, int* err, BGeom g) {
+  // this CTA's segments: the round-robin stride, or its list (bwd_balance_kernel)
+  const bool rr = seg_beg[kMaxBwdCtas] != 0;
+  const int64_t s_first = rr ? (int64_t)blockIdx.x : (int64_t)seg_beg[blockIdx.x];
+  const int64_t s_last = rr ? g.nseg : (int64_t)seg_beg[blockIdx.x + 1];
+  const int64_t s_step = rr ? (int64_t)gridDim.x : 1;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* base = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -309,7 +406,8 @@ attn_bwd_tiles_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
     int n = 0;
     bool stop = false;
     int ent_next[kPerLane];
-    for (int64_t s = blockIdx.x; s < g.nseg && !stop; s += gridDim.x) {
+    for (int64_t si = s_first; si < s_last && !stop; si += s_step) {
+      const int64_t s = rr ? si : seg_list[si];
       const int ta = tile_off[s], tb = tile_off[s + 1];
       if (ta == tb) continue;
       const SegId id = seg_id(s, g);
@@ -401,7 +499,8 @@ attn_bwd_tiles_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
       auto moff = [](int ks) -> uint64_t { return (uint64_t)ks * (2048 >> 4); };  // 16 K-rows
       int n = 0, sc = 0;
       bool ok = true;
-      for (int64_t s = blockIdx.x; s < g.nseg && ok; s += gridDim.x) {
+      for (int64_t si = s_first; si < s_last && ok; si += s_step) {
+        const int64_t s = rr ? si : seg_list[si];
         const int ta = tile_off[s], tb = tile_off[s + 1];
         if (ta == tb) continue;
         if (!mbar_wait(&bars->kv_full, (uint32_t)sc & 1)) { ok = false; break; }
@@ -459,7 +558,8 @@ attn_bwd_tiles_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
     const uint32_t sDS = smem_u32(DSs);
     int n = 0;
     bool ok = true;
-    for (int64_t s = blockIdx.x; s < g.nseg && ok; s += gridDim.x) {
+    for (int64_t si = s_first; si < s_last && ok; si += s_step) {
+      const int64_t s = rr ? si : seg_list[si];
       const int ta = tile_off[s], tb = tile_off[s + 1];
       if (ta == tb) continue;
       const SegId id = seg_id(s, g);
@@ -656,7 +756,8 @@ bwd_merge_dq_kernel(const int32_t* __restrict__ idx, const __nv_bfloat16* __rest
 
 // ------------------------------------------------------------------ host side
 struct BLayout {
-  size_t counts, totals, seg_off, tile_off, n_tiles, entries, tiles, part, dd, total;
+  size_t counts, totals, seg_off, tile_off, n_tiles, entries, tiles, part, dd, seg_list,
+      seg_beg, total;
 };
 
 size_t up256b(size_t x) { return (x + 255) / 256 * 256; }
@@ -693,6 +794,8 @@ BLayout blayout(const Shape& s, int64_t slab) {
   L.tiles = o;    o += up256b((size_t)n_tiles_max * 16);
   L.part = o;     o += up256b((size_t)rows * g.kslots * g.G * kD * 2);
   L.dd = o;       o += up256b((size_t)s.batch * s.hq * s.seq * 4);
+  L.seg_list = o; o += up256b((size_t)g.nseg * 4);
+  L.seg_beg = o;  o += up256b((size_t)(kMaxBwdCtas + 1) * 4);
   L.total = o;
   return L;
 }
@@ -724,9 +827,13 @@ cudaError_t run_bwd(const Shape& s, const BGeom& g, const CUtensorMap& mk, const
   if (e != cudaSuccess) return e;
   int grid = sm_count();
   if (g.nseg < grid) grid = (int)g.nseg;
+  if (grid > kMaxBwdCtas - 1) grid = kMaxBwdCtas - 1;      // seg_beg[kMaxBwdCtas] is the mode
+  bwd_balance_kernel<<<1, kBalThreads, 0, st>>>((const int*)(ws + L.tile_off), g.nseg, grid,
+                                                (int*)(ws + L.seg_list), (int*)(ws + L.seg_beg));
   attn_bwd_tiles_kernel<G><<<grid, kBwdThreads, smem, st>>>(
       mk, mv, mq, mdo, (const int4*)(ws + L.tiles), (const int*)(ws + L.tile_off),
-      (const int*)(ws + L.entries), lse, (const float*)(ws + L.dd),
+      (const int*)(ws + L.entries), (const int*)(ws + L.seg_list),
+      (const int*)(ws + L.seg_beg), lse, (const float*)(ws + L.dd),
       (__nv_bfloat16*)(ws + L.part), dk, dv, err, g);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const int64_t rows = s.batch * s.hkv * g.slab;
