@@ -37,6 +37,7 @@ SIGNATURES = {
     "msa_decode_fwd_static": (c_int32, [c_void_p, c_int64, c_void_p, c_void_p, c_void_p,
                                         c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                         c_void_p, c_void_p]),
+    "msa_decode_static_read_error": (c_int32, [c_void_p, c_void_p]),
     "msa_bank_tiles_bytes": (c_size_t, [c_void_p, c_int32]),
     "msa_encode_bank": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                   c_void_p, c_void_p, c_void_p]),

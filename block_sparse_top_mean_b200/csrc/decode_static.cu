@@ -67,3 +67,11 @@ extern "C" msa_status msa_decode_fwd_static(const msa_params* p, int64_t n_query
   return msa_decode_fwd(p, n_query, q, kbar, kbar_hi, kbar_lo, k_bank, v_bank, idx, o, lse,
                         scratch, kMsaDecodeStaticScratch, stream);
 }
+
+extern "C" msa_status msa_decode_static_read_error(int32_t* bits, msa_stream_t stream) {
+  if (bits == nullptr) return MSA_ERR_INVALID_ARG;
+  void* scratch = nullptr;
+  const msa_status st = scratch_address(&scratch);
+  if (st != MSA_OK) return st;
+  return msa_read_device_error(scratch, bits, stream);
+}

@@ -59,7 +59,7 @@ constexpr int kOwned = kN / kEpiWarps;    // queries per owner warp
 constexpr uint32_t kPlane = 16384;        // 128 rows x 128 B: one plane of a half-chunk
 constexpr uint32_t kStageBytes = 2 * kPlane;
 constexpr uint32_t kQHalf = 8192;         // 64 rows x 128 B: 64 dims of one query plane
-constexpr uint32_t kQBytes = 4 * kQHalf;  // hi (2 halves), lo (2 halves)
+constexpr uint32_t kQBytes = 4 * kQHalf;  // per 64-dim half: hi rows, then lo rows
 
 struct __align__(8) DBars {
   uint64_t full[kStagesMax], empty[kStagesMax], acc_full[kAcc], acc_empty[kAcc], q_full;
@@ -198,8 +198,10 @@ __device__ __forceinline__ void write_query_planes(unsigned char* QI,
       lw[k / 2] = pack_bf16x2(acc8[k] - bf16lo_to_f32(hp), acc8[k + 1] - bf16hi_to_f32(hp));
     }
     const uint32_t off = (uint32_t)n * 128u + ((uint32_t)(cc ^ (n & 7)) << 4);
-    *reinterpret_cast<uint4*>(QI + hf * kQHalf + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-    *reinterpret_cast<uint4*>(QI + (2 + hf) * kQHalf + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    // half hf: the hi plane's 64 rows, then the lo plane's: one 128-row B operand
+    *reinterpret_cast<uint4*>(QI + (2 * hf) * kQHalf + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    *reinterpret_cast<uint4*>(QI + (2 * hf + 1) * kQHalf + off) =
+        make_uint4(lw[0], lw[1], lw[2], lw[3]);
   }
 }
 
@@ -215,6 +217,22 @@ __device__ __forceinline__ uint32_t pass_mask(const uint32_t (&v)[32], const flo
     pm |= (__uint_as_float(v[n4 * 4 + 3]) >= t4.w ? 1u : 0u) << (n4 * 4 + 3);
   }
   return pm;
+}
+
+// This thread's 32 scores of an accumulator (TMEM address `taddr`): HI = the two terms
+// in columns c and c + 64, added in fp32.
+template <bool HI>
+__device__ __forceinline__ void load_scores(uint32_t taddr, uint32_t (&v)[32]) {
+  tmem_ld32(taddr, v);
+  if constexpr (HI) {
+    uint32_t w[32];
+    tmem_ld32(taddr + kN, w);
+    tmem_ld_wait();
+#pragma unroll
+    for (int n = 0; n < 32; ++n) v[n] = __float_as_uint(__uint_as_float(v[n]) + __uint_as_float(w[n]));
+  } else {
+    tmem_ld_wait();
+  }
 }
 
 // v[n] for a warp-uniform n (a select tree: no dynamic register indexing).
@@ -262,6 +280,10 @@ topk_decode_tc_kernel(const __grid_constant__ CUtensorMap tmHi,
   static_assert(!(GMAX && FILTER), "the sample pass keeps group maxima");
   static_assert(!HI || GMAX || FILTER, "the hi-plane scan has no list form");
   constexpr int NST = ring_stages(MODE);                  // ring stages
+  // accumulators: 64 columns (the three-term score), or 128 in the hi-plane modes (the
+  // two terms side by side); all 512 TMEM columns either way
+  constexpr uint32_t ACOLS = HI ? 2 * kN : kN;
+  constexpr int NACC = (int)((kAcc * kN) / ACOLS);
   constexpr uint32_t SB = stage_bytes(MODE);              // bytes per stage
   if (g.run_if != nullptr && *(volatile const int*)g.run_if == 0) return;
   const int64_t total = (int64_t)g.hkv * g.nch;
@@ -345,6 +367,7 @@ topk_decode_tc_kernel(const __grid_constant__ CUtensorMap tmHi,
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16(kM, kN, 0, 0);
+      constexpr uint32_t idesc_hl = idesc_bf16(kM, 2 * kN, 0, 0);   // hi and lo rows at once
       const uint64_t qd = sdesc_sw128(smem_u32(QI), 16, 1024);
       const uint64_t kd0 = sdesc_sw128(smem_u32(KS), 16, 1024);
       int64_t step = 0, tile = 0;
@@ -354,14 +377,14 @@ topk_decode_tc_kernel(const __grid_constant__ CUtensorMap tmHi,
           if (!mbar_wait(&bars->q_full, seg & 1)) { fail(); break; }
           ++seg;
         }
-        const int a = (int)(tile % kAcc);
-        if (tile >= kAcc &&
-            !mbar_wait(&bars->acc_empty[a], (uint32_t)((tile / kAcc) - 1) & 1)) {
+        const int a = (int)(tile % NACC);
+        if (tile >= NACC &&
+            !mbar_wait(&bars->acc_empty[a], (uint32_t)((tile / NACC) - 1) & 1)) {
           fail();
           break;
         }
         tc_fence_after();
-        const uint32_t acc = tmem + a * kN;
+        const uint32_t acc = tmem + a * ACOLS;
         bool ok = true;
         for (int hf = 0; hf < 2; ++hf, ++step) {
           const int st = (int)(step % NST);
@@ -369,14 +392,19 @@ topk_decode_tc_kernel(const __grid_constant__ CUtensorMap tmHi,
           tc_fence_after();
           const uint64_t kh = kd0 + (uint64_t)((st * SB) >> 4);
           const uint64_t kl = kh + (kPlane >> 4);
-          const uint64_t qh = qd + (uint64_t)((hf * kQHalf) >> 4);
-          const uint64_t ql = qd + (uint64_t)(((2 + hf) * kQHalf) >> 4);
+          const uint64_t qh = qd + (uint64_t)((2 * hf * kQHalf) >> 4);
+          const uint64_t ql = qd + (uint64_t)(((2 * hf + 1) * kQHalf) >> 4);
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks) {
             const uint64_t o = (uint64_t)(ks * 2);   // 32 bytes per k-step, in 16-B units
-            umma_ss(acc, kh + o, qh + o, idesc, (hf | ks) ? 1u : 0u);
-            umma_ss(acc, kh + o, ql + o, idesc, 1u);
-            if (!HI) umma_ss(acc, kl + o, qh + o, idesc, 1u);
+            if (HI) {
+              // columns [0, 64): Khi.Qhi, [64, 128): Khi.Qlo (the epilogue adds them)
+              umma_ss(acc, kh + o, qh + o, idesc_hl, (hf | ks) ? 1u : 0u);
+            } else {
+              umma_ss(acc, kh + o, qh + o, idesc, (hf | ks) ? 1u : 0u);
+              umma_ss(acc, kh + o, ql + o, idesc, 1u);
+              umma_ss(acc, kl + o, qh + o, idesc, 1u);
+            }
           }
           umma_commit(&bars->empty[st]);
         }
@@ -414,17 +442,16 @@ topk_decode_tc_kernel(const __grid_constant__ CUtensorMap tmHi,
       const int64_t slot = (int64_t)blockIdx.x - ((int64_t)gg * g.nch) / g.per;
       const int64_t seg0 = ((int64_t)gg * g.ns_max + slot) * g.nq_pad + qt * kN;
       for (; u < ue; ++u, ++tile) {
-        const int a = (int)(tile % kAcc);
+        const int a = (int)(tile % NACC);
         if (!aborted && __any_sync(0xffffffffu, *abort_flag != 0)) aborted = true;
-        if (!aborted && !mbar_wait_warp(&bars->acc_full[a], (uint32_t)(tile / kAcc) & 1)) {
+        if (!aborted && !mbar_wait_warp(&bars->acc_full[a], (uint32_t)(tile / NACC) & 1)) {
           fail();
           aborted = true;
         }
         if (aborted) continue;
         tc_fence_after();
         uint32_t v[32];
-        tmem_ld32(lane_base + a * kN, v);
-        tmem_ld_wait();
+        load_scores<HI>(lane_base + a * ACOLS, v);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->acc_empty[a]);   // the scores are in registers
@@ -481,9 +508,9 @@ topk_decode_tc_kernel(const __grid_constant__ CUtensorMap tmHi,
       asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
 
       for (; u < ue; ++u, ++tile) {
-        const int a = (int)(tile % kAcc);
+        const int a = (int)(tile % NACC);
         if (!aborted && __any_sync(0xffffffffu, *abort_flag != 0)) aborted = true;
-        if (!aborted && !mbar_wait_warp(&bars->acc_full[a], (uint32_t)(tile / kAcc) & 1)) {
+        if (!aborted && !mbar_wait_warp(&bars->acc_full[a], (uint32_t)(tile / NACC) & 1)) {
           fail();
           aborted = true;
         }
@@ -491,8 +518,7 @@ topk_decode_tc_kernel(const __grid_constant__ CUtensorMap tmHi,
           if (!aborted) {
             tc_fence_after();
             uint32_t v[32];
-            tmem_ld32(lane_base + a * kN, v);
-            tmem_ld_wait();
+            load_scores<HI>(lane_base + a * ACOLS, v);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->acc_empty[a]);
@@ -513,7 +539,7 @@ topk_decode_tc_kernel(const __grid_constant__ CUtensorMap tmHi,
         if (!aborted) {
           tc_fence_after();
           uint32_t v[32];
-          tmem_ld32(lane_base + a * kN, v);
+          tmem_ld32(lane_base + a * ACOLS, v);
           tmem_ld_wait();
           const int64_t j = (u % g.nch) * g.stride * kM + quarter * 32 + lane;
           const bool valid = j < nbv;
@@ -538,7 +564,7 @@ topk_decode_tc_kernel(const __grid_constant__ CUtensorMap tmHi,
               const bool pass = (pm >> n) & 1u;
               const uint32_t mn = __ballot_sync(0xffffffffu, pass);
               const int bn = __shfl_sync(0xffffffffu, base, n);
-              const uint32_t sv = tmem_ld1(lane_base + a * kN + n);
+              const uint32_t sv = tmem_ld1(lane_base + a * ACOLS + n);
               tmem_ld_wait();
               if (pass)
                 pend[(size_t)(qh * 32 + n) * kPend + bn + __popc(mn & lt_mask)] =
@@ -877,8 +903,8 @@ rescore_kernel(const unsigned char* __restrict__ ktiles, int64_t nch_full,
     for (int hf = 0; hf < 2; ++hf) {
       const uint64_t kh = ad + (uint64_t)((hf * kPlane) >> 4);
       const uint64_t kl = kh + (uint64_t)((2 * kPlane) >> 4);
-      const uint64_t qh = qd + (uint64_t)((hf * kQHalf) >> 4);
-      const uint64_t ql = qd + (uint64_t)(((2 + hf) * kQHalf) >> 4);
+      const uint64_t qh = qd + (uint64_t)((2 * hf * kQHalf) >> 4);
+      const uint64_t ql = qd + (uint64_t)(((2 * hf + 1) * kQHalf) >> 4);
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks) {
         const uint64_t o = (uint64_t)(ks * 2);

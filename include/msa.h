@@ -374,7 +374,7 @@ MSA_API msa_status msa_decode_fwd_offload(const msa_params* p, int64_t n_query, 
  *   - Checks: every argument is checked first, with msa_decode_fwd's statuses, before
  *     any CUDA call.  Returns MSA_ERR_WORKSPACE, launching nothing, when
  *     msa_workspace_bytes(p, MSA_OP_DECODE, n_query) exceeds the array (64 queries x 32
- *     heads against a 10M-token bank need about 21 MB).
+ *     heads against a 10M-token bank need about 28 MB).
  *   - Set-up: the first call on a device looks up the array's device address with that
  *     device current (cudaGetSymbolAddress) and caches it for the process; make that
  *     first call before any stream capture.  cudaDeviceReset on a device invalidates the
@@ -382,12 +382,20 @@ MSA_API msa_status msa_decode_fwd_offload(const msa_params* p, int64_t n_query, 
  *   - Sharing: every call on a device uses the same array, which keeps the last call's
  *     contents; the call clears what must start at zero.  Calls that overlap on the GPU
  *     (concurrent streams, or several host threads) race on the array: serialise them.
- *   - Device error bits are not reported to the caller (they live in the shared array). */
+ *   - Device error bits: the call returns MSA_OK even when a kernel skipped work (a
+ *     bounded wait ran out, an index out of range); msa_decode_static_read_error reads
+ *     the bits of the last call on the current device. */
 MSA_API msa_status msa_decode_fwd_static(const msa_params* p, int64_t n_query, const void* q,
                                          const float* kbar, const void* kbar_hi,
                                          const void* kbar_lo, const void* k_bank,
                                          const void* v_bank, int32_t* idx, void* o, float* lse,
                                          msa_stream_t stream);
+
+/* The device error word of msa_decode_fwd_static's array on the current device (the last
+ * call's bits: each call clears them first), read after synchronising `stream`; returns
+ * MSA_ERR_DEVICE when any bit is set, else MSA_OK, and MSA_ERR_INVALID_ARG for a null
+ * `bits`.  No other call may be using the array meanwhile. */
+MSA_API msa_status msa_decode_static_read_error(int32_t* bits, msa_stream_t stream);
 
 /* Copies the workspace's device error word to *bits after synchronising `stream`;
  * returns MSA_ERR_DEVICE when any bit is set, else MSA_OK. */

@@ -213,6 +213,8 @@ def test_static_decode_rejects_before_touching_the_device(lib):
     for kw in (dict(d=96), dict(hq=24)):              # G = 3 and d = 96 are unsupported
         bad = _p(seq=10_000, block=64, topk=32, **kw)
         assert st(ctypes.byref(bad), 4, *args, None, None) == _lib.MSA_ERR_UNSUPPORTED
+    # the array's error bits: a null destination is rejected before any CUDA call
+    assert lib.msa_decode_static_read_error(None, None) == _lib.MSA_ERR_INVALID_ARG
 
 
 def test_empty_inputs_are_noops(lib):

@@ -43,13 +43,19 @@ def test_static_scratch_decode_matches_workspace_decode():
         lse = torch.empty(w.n_query, w.hq, dtype=torch.float32, device="cuda")
         idx = torch.empty(w.n_query, w.hkv, w.topk, dtype=torch.int32, device="cuda")
         Pn = lambda t: None if t is None else P(t)  # noqa: E731
+        torch.cuda.synchronize()
+        held = torch.cuda.memory_allocated()
         st = lib.msa_decode_fwd_static(ctypes.byref(p), w.n_query, P(q), P(kbar), Pn(hi), Pn(lo),
                                        P(kb), P(vb), P(idx), P(o), P(lse), stream)
         assert st == _lib.MSA_OK, (call, st)
         torch.cuda.synchronize()
+        assert torch.cuda.memory_allocated() == held, call   # nothing from torch's allocator
         assert torch.equal(idx, idx_ref), call
         assert torch.equal(o, o_ref), call
         assert torch.equal(lse, lse_ref), call
+        bits = ctypes.c_int32(-1)
+        assert lib.msa_decode_static_read_error(ctypes.byref(bits), stream) == _lib.MSA_OK
+        assert bits.value == 0, call
 
 
 def test_static_scratch_rejects_sizes_beyond_the_limit():
