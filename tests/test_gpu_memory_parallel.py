@@ -82,3 +82,37 @@ def test_decode_step_single_rank_is_the_tiled_decode(msa):
     # one shard: the combine only re-normalises the single partial (weight 1)
     assert torch.equal(o, o_ref)
     assert torch.equal(lse, lse_ref)
+
+
+def test_large_shards_take_the_certified_selection(msa):
+    """Two shards of 8.5M tokens each: every shard's selection is the certified hi-plane
+    path (keys written by the rescoring), and the merged selection is still exactly the
+    unsharded one, whose bank (17M tokens) also takes that path."""
+    from block_sparse_top_mean_b200.memory_parallel import BankShard, shard_ranges
+    w = mi.Workload("mp_big", "decode", 1, 17_000_000, 4, 1, 128, 64, 32, "bf16", n_query=8)
+    q, kb, vb = mi.decode_inputs(w, device="cuda", seed=5)
+    _, khi, klo = (t[0] for t in msa.pool_keys(kb[None], w.block, split=True))
+    kt, vt, bt = msa.encode_bank(kb, vb, khi, klo, w.block)
+    del khi, klo
+    o_ref, lse_ref, idx_ref = msa.decode_fwd_tiled(q, bt, kt, vt, w.seq, w.hkv, w.block, w.topk,
+                                                   w.scale)
+    del kt, vt, bt
+    shards = []
+    for begin, count in shard_ranges(w.nb, 2):
+        t0, t1 = begin * w.block, min(w.seq, (begin + count) * w.block)
+        shards.append(BankShard(kb[t0:t1].contiguous(), vb[t0:t1].contiguous(), w.block, begin))
+    keys = torch.stack([msa.decode_select_shard(q, sh.kbar_tiles, sh.seq, sh.hkv, w.block, w.topk,
+                                                sh.block_begin) for sh in shards])
+    o_parts, l_parts = [], []
+    for sh in shards:
+        idx, idx_local = msa.decode_merge_shards(keys, w.hq, w.d, sh.block_begin, sh.block_count)
+        assert torch.equal(idx, idx_ref)
+        o_p, l_p = msa.decode_attn_tiled(q, sh.k_tiles, sh.v_tiles, idx_local, sh.seq, sh.hkv,
+                                         w.block, scale=w.scale)
+        o_parts.append(o_p)
+        l_parts.append(l_p)
+    o, lse = msa.decode_combine_shards(torch.stack(o_parts), torch.stack(l_parts), w.hkv)
+    torch.cuda.synchronize()
+    # the combine re-weights per-shard partials: the one-bank result to the bf16 bars
+    torch.testing.assert_close(o.float(), o_ref.float(), atol=2e-2, rtol=0)
+    torch.testing.assert_close(lse, lse_ref, atol=2e-3, rtol=0)

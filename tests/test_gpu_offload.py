@@ -61,3 +61,21 @@ def test_offload_rejects_pageable_memory_and_ragged_banks(msa):
     st = lib.msa_decode_fwd_offload(ctypes.byref(p), 2, P(q), P(bt), P(kt), P(vt), P(out[0]),
                                     P(out[1]), None, P(ws), ws.numel(), None)
     assert st == _lib.MSA_ERR_UNSUPPORTED
+
+
+def test_offload_of_a_10m_token_bank(msa):
+    # a bank long enough for the certified hi-plane selection, its K/V in host memory
+    w = mi.Workload("off_10m", "decode", 1, 10_000_000, 4, 1, 128, 64, 32, "bf16", n_query=8)
+    q, kb, vb = mi.decode_inputs(w, device="cuda", seed=4)
+    _, khi, klo = (t[0] for t in msa.pool_keys(kb[None], w.block, split=True))
+    kt, vt, bt = msa.encode_bank(kb, vb, khi, klo, w.block)
+    o_ref, lse_ref, idx_ref = msa.decode_fwd_tiled(q, bt, kt, vt, w.seq, w.hkv, w.block, w.topk,
+                                                   w.scale)
+    kt_h, vt_h = kt.cpu().pin_memory(), vt.cpu().pin_memory()
+    del kt, vt
+    o, lse, idx = msa.decode_fwd_offload(q, bt, kt_h, vt_h, w.seq, w.hkv, w.block, w.topk,
+                                         w.scale)
+    torch.cuda.synchronize()
+    assert torch.equal(idx, idx_ref)
+    assert torch.equal(o, o_ref)
+    assert torch.equal(lse, lse_ref)
