@@ -465,11 +465,15 @@ class PrefillRunner:
     rank holds its KV-group slice of the one sequence (contiguous tensors of its heads, as
     a head-sharded QKV projection produces them) and runs the same calls on it."""
 
-    def __init__(self, w: mi.Workload, seed: int, rank: int = 0, world: int = 1):
+    def __init__(self, w: mi.Workload, seed: int, rank: int = 0, world: int = 1,
+                 select_only: bool = False):
         import block_sparse_top_mean_b200 as msa
         from block_sparse_top_mean_b200 import _lib
         self.msa, self.lib = msa, _lib.load()
+        self.select_only = select_only
         q, k, v = mi.prefill_inputs(w, device="cuda", seed=seed)
+        if select_only:
+            v = torch.empty(0, dtype=q.dtype, device=q.device)
         if world > 1:
             wl = kv_group_split(w, rank, world)
             g0, g1 = rank * wl.hkv, (rank + 1) * wl.hkv
@@ -489,10 +493,12 @@ class PrefillRunner:
         self.khi = torch.empty(w.batch, w.nb, w.hkv, w.d, dtype=torch.bfloat16, device=dev)
         self.klo = torch.empty_like(self.khi)
         self.idx = torch.empty(w.batch, w.hkv, w.seq, w.topk, dtype=torch.int32, device=dev)
-        self.o = torch.empty_like(self.q)
-        self.lse = torch.empty(w.batch, w.hq, w.seq, dtype=torch.float32, device=dev)
-        n = max(self.lib.msa_workspace_bytes(ctypes.byref(self.p), _lib.OP_TOPK_SELECT, 0),
-                self.lib.msa_workspace_bytes(ctypes.byref(self.p), _lib.OP_SPARSE_ATTN, 0))
+        self.o = torch.empty(0 if select_only else self.q.numel(), dtype=self.q.dtype, device=dev)
+        self.lse = torch.empty(0 if select_only else w.batch * w.hq * w.seq, dtype=torch.float32,
+                               device=dev)
+        n = self.lib.msa_workspace_bytes(ctypes.byref(self.p), _lib.OP_TOPK_SELECT, 0)
+        if not select_only:
+            n = max(n, self.lib.msa_workspace_bytes(ctypes.byref(self.p), _lib.OP_SPARSE_ATTN, 0))
         self.ws = torch.zeros(n, dtype=torch.uint8, device=dev)
         self.check = _lib.check
         P = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
@@ -502,6 +508,10 @@ class PrefillRunner:
         # own kernels per step (memsets excluded): pool 1; selection: tensor-core pass +
         # exact pass over flagged tiles = 2; attention, per token slab: count, scan, fill,
         # tile table, tiles, merge = 6
+        if select_only:
+            self.n_slabs = 0
+            self.launches_per_step = 3
+            return
         slab = msa.attn_slab_tokens(self.p, _lib.OP_SPARSE_ATTN, n)
         self.n_slabs = -(-w.seq // slab)
         self.launches_per_step = 3 + 6 * self.n_slabs
@@ -520,6 +530,8 @@ class PrefillRunner:
             s))
         if events:
             events[2].record()
+        if self.select_only:
+            return
         self.check("msa_sparse_attn_fwd", lib.msa_sparse_attn_fwd(
             self.pp, P["q"], P["k"], P["v"], P["idx"], P["o"], P["lse"], P["ws"],
             self.ws.numel(), s))
@@ -1081,6 +1093,29 @@ class SelectOnlyRunner:
             events[1].record()
 
 
+def bench_prefill_select_only(w, args, local):
+    """Pooling and selection of a prefill workload alone (no V, O or attention workspace)."""
+    r = PrefillRunner(w, seed=0, select_only=True)
+    ms, ev, clocks = timed_steps(r, args, 1, local, 3)
+    _, score_flops = prefill_flops(w)
+    sel_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    line = {
+        "metric": "prefill selection ms/step", "value": round(sel_ms, 3), "unit": "ms/step",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
+        "higher_is_better": False, "scaling": "strong", "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "seq": w.seq, "hq": w.hq,
+                   "hkv": w.hkv, "d": w.d, "block": w.block, "topk": w.topk,
+                   "scope": "msa_pool_keys + msa_topk_select alone"},
+        "scoring_tflops": round(score_flops / (sel_ms * 1e-3) / 1e12, 2),
+        "gpu_launches": r.launches_per_step * args.steps, "clocks": clocks,
+        "device_error_bits": r.msa.read_device_error(r.ws),
+    }
+    del r
+    torch.cuda.empty_cache()
+    return line
+
+
 def bench_decode_select_only(w, args, local):
     r = SelectOnlyRunner(w, seed=0)
     ms, _, clocks = timed_steps(r, args, 1, local, 2)
@@ -1169,7 +1204,10 @@ def bench_decode_sharded(w, r, args, world, ms, clocks, peaks, peak_src, work):
 def bench_one(name, args, world, rank, local, pool):
     w = workload_of(name, args.seq)
     if getattr(args, "select_only", False):
-        assert w.kind == "decode" and world == 1, "--select-only: one GPU, a decode workload"
+        assert world == 1 and w.kind in ("decode", "prefill"), \
+            "--select-only: one GPU, a decode or prefill workload"
+        if w.kind == "prefill":
+            return bench_prefill_select_only(w, args, local)
         return bench_decode_select_only(w, args, local)
     fn = {"prefill": bench_prefill, "decode": bench_decode, "prefill_docs": bench_docs,
           "prefill_bwd": bench_bwd}[w.kind]
@@ -1265,9 +1303,10 @@ def main():
                     help="override the workload's sequence / bank length (small profiling "
                          "captures only; the JSON line then names the changed workload)")
     ap.add_argument("--select-only", action="store_true",
-                    help="decode workloads: build only the bank's pooled-key image and time "
-                         "the selection alone (a small footprint for profiling captures; "
-                         "the JSON line names it)")
+                    help="decode: build only the bank's pooled-key image and time the "
+                         "selection alone; prefill: pooling and selection without V, O or the "
+                         "attention workspace (small footprints for profiling captures; the "
+                         "JSON line names it)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     args.default_set = args.workload is None
