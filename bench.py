@@ -1265,14 +1265,14 @@ def run_reference(args, world, rank, pool):
         t = statistics.mean(times)
         value, unit, hib, metric = (attn + score) / t / 1e12, "TFLOP/s", True, \
             "sparse-attn prefill TFLOP/s"
-        cfg = {"workload": w.name, "batch_per_gpu": w.batch, "seq": w.seq, "hq": w.hq,
+        cfg = {"workload": w.name, "batch": w.batch, "seq": w.seq, "hq": w.hq,
                "hkv": w.hkv, "d": w.d, "block": w.block, "topk": w.topk,
                "planted_frac": w.planted_frac}
     cfg["parallelism"] = "host oracle, rank 0 only"
     line = {
         "impl": "reference", "metric": metric, "value": value, "unit": unit, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3,
-        "higher_is_better": hib, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "higher_is_better": hib, "scaling": "strong", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": cfg,
         "cpu_baseline": {"value": value, "unit": unit, "cores": pool.n, "kind": "oracle",
                          "sample": sample},
