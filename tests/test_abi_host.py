@@ -31,6 +31,21 @@ def test_header_declares_the_boundary():
         assert n in names
 
 
+def test_header_is_plain_c(tmp_path):
+    """include/msa.h is a C header (no C++ or CUDA types): it compiles as C99 alone."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use_header.c"
+    src.write_text('#include "msa.h"\nint main(void) { msa_params p; (void)p; return 0; }\n')
+    r = subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-I",
+                        os.path.join(ROOT, "include"), "-c", str(src), "-o",
+                        str(tmp_path / "use_header.o")], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+
+
 def test_library_exports_every_declared_symbol(lib):
     names = _declared_symbols()
     assert set(names) == set(_lib.SIGNATURES), "binding and header disagree"
