@@ -102,8 +102,12 @@ __host__ __device__ constexpr bool mode_filter(int m) { return (m & kModeFilter)
 __host__ __device__ constexpr int ring_stages(int m) {
   return mode_filter(m) ? (mode_hi(m) ? kStagesMax : 5) : (mode_hi(m) ? 2 * kStages : kStages);
 }
-__host__ __device__ constexpr uint32_t stage_bytes(int m) { return mode_hi(m) ? kPlane : kStageBytes; }
-__host__ __device__ constexpr size_t pend_bytes(int m) { return mode_filter(m) ? 0 : (size_t)kN * kPend * 8; }
+__host__ __device__ constexpr uint32_t stage_bytes(int m) {
+  return mode_hi(m) ? kPlane : kStageBytes;
+}
+__host__ __device__ constexpr size_t pend_bytes(int m) {
+  return mode_filter(m) ? 0 : (size_t)kN * kPend * 8;
+}
 __host__ __device__ constexpr size_t smem_bytes(int m) {
   return 1024 + kQBytes + (size_t)ring_stages(m) * stage_bytes(m) + pend_bytes(m) +
          (size_t)kN * 8 + sizeof(DBars);
@@ -199,7 +203,8 @@ __device__ __forceinline__ void write_query_planes(unsigned char* QI,
     }
     const uint32_t off = (uint32_t)n * 128u + ((uint32_t)(cc ^ (n & 7)) << 4);
     // half hf: the hi plane's 64 rows, then the lo plane's: one 128-row B operand
-    *reinterpret_cast<uint4*>(QI + (2 * hf) * kQHalf + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    *reinterpret_cast<uint4*>(QI + (2 * hf) * kQHalf + off) =
+        make_uint4(hw[0], hw[1], hw[2], hw[3]);
     *reinterpret_cast<uint4*>(QI + (2 * hf + 1) * kQHalf + off) =
         make_uint4(lw[0], lw[1], lw[2], lw[3]);
   }
@@ -229,7 +234,8 @@ __device__ __forceinline__ void load_scores(uint32_t taddr, uint32_t (&v)[32]) {
     tmem_ld32(taddr + kN, w);
     tmem_ld_wait();
 #pragma unroll
-    for (int n = 0; n < 32; ++n) v[n] = __float_as_uint(__uint_as_float(v[n]) + __uint_as_float(w[n]));
+    for (int n = 0; n < 32; ++n)
+      v[n] = __float_as_uint(__uint_as_float(v[n]) + __uint_as_float(w[n]));
   } else {
     tmem_ld_wait();
   }
@@ -527,7 +533,8 @@ topk_decode_tc_kernel(const __grid_constant__ CUtensorMap tmHi,
             uint32_t mine = 0u;                   // lane n: group max of query 32*qh + n
 #pragma unroll
             for (int n = 0; n < 32; ++n) {
-              const uint32_t m = __reduce_max_sync(0xffffffffu, valid ? score_ord(__uint_as_float(v[n])) : 0u);
+              const uint32_t m =
+                  __reduce_max_sync(0xffffffffu, valid ? score_ord(__uint_as_float(v[n])) : 0u);
               if (lane == n) mine = m;
             }
             const int qn = qh * 32 + lane;
