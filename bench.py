@@ -987,12 +987,13 @@ def bench_decode(w, args, world, rank, local, pool):
                    "kernel": "msa_decode_select_tiled (hi-plane sample scan + threshold + "
                              "hi-plane filter scan + candidate select + exact rescoring "
                              "with certificate; the exact rescan launches exit at once)",
-                   # DRAM bytes of its kernels in one ncu capture of this 10M-token bank's
-                   # planes (profiles/decode_bank10m_b64_k32_select_dram.md): the two scans
-                   # (40.69 + 321.94 MB) scale with the bank's blocks, the threshold, select
-                   # and rescoring (1.26 + 2.86 + 17.10 MB) with the 512 (query, group) rows
-                   "traffic": (40.69e6 + 321.94e6) * w.nb / 156250 +
-                              (1.26e6 + 2.86e6 + 17.10e6) * w.n_query * w.hkv / 512},
+                   # DRAM bytes (read + write) of its kernels in one ncu capture of this
+                   # 10M-token bank's planes (profiles/decode_bank10m_b64_k32_select_dram.md):
+                   # the two scans (40.70 + 322.04 MB) scale with the bank's blocks; the
+                   # threshold, select, rescoring and the two exiting launches (1.26 + 2.83
+                   # + 17.14 + 0.10 MB) with the 512 (query, group) rows
+                   "traffic": (40.70e6 + 322.04e6) * w.nb / 156250 +
+                              (1.26e6 + 2.83e6 + 17.14e6 + 0.10e6) * w.n_query * w.hkv / 512},
         "attend": {"ms": att_ms, "bytes": work["attn_bytes"],
                    "kernel": "msa_decode_attn_tiled (streamed attention + split combine)",
                    # the attention kernel's DRAM bytes in the same capture (526.3 MB read,
