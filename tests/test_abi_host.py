@@ -46,6 +46,23 @@ def test_header_is_plain_c(tmp_path):
     assert r.returncode == 0, r.stderr
 
 
+def test_binding_constants_match_the_header():
+    """Status codes, dtypes, workspace ops and device-error bits: the binding's values are
+    the header's."""
+    src = open(os.path.join(ROOT, "include", "msa.h")).read()
+    enum = {k: int(v) for k, v in re.findall(r"\b(MSA_[A-Z0-9_]+)\s*=\s*(\d+)", src)}
+    defs = {k: int(v, 0) for k, v in re.findall(r"#define\s+(MSA_DEVERR_\w+)\s+(0x[0-9a-fA-F]+)",
+                                                 src)}
+    for name in ("MSA_OK", "MSA_ERR_INVALID_ARG", "MSA_ERR_UNSUPPORTED", "MSA_ERR_WORKSPACE",
+                 "MSA_ERR_CUDA", "MSA_ERR_DEVICE", "MSA_ERR_TIMEOUT", "MSA_F32", "MSA_BF16"):
+        assert getattr(_lib, name) == enum[name], name
+    for name in ("TOPK_SELECT", "SPARSE_ATTN", "PREFILL", "DECODE", "SPARSE_ATTN_MIN",
+                 "PREFILL_MIN", "DECODE_OFFLOAD", "SPARSE_ATTN_BWD", "SPARSE_ATTN_BWD_MIN"):
+        assert getattr(_lib, "OP_" + name) == enum["MSA_OP_" + name], name
+    assert _lib.DEVERR_IDX_RANGE == defs["MSA_DEVERR_IDX_RANGE"]
+    assert _lib.DEVERR_TIMEOUT == defs["MSA_DEVERR_TIMEOUT"]
+
+
 def test_library_exports_every_declared_symbol(lib):
     names = _declared_symbols()
     assert set(names) == set(_lib.SIGNATURES), "binding and header disagree"
